@@ -1,0 +1,251 @@
+"""Pins of the fp64 oracle against values fixed independently of it.
+
+Each test checks the oracle against something other than itself: a
+hand-derived closed form (tests/golden), a float64 library routine on a
+special case that reduces to it, brute force on tiny inputs, or an invariant
+the method guarantees.  Together they are chosen so that a dropped term, a
+wrong sign or index, or a transposed operand in any oracle step fails one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import Inputs, Workload, make_small
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _sig(z):
+    return 1.0 / (1.0 + math.exp(-z))
+
+
+def _ev(expr: str) -> float:
+    return float(eval(expr, {"__builtins__": {}}, {"sig": _sig, "exp": math.exp}))
+
+
+def _bf16(a):
+    return torch.tensor(a, dtype=torch.float32).to(torch.bfloat16)
+
+
+def _fixture_inputs(fx) -> Inputs:
+    wl = Workload("hand", T=fx["T"], d=fx["d"], E=fx["E"], k=fx["k"], F=fx["F"], S=fx["S"])
+    return Inputs(wl, _bf16(fx["x"]), torch.tensor(fx["W_router"], dtype=torch.float32), None,
+                  _bf16(fx["W_gate"]), _bf16(fx["W_up"]), _bf16(fx["W_down"]),
+                  _bf16(fx["Ws_gate"]), _bf16(fx["Ws_up"]), _bf16(fx["Ws_down"]))
+
+
+def test_hand_worked_example():
+    """Every stage of the oracle against the closed forms worked out by hand."""
+    with open(os.path.join(GOLDEN, "hand_worked_T2_d3_E3_k2_F2_S1.json")) as f:
+        fx = json.load(f)
+    inp = _fixture_inputs(fx)
+    out = oracle.forward(inp)
+    ex = fx["expect"]
+    np.testing.assert_array_equal(out["logits"], [[_ev(v) for v in r] for r in ex["logits"]])
+    np.testing.assert_array_equal(out["idx"], ex["idx"])
+    np.testing.assert_allclose(out["w"], [[_ev(v) for v in r] for r in ex["w"]], rtol=1e-14)
+    np.testing.assert_array_equal(out["margin"], [_ev(v) for v in ex["margin"]])
+    for key in ("counts", "offsets", "perm", "pos"):
+        np.testing.assert_array_equal(out[key], ex[key], err_msg=key)
+    np.testing.assert_allclose(out["y"], [[_ev(v) for v in r] for r in ex["y"]],
+                               rtol=1e-14, atol=1e-15)
+    h, y = oracle.expert_one(inp.x[0], inp.W_gate[1], inp.W_up[1], inp.W_down[1])
+    np.testing.assert_allclose(h, [_ev(v) for v in ex["h_token0_e1"]], rtol=1e-14)
+    np.testing.assert_allclose(y, [_ev(v) for v in ex["y_token0_e1"]], rtol=1e-14)
+
+
+def test_router_logits_equal_float64_matmul():
+    inp = make_small(T=37, d=96, E=11, k=3, F=64, S=1, seed=3, bias_scale=0.5)
+    got = oracle.router_logits(inp.x, inp.W_router, inp.bias)
+    ref = (inp.x.double() @ inp.W_router.double().T + inp.bias.double()).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-13, atol=1e-13)
+    got_nb = oracle.router_logits(inp.x, inp.W_router, None)
+    np.testing.assert_allclose(got_nb, (inp.x.double() @ inp.W_router.double().T).numpy(),
+                               rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("E,k", [(1, 1), (5, 2), (16, 4), (64, 4), (64, 8), (9, 9)])
+def test_topk_brute_force_with_ties(E, k):
+    """Top-k equals a full sort by (logit desc, expert asc); ties are frequent here."""
+    rng = np.random.default_rng(E * 100 + k)
+    T = 200
+    logits = rng.integers(-3, 4, size=(T, E)).astype(np.float64) * 0.25  # many exact ties
+    idx, w, margin = oracle.route(logits, k)
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-logits[t, e], e))
+        assert list(idx[t]) == order[:k]
+        if k < E:
+            assert margin[t] == logits[t, order[k - 1]] - logits[t, order[k]]
+        else:
+            assert margin[t] == math.inf
+        sel = logits[t, order[:k]]
+        ref_w = np.exp(sel - sel.max()) / np.exp(sel - sel.max()).sum()  # softmax over the top-k
+        np.testing.assert_allclose(w[t], ref_w, rtol=1e-13)
+
+
+def test_k_equals_E_gives_full_softmax():
+    from scipy.special import softmax
+    rng = np.random.default_rng(1)
+    logits = rng.normal(size=(50, 12))
+    idx, w, margin = oracle.route(logits, 12)
+    p = softmax(logits, axis=1)
+    for t in range(50):
+        np.testing.assert_allclose(w[t], p[t, idx[t]], rtol=1e-13)
+        assert np.all(np.diff(logits[t, idx[t]]) <= 0)
+    assert np.all(np.isinf(margin))
+
+
+def test_gate_weights_properties():
+    inp = make_small(T=300, d=64, E=64, k=8, F=64, S=1, seed=5)
+    logits = oracle.router_logits(inp.x, inp.W_router)
+    idx, w, margin = oracle.route(logits, 8)
+    assert np.all(w >= 0)
+    np.testing.assert_allclose(w.sum(1), 1.0, rtol=1e-14)
+    assert np.all(np.diff(w, axis=1) <= 0)          # non-increasing, like the logits
+    assert np.all(margin >= 0)
+    for t in range(300):
+        assert len(set(idx[t])) == 8
+
+
+def test_pages_example_64_experts_top4():
+    """The explainer's example (section 2.2): 64 experts, K=4 -> 4 active, 60 idle per token."""
+    inp = make_small(T=128, d=64, E=64, k=4, F=64, S=0, seed=7)
+    logits = oracle.router_logits(inp.x, inp.W_router)
+    idx, _, _ = oracle.route(logits, 4)
+    for t in range(128):
+        active = set(idx[t].tolist())
+        assert len(active) == 4 and 64 - len(active) == 60
+    counts, offsets, perm, pos = oracle.dispatch(idx, 64)
+    assert counts.sum() == 128 * 4
+
+
+@pytest.mark.parametrize("T,E,k", [(0, 4, 2), (1, 1, 1), (7, 3, 2), (300, 64, 8), (64, 16, 2)])
+def test_dispatch_against_stable_argsort(T, E, k):
+    rng = np.random.default_rng(T + E)
+    idx = np.array([rng.permutation(E)[:k] for _ in range(T)], np.int32).reshape(T, k)
+    counts, offsets, perm, pos = oracle.dispatch(idx, E)
+    flat = idx.reshape(-1)
+    np.testing.assert_array_equal(counts, np.bincount(flat, minlength=E))
+    np.testing.assert_array_equal(offsets, np.concatenate([[0], np.cumsum(counts)]))
+    np.testing.assert_array_equal(perm, np.argsort(flat, kind="stable"))
+    assert counts.sum() == T * k and offsets[-1] == T * k and np.all(counts <= T)
+    np.testing.assert_array_equal(perm[pos], np.arange(T * k))   # pos o perm = id
+    np.testing.assert_array_equal(np.sort(perm), np.arange(T * k))  # bijection
+    for e in range(E):
+        seg = perm[offsets[e]:offsets[e + 1]]
+        assert np.all(np.diff(seg) > 0) and np.all(flat[seg] == e)
+
+
+def _dense_swiglu_f64(x, Wg, Wu, Wd):
+    """One dense SwiGLU FFN with torch float64 matmuls (the library routine)."""
+    x = x.double()
+    g = x @ Wg.double().T
+    u = x @ Wu.double().T
+    return (torch.nn.functional.silu(g) * u) @ Wd.double().T
+
+
+def test_single_expert_reduces_to_dense_ffn():
+    """E=1, k=1, S=0: the layer is one dense SwiGLU FFN (the dense first layer's form)."""
+    inp = make_small(T=19, d=128, E=1, k=1, F=64, S=0, seed=11)
+    out = oracle.forward(inp)
+    assert np.all(out["idx"] == 0) and np.all(out["w"] == 1.0)
+    ref = _dense_swiglu_f64(inp.x, inp.W_gate[0], inp.W_up[0], inp.W_down[0]).numpy()
+    np.testing.assert_allclose(out["y"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_single_expert_plus_shared_equals_concatenated_ffn():
+    """E=1, k=1, S=1: routed + shared equals one dense FFN of width 2F (weights concatenated)."""
+    inp = make_small(T=13, d=64, E=1, k=1, F=64, S=1, seed=12)
+    out = oracle.forward(inp)
+    Wg = torch.cat([inp.W_gate[0], inp.Ws_gate[0]], 0)
+    Wu = torch.cat([inp.W_up[0], inp.Ws_up[0]], 0)
+    Wd = torch.cat([inp.W_down[0], inp.Ws_down[0]], 1)
+    ref = _dense_swiglu_f64(inp.x, Wg, Wu, Wd).numpy()
+    np.testing.assert_allclose(out["y"], ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed,S", [(21, 1), (22, 0), (23, 2)])
+def test_brute_force_all_experts_masked(seed, S):
+    """Running every expert on every token and masking to the top-k gates gives the same y."""
+    inp = make_small(T=24, d=64, E=6, k=3, F=64, S=S, seed=seed, bias_scale=0.3)
+    out = oracle.forward(inp)
+    x = inp.x.double()
+    logits = x @ inp.W_router.double().T + inp.bias.double()
+    p = torch.softmax(logits, dim=1)
+    mask = torch.zeros_like(p)
+    top = torch.tensor(out["idx"], dtype=torch.long)
+    mask.scatter_(1, top, 1.0)
+    gates = p * mask
+    gates = gates / gates.sum(1, keepdim=True)
+    ref = torch.zeros(inp.wl.T, inp.wl.d, dtype=torch.float64)
+    for e in range(inp.wl.E):
+        ref += gates[:, e:e + 1] * _dense_swiglu_f64(inp.x, inp.W_gate[e], inp.W_up[e],
+                                                     inp.W_down[e])
+    for s in range(S):
+        ref += _dense_swiglu_f64(inp.x, inp.Ws_gate[s], inp.Ws_up[s], inp.Ws_down[s])
+    # the top-k of the brute force is the full sort of the fp64 library logits
+    for t in range(inp.wl.T):
+        order = sorted(range(inp.wl.E), key=lambda e: (-logits[t, e].item(), e))
+        assert list(out["idx"][t]) == order[:3]
+    np.testing.assert_allclose(out["y"], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_token_independence_and_duplicates():
+    inp = make_small(T=40, d=64, E=8, k=2, F=64, S=1, seed=31)
+    full = oracle.forward(inp)
+    sub = [39, 3, 17, 3]
+    part = oracle.forward(inp, tokens=sub)
+    np.testing.assert_array_equal(part["y"], full["y"][sub])
+    np.testing.assert_array_equal(part["y"][1], part["y"][3])
+
+
+def test_linearity_in_down_projection():
+    inp = make_small(T=16, d=64, E=8, k=2, F=64, S=1, seed=41)
+    y1 = oracle.forward(inp)["y"]
+    inp2 = Inputs(inp.wl, inp.x, inp.W_router, inp.bias, inp.W_gate, inp.W_up, inp.W_down * 2,
+                  inp.Ws_gate, inp.Ws_up, inp.Ws_down * 2)
+    y2 = oracle.forward(inp2)["y"]
+    np.testing.assert_array_equal(y2, 2 * y1)   # powers of two are exact in bf16 and fp64
+
+
+def test_expert_relabelling_permutes_idx_and_keeps_y():
+    inp = make_small(T=32, d=64, E=8, k=3, F=64, S=1, seed=51)
+    out = oracle.forward(inp)
+    pi = torch.randperm(8, generator=torch.Generator().manual_seed(0))  # new label j -> old pi[j]
+    inp2 = Inputs(inp.wl, inp.x, inp.W_router[pi], None, inp.W_gate[pi], inp.W_up[pi],
+                  inp.W_down[pi], inp.Ws_gate, inp.Ws_up, inp.Ws_down)
+    out2 = oracle.forward(inp2)
+    inv = torch.argsort(pi).numpy()   # old label -> new label
+    np.testing.assert_array_equal(out2["idx"], inv[out["idx"]])
+    np.testing.assert_allclose(out2["y"], out["y"], rtol=1e-13, atol=1e-13)
+
+
+def test_override_idx_and_sparse_weight_mapping():
+    inp = make_small(T=10, d=64, E=8, k=2, F=64, S=1, seed=61)
+    out = oracle.forward(inp)
+    # the same routing passed as an override gives the same result
+    out2 = oracle.forward(inp, idx_override=out["idx"])
+    np.testing.assert_allclose(out2["w"], out["w"], rtol=1e-14)
+    np.testing.assert_allclose(out2["y"], out["y"], rtol=1e-13, atol=1e-14)
+    # supplying only the experts the chosen tokens use
+    toks = [2, 5]
+    used = sorted(set(out["idx"][toks].reshape(-1).tolist()))
+    sparse = {"W_gate": {e: inp.W_gate[e] for e in used}, "W_up": {e: inp.W_up[e] for e in used},
+              "W_down": {e: inp.W_down[e] for e in used}}
+    out3 = oracle.forward(inp, tokens=toks, weights=sparse)
+    np.testing.assert_array_equal(out3["y"], out["y"][toks])
+    missing = {"W_gate": {used[0]: inp.W_gate[used[0]]}, "W_up": {}, "W_down": {}}
+    with pytest.raises(ValueError):
+        oracle.forward(inp, tokens=toks, weights=missing)
+
+
+def test_bad_arguments_rejected():
+    with pytest.raises(ValueError):
+        oracle.route(np.zeros((2, 3)), 4)          # k > E
+    with pytest.raises(ValueError):
+        oracle.dispatch(np.array([[0, 5]], np.int32), 4)   # expert id out of range
