@@ -1,0 +1,438 @@
+"""Benchmark of the B200 MoE FFN layer forward (tokens/s), one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+    python bench.py --impl reference ...      # the fp64 CPU oracle arm
+
+A step is one moe_forward over one batch of T tokens: router, dispatch,
+gather, gate/up GEMM + SwiGLU, down GEMM, combine.  With N GPUs (torchrun, one
+process per GPU) every rank runs its own replica of the layer on its own batch
+(the layer has no exchange between token batches): "scaling": "weak", value =
+tokens of all ranks / the slowest rank's time.
+
+Timing: W untimed warm-up steps, then exactly K steps.  Before each step a
+1 GB buffer (eight times L2) is written on the same stream, outside the timed
+interval, so every step starts with a cold L2; each step is bracketed by CUDA
+events on the launching stream; a barrier and synchronisation bracket the
+timed loop; the per-rank total is max-reduced over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, Workload, make_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "decode"
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clocks_setting": 0x100,
+    }
+
+    def __init__(self, device: torch.device, period_s: float = 0.01):
+        self.period = period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            p = torch.cuda.get_device_properties(device)
+            try:   # NVML indices ignore CUDA_VISIBLE_DEVICES: find the GPU by its PCI address
+                bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device.index or 0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - NVML missing
+            self._nvml = None
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self) -> dict:
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML unavailable"}
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (barrier, max over ranks); no collective on the data path
+# ----------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, local, world
+
+
+def init_dist(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend=backend,
+                                             timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# algorithmic work of one forward (counts only touched expert weights, W_r, x, y)
+# ----------------------------------------------------------------------------
+def algorithmic_work(wl: Workload, counts: np.ndarray) -> dict:
+    touched = int((counts > 0).sum())
+    per_expert_w = 3 * wl.F * wl.d * 2
+    w_bytes = (touched + wl.S) * per_expert_w
+    rows = wl.T * wl.k + wl.S * wl.T
+    gate_up_bytes = (touched + wl.S) * 2 * wl.F * wl.d * 2
+    down_bytes = (touched + wl.S) * wl.F * wl.d * 2
+    return {
+        "touched_experts": touched,
+        "layer_bytes": w_bytes + wl.E * wl.d * 4 + 2 * wl.T * wl.d * 2,
+        "expert_flops": 6 * wl.d * wl.F * rows,
+        "router_flops": 2 * wl.T * wl.d * wl.E,
+        "gate_up_bytes": gate_up_bytes,
+        "gate_up_flops": 4 * wl.d * wl.F * rows,
+        "down_bytes": down_bytes,
+        "down_flops": 2 * wl.d * wl.F * rows,
+    }
+
+
+def hbm_bound(wl: Workload, work: dict, peaks: dict) -> bool:
+    """Arithmetic intensity of the gate/up GEMM against the machine balance."""
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    return work["gate_up_flops"] / work["gate_up_bytes"] < ridge
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+def run_ours(args, rank, local, world):
+    import mixture_experts_layer_47_b200 as moe
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = WORKLOADS[args.workload]
+    inp = make_inputs(wl, device=device)
+    if world > 1 and rank > 0:
+        # every rank holds the same weights (one replica each) and its own batch of tokens
+        g = torch.Generator().manual_seed(wl.seed + 1000 * rank)
+        inp.x = torch.randn(wl.T, wl.d, generator=g).to(torch.bfloat16).to(device)
+    h = moe.moe_create(wl.d, wl.E, wl.k, wl.F, wl.S)
+    ws = torch.empty(moe.moe_workspace_size(h, wl.T), dtype=torch.uint8, device=device)
+    y = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=device)
+    # 1 GB: eight times L2, and long enough (~0.2 ms) for the host to queue the whole
+    # step behind it, so no launch latency falls inside the timed interval
+    flush = torch.empty(1 << 30, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    weights = (inp.W_gate, inp.W_up, inp.W_down, inp.Ws_gate, inp.Ws_up, inp.Ws_down)
+
+    stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_STAGE_EVENTS)]
+    for ev in stage_ev:
+        ev.record(stream)
+    moe.moe_set_stage_events(h, stage_ev)
+
+    def step():
+        moe.moe_forward(h, inp.x, inp.W_router, inp.bias, *weights, y, ws, stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize(device)
+    st, detail = moe.moe_device_status(h, wl.T, ws, stream)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status {st} ({detail:#x}) after warm-up")
+    counts = moe.workspace_views(h, wl.T, ws)["counts"].cpu().numpy()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stage_ms = np.zeros((args.steps, moe.MOE_STAGE_EVENTS - 1))
+    barrier(world)
+    torch.cuda.synchronize(device)
+    with ClockSampler(device) as clocks:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)      # cold L2 for every step, outside the timed interval
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+            ends[i].synchronize()
+            for j in range(moe.MOE_STAGE_EVENTS - 1):
+                stage_ms[i, j] = stage_ev[j].elapsed_time(stage_ev[j + 1])
+        torch.cuda.synchronize(device)
+    barrier(world)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms), world, device)
+    ms_per_step = total_ms / args.steps
+    tokens_all = wl.T * world * args.steps
+    value = tokens_all / (total_ms / 1e3)
+    st, detail = moe.moe_device_status(h, wl.T, ws, stream)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status {st} ({detail:#x}) after the timed loop")
+
+    # ---- end to end: pinned host x in, host y out, through moe_forward_host ----
+    x_host = inp.x.cpu().pin_memory()
+    y_host = torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory()
+    moe.moe_set_stage_events(h, None)
+    for _ in range(max(1, args.warmup)):
+        moe.moe_forward_host(h, x_host, inp.W_router, inp.bias, *weights, y_host, ws, stream)
+    torch.cuda.synchronize(device)
+    barrier(world)
+    e2e_ms = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        torch.cuda.synchronize(device)
+        t0 = time.perf_counter()
+        moe.moe_forward_host(h, x_host, inp.W_router, inp.bias, *weights, y_host, ws, stream)
+        stream.synchronize()
+        e2e_ms.append((time.perf_counter() - t0) * 1e3)
+    barrier(world)
+    e2e_total = max_over_ranks(sum(e2e_ms), world, device)
+    e2e_value = tokens_all / (e2e_total / 1e3)
+
+    # ---- roofline of the dominant kernel, from the live stage events ----
+    peaks = load_peaks()
+    work = algorithmic_work(wl, counts)
+    names = moe.STAGE_NAMES
+    stage_mean = {n: float(stage_ms[:, j].mean()) for j, n in enumerate(names)}
+    dominant = max(("gate_up_gemm", "down_gemm"), key=lambda n: stage_mean[n])
+    dom_ms = stage_mean[dominant]
+    key = "gate_up" if dominant == "gate_up_gemm" else "down"
+    if hbm_bound(wl, work, peaks):
+        achieved = work[key + "_bytes"] / (dom_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4)}
+    else:
+        achieved = work[key + "_flops"] / (dom_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4)}
+    roof.update({"kernel": dominant, "traffic": None, "peak_source": peaks["source"],
+                 "algorithmic_per_launch": work[key + ("_bytes" if roof["bound"] == "hbm"
+                                                       else "_flops")],
+                 "launch_ms": round(dom_ms, 4)})
+    layer = {
+        "tflops": round((work["expert_flops"] + work["router_flops"]) / (ms_per_step / 1e3)
+                        / 1e12, 2),
+        "gbs": round(work["layer_bytes"] / (ms_per_step / 1e3) / 1e9, 1),
+        "touched_experts": work["touched_experts"],
+        "hbm_frac": round(work["layer_bytes"] / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+        "tensor_frac": round(work["expert_flops"] / (ms_per_step / 1e3) / 1e12
+                             / peaks["bf16_tflops"], 4),
+        "stage_ms": {n: round(v, 4) for n, v in stage_mean.items()},
+        "max_expert_rows": int(counts.max()), "min_expert_rows": int(counts.min()),
+    }
+
+    out = {
+        "metric": "MoE-layer tokens/s", "value": round(value, 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, random-init weights)",
+        "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d, "n_experts": wl.E,
+                   "top_k": wl.k, "d_ff": wl.F, "n_shared": wl.S, "router": wl.router,
+                   "zipf_s": wl.zipf_s, "global_batch": wl.T * world,
+                   "parallelism": f"replicas{world}",
+                   "l2": "flushed before every step (1 GB write, outside the timed interval)"},
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": wl.T * wl.d * 2, "d2h_bytes_per_step": wl.T * wl.d * 2,
+                "api": "moe_forward_host (pinned host x in, host y out)"},
+        "gpu_launches": 9 * args.steps,
+        "roofline": roof,
+        "layer": layer,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(inp, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    moe.moe_set_stage_events(h, None)
+
+
+# ----------------------------------------------------------------------------
+# the fp64 oracle on the host cores (CPU baseline and reference arm)
+# ----------------------------------------------------------------------------
+def _oracle_sample(inp, tokens: np.ndarray):
+    """Host copies the oracle needs for these tokens: x, router, bias, used experts."""
+    import oracle
+    x = inp.x.cpu()
+    Wr = inp.W_router.cpu()
+    b = None if inp.bias is None else inp.bias.cpu()
+    logits = oracle.router_logits(x[tokens], Wr, b)
+    idx, _, _ = oracle.route(logits, inp.wl.k)
+    used = sorted(set(idx.reshape(-1).tolist()))
+    W = {"W_gate": {e: inp.W_gate[e].cpu() for e in used},
+         "W_up": {e: inp.W_up[e].cpu() for e in used},
+         "W_down": {e: inp.W_down[e].cpu() for e in used},
+         "Ws_gate": inp.Ws_gate.cpu(), "Ws_up": inp.Ws_up.cpu(), "Ws_down": inp.Ws_down.cpu()}
+    return x[tokens].contiguous(), Wr, b, W
+
+
+def _oracle_pass(x, Wr, b, W, wl) -> None:
+    """One oracle forward of the sampled tokens: route, dispatch, experts, combine."""
+    import oracle
+    logits = oracle.router_logits(x, Wr, b)
+    idx, w, _ = oracle.route(logits, wl.k)
+    oracle.dispatch(idx, wl.E)
+    oracle.moe_ffn_tokens(x, idx, w, W["W_gate"], W["W_up"], W["W_down"], W["Ws_gate"],
+                          W["Ws_up"], W["Ws_down"], None, E=wl.E, F=wl.F, S=wl.S)
+
+
+def _sample_tokens(wl: Workload) -> np.ndarray:
+    n = min(wl.T, 16)
+    return np.unique(np.linspace(0, wl.T - 1, n).round().astype(np.int64))
+
+
+def cpu_baseline(inp, seconds: float) -> dict:
+    import oracle
+    wl = inp.wl
+    tokens = _sample_tokens(wl)
+    x, Wr, b, W = _oracle_sample(inp, tokens)
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        _oracle_pass(x, Wr, b, W, wl)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or passes >= 1000:
+            break
+    return {"value": round(passes * len(tokens) / el, 3), "unit": "tokens/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(tokens)} of the {wl.T} tokens (evenly spaced) through the whole "
+                      f"fp64 layer, {passes} passes in {el:.1f} s"}
+
+
+def run_reference(args, rank, local, world):
+    if rank != 0:
+        return
+    import oracle
+    wl = WORKLOADS[args.workload]
+    device = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    inp = make_inputs(wl, device=device)
+    tokens = _sample_tokens(wl)
+    x, Wr, b, W = _oracle_sample(inp, tokens)
+    for _ in range(args.warmup):
+        _oracle_pass(x, Wr, b, W, wl)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_pass(x, Wr, b, W, wl)
+    el = time.perf_counter() - t0
+    value = args.steps * len(tokens) / el
+    sample = (f"each step: {len(tokens)} of the {wl.T} tokens (evenly spaced) through the "
+              f"whole fp64 layer")
+    out = {
+        "impl": "reference", "metric": "MoE-layer tokens/s", "value": round(value, 3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, random-init weights)",
+        "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d, "n_experts": wl.E,
+                   "top_k": wl.k, "d_ff": wl.F, "n_shared": wl.S, "global_batch": wl.T,
+                   "parallelism": "cpu oracle"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s",
+                         "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("at least 3 warm-up steps are required")
+    rank, local, world = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, local, world)   # rank 0 only; no process group needed
+        return
+    init_dist(world, "nccl")
+    try:
+        run_ours(args, rank, local, world)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

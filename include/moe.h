@@ -1,0 +1,216 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) forward pass of one mixture-of-experts
+ * FFN layer of the Hy4-preview shape.
+ *
+ * The layer, as the pages state it (m.xxqk.cn Hy4-preview MoE explainer,
+ * section 2.1 "FFN split" and section 2.2 "router mechanism"; ZAKER Hy4 Preview
+ * release news, MoE paragraph): a router scores every token against every
+ * routed expert and keeps the top-k; the tokens are grouped per expert; every
+ * chosen expert and every always-on shared expert runs its FFN on the token;
+ * the results are merged with the gate weights into the layer output.
+ * Readings where the pages are silent (applied identically by the CPU
+ * oracle): softmax gate over the router logits, top-k gate values
+ * renormalised to sum 1 (equal to a softmax over the k selected logits),
+ * ties broken toward the lower expert index, SwiGLU experts without bias
+ * y = W_down (silu(W_gate x) * (W_up x)), shared experts added with weight 1,
+ * no capacity limit (dropless).
+ *
+ * Conventions for every call below.
+ *  - Pointers named x, W_*, y, Y, topk_*, counts, offsets, perm, pos,
+ *    workspace are DEVICE pointers on the current CUDA device, except where a
+ *    parameter name ends in _host.  The caller allocates and owns all of
+ *    them; the library keeps no pointer after a call returns.
+ *  - bf16 tensors are passed as uint16_t bit patterns.  All matrices are
+ *    row-major and C-contiguous.  Every device pointer must be 16-byte
+ *    aligned.
+ *  - stream is a cudaStream_t (NULL = the legacy default stream).  Every call
+ *    is asynchronous on it: inputs must stay valid, and outputs must not be
+ *    read, until the stream reaches the call.
+ *  - Errors found on the host are returned before anything is enqueued.
+ *    Errors found on the device (an expert index outside [0, E) given to
+ *    moe_dispatch, a bounded wait inside a kernel that expired) are recorded
+ *    in the workspace's status word; read it with moe_device_status().
+ *    No call traps the GPU.
+ *  - T == 0 is a no-op that returns MOE_OK.
+ *  - Results are deterministic: the same inputs give bit-identical outputs
+ *    (no floating-point atomics).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_ctx *moe_handle;
+typedef int moe_status;
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG 1  /* null pointer, negative size, k < 1 or k > E, ...  */
+#define MOE_ERR_UNSUPPORTED 2  /* shape outside the supported envelope, not sm_100  */
+#define MOE_ERR_WORKSPACE 3    /* workspace too small                                */
+#define MOE_ERR_CUDA 4         /* a CUDA runtime call or kernel launch failed        */
+#define MOE_ERR_TIMEOUT 5      /* a bounded device wait expired (moe_device_status)  */
+#define MOE_ERR_BAD_INDEX 6    /* an expert index outside [0, E) reached the device  */
+#define MOE_ERR_ALIGNMENT 7    /* a device pointer is not 16-byte aligned            */
+
+/* Device status words written into the workspace (see moe_device_status). */
+#define MOE_DEVICE_OK 0
+
+/*
+ * Create a layer context.  d_model = hidden size, n_experts = E routed
+ * experts, top_k = k experts per token, d_ff = F expert width, n_shared = S
+ * always-on shared experts (Hy4 preview: 6144, 256, 8, 2048 assumed, 1).
+ * Supported envelope: d_model and d_ff multiples of 64 in [64, 65536];
+ * 1 <= E <= 1024; 1 <= k <= min(E, 32); 0 <= S <= 8.  Shapes outside it give
+ * MOE_ERR_UNSUPPORTED, impossible ones MOE_ERR_INVALID_ARG.  No CUDA call is
+ * made here; the device is checked (sm_100 required) at the first launch.
+ */
+moe_status moe_create(int d_model, int n_experts, int top_k, int d_ff, int n_shared,
+                      moe_handle *out);
+
+/* Release a context (NULL is allowed).  Does not synchronise any stream. */
+moe_status moe_destroy(moe_handle h);
+
+/*
+ * Bytes of device workspace that any call below needs for T tokens
+ * (0 when h is NULL or T < 0).  One workspace of this size serves every
+ * call; it holds intermediates only and may be reused across calls that the
+ * stream orders.  At the Hy4 shape and T = 8192 it is about 3 GB.
+ */
+size_t moe_workspace_size(moe_handle h, int T);
+
+/* Offsets (bytes from the workspace pointer) of the intermediates that
+ * moe_forward leaves in the workspace, for inspection after the stream has
+ * reached the call.  The workspace pointer itself need not be aligned: the
+ * library aligns it up to 1024 bytes and 'base' is that adjustment's offset
+ * for a pointer with the given low bits. */
+typedef struct {
+    size_t status;    /* int32 device status word                            */
+    size_t topk_idx;  /* int32 [T][k]                                        */
+    size_t topk_w;    /* fp32  [T][k]                                        */
+    size_t counts;    /* int32 [E]                                           */
+    size_t offsets;   /* int32 [E+1]                                         */
+    size_t perm;      /* int32 [T*k]                                         */
+    size_t pos;       /* int32 [T*k]                                         */
+    size_t h_act;     /* bf16  [T*k + S*T][F]  SwiGLU activations            */
+    size_t y_rows;    /* fp32  [T*k + S*T][d]  per-(slot, expert) outputs    */
+    size_t total;     /* bytes used, including the alignment slack           */
+} moe_workspace_layout;
+moe_status moe_get_workspace_layout(moe_handle h, int T, uintptr_t workspace_addr,
+                                    moe_workspace_layout *out);
+
+/*
+ * Router: score, top-k select and gate (explainer section 2.2).
+ *   logits[t][e] = sum_j x[t][j] * W_router[e][j] + bias[e]     (fp32 FMA on
+ *                  CUDA cores, no TF32; split-K partial sums added in a fixed
+ *                  order)
+ *   topk_idx[t][i] = the i-th largest logit's expert (ties: lower index)
+ *   topk_w[t][i]   = exp(l_i - l_0) / sum_{j<k} exp(l_j - l_0)
+ * x: bf16 [T][d]; W_router: fp32 [E][d]; bias: fp32 [E] or NULL;
+ * topk_idx: int32 [T][k]; topk_w: fp32 [T][k] (outputs).
+ */
+moe_status moe_route(moe_handle h, const uint16_t *x, const float *W_router, const float *bias,
+                     int T, int32_t *topk_idx, float *topk_w, void *workspace,
+                     size_t ws_bytes, void *stream);
+
+/*
+ * Dispatch: group the T*k (token, choice) slots s = t*k + i by expert with a
+ * stable counting sort (per-expert histogram, exclusive scan, permutation).
+ *   counts[e]  = #{s : topk_idx[s] == e}                     int32 [E]
+ *   offsets[e] = sum_{e' < e} counts[e'], offsets[E] = T*k   int32 [E+1]
+ *   perm[p]    = slot at position p; ascending slots within each expert
+ *   pos[s]     = position of slot s (perm[pos[s]] == s)      int32 [T*k] each
+ * Indices outside [0, E) are skipped and flagged MOE_ERR_BAD_INDEX in the
+ * workspace status word.
+ */
+moe_status moe_dispatch(moe_handle h, const int32_t *topk_idx, int T, int32_t *counts,
+                        int32_t *offsets, int32_t *perm, int32_t *pos, void *workspace,
+                        size_t ws_bytes, void *stream);
+
+/*
+ * Expert FFNs (explainer section 2.1: each expert is one FFN sub-network;
+ * ZAKER release news: the shared expert runs on every token).  Rows of Y:
+ *   Y[p]           = FFN_e(x[perm[p] / k])  for p in expert e's segment
+ *                    [offsets[e], offsets[e+1]),
+ *   Y[T*k + s*T+t] = FFN_shared_s(x[t]),
+ *   FFN(x) = W_down (silu(W_gate x) * (W_up x)); bf16 tensor-core GEMMs
+ *   (tcgen05, fp32 accumulation), the activation rounded to bf16 before the
+ *   down projection, Y in fp32.
+ * W_gate, W_up: bf16 [E][F][d]; W_down: bf16 [E][d][F];
+ * Ws_gate, Ws_up: bf16 [S][F][d]; Ws_down: bf16 [S][d][F] (NULL when S == 0);
+ * Y: fp32 [T*k + S*T][d] (output).
+ */
+moe_status moe_expert_ffn(moe_handle h, const uint16_t *x, const int32_t *perm,
+                          const int32_t *offsets, int T, const uint16_t *W_gate,
+                          const uint16_t *W_up, const uint16_t *W_down, const uint16_t *Ws_gate,
+                          const uint16_t *Ws_up, const uint16_t *Ws_down, float *Y,
+                          void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Combine (explainer section 2.2: the chosen experts' results are merged into
+ * the layer output):
+ *   y[t] = sum_{s<S} Y[T*k + s*T + t] + sum_{i<k} topk_w[t][i] * Y[pos[t*k+i]]
+ * in fp32, in exactly that order, rounded once to bf16.
+ * Y: fp32 [T*k + S*T][d]; topk_w: fp32 [T][k]; pos: int32 [T*k];
+ * y: bf16 [T][d] (output).
+ */
+moe_status moe_combine(moe_handle h, const float *Y, const float *topk_w, const int32_t *pos,
+                       int T, uint16_t *y, void *stream);
+
+/*
+ * The whole layer: moe_route, moe_dispatch, moe_expert_ffn and moe_combine
+ * in one call, intermediates kept in the workspace (moe_get_workspace_layout).
+ * Arguments as in those calls; y: bf16 [T][d] (output).
+ */
+moe_status moe_forward(moe_handle h, const uint16_t *x, const float *W_router, const float *bias,
+                       const uint16_t *W_gate, const uint16_t *W_up, const uint16_t *W_down,
+                       const uint16_t *Ws_gate, const uint16_t *Ws_up, const uint16_t *Ws_down,
+                       int T, uint16_t *y, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * moe_forward with the activations in HOST memory: copies x_host (bf16
+ * [T][d]) to the device, runs the layer, copies y back to y_host (bf16
+ * [T][d]), all on the stream; returns once the copies are enqueued (the
+ * caller synchronises the stream before reading y_host).  Host buffers
+ * should be page-locked for the copies to be asynchronous.  Weights and the
+ * workspace are device memory as in moe_forward.
+ */
+moe_status moe_forward_host(moe_handle h, const uint16_t *x_host, const float *W_router,
+                            const float *bias, const uint16_t *W_gate, const uint16_t *W_up,
+                            const uint16_t *W_down, const uint16_t *Ws_gate,
+                            const uint16_t *Ws_up, const uint16_t *Ws_down, int T,
+                            uint16_t *y_host, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronise the stream and read the workspace's device status word, which
+ * the last call on this workspace wrote: MOE_OK, MOE_ERR_TIMEOUT or
+ * MOE_ERR_BAD_INDEX.  *device_detail receives the raw word (0 if none).
+ */
+moe_status moe_device_status(moe_handle h, int T, const void *workspace, void *stream,
+                             int32_t *device_detail);
+
+/*
+ * Profiling hook.  With n_events == MOE_STAGE_EVENTS and events non-NULL,
+ * every later moe_forward / moe_forward_host call on this context records
+ * events[0..6] (cudaEvent_t handles the caller created) on its stream at the
+ * stage boundaries: before the router, after the router, after dispatch,
+ * after the gather, after the gate/up GEMM, after the down GEMM, after the
+ * combine.  The elapsed time between consecutive events is then the device
+ * time of one stage.  events == NULL (n_events == 0) switches it off.  The
+ * context keeps the handles only; the caller keeps the events alive.
+ */
+#define MOE_STAGE_EVENTS 7
+moe_status moe_set_stage_events(moe_handle h, void *const *events, int n_events);
+
+/* Static text for a status code. */
+const char *moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

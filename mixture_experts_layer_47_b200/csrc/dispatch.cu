@@ -1,0 +1,199 @@
+// dispatch.cu -- group the (token, choice) slots by expert on sm_100a.
+//
+// The pages' explainer (m.xxqk.cn Hy4-preview MoE, section 2.2) has the
+// activated experts process the tokens routed to them; grouping the slots
+// s = t*k + i per expert makes each expert's tokens one contiguous segment
+// that a grouped GEMM can read.  The grouping is a stable counting sort,
+// deterministic by construction (no order-dependent atomics):
+//   dispatch_count    per block of 4096 slots, a shared-memory histogram
+//                     (integer atomics: the counts do not depend on order);
+//   dispatch_scan     one CTA: for every expert the exclusive prefix over
+//                     blocks, counts, the exclusive scan over experts
+//                     (offsets), and the grouped GEMM's M-tile schedule;
+//   dispatch_scatter  per block, each warp owns a contiguous run of slots;
+//                     __match_any_sync gives each slot its rank among equal
+//                     experts in the warp; per-warp, per-expert running
+//                     counts make the order ascending in slot index.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kCountThreads = 512;
+constexpr int kScatterWarps = 8;
+constexpr int kScanThreads = 1024;
+constexpr int kTileM = 128;   // rows per grouped-GEMM M tile
+
+__global__ void __launch_bounds__(kCountThreads)
+    dispatch_count_kernel(const int32_t* __restrict__ idx, int n, int E,
+                          int32_t* __restrict__ blk_hist, int* status) {
+  extern __shared__ int32_t hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int beg = blockIdx.x * kDispatchChunk;
+  const int end = min(n, beg + kDispatchChunk);
+  bool bad = false;
+  for (int s = beg + threadIdx.x; s < end; s += blockDim.x) {
+    const int e = idx[s];
+    if (e >= 0 && e < E)
+      atomicAdd(&hist[e], 1);
+    else
+      bad = true;
+  }
+  if (bad) report_error(status, kDevBadIndex, kSiteDispatch);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) blk_hist[size_t(blockIdx.x) * E + e] = hist[e];
+}
+
+// Inclusive block-wide scan of one int per thread (blockDim.x == kScanThreads).
+__device__ int block_inclusive_scan(int v, int* warp_sums) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += o;
+  }
+  if (lane == 31) warp_sums[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += o;
+    }
+    warp_sums[lane] = w;
+  }
+  __syncthreads();
+  const int r = v + (warp > 0 ? warp_sums[warp - 1] : 0);
+  __syncthreads();
+  return r;
+}
+
+// Grouped-GEMM schedule: sched[g] = sum over groups g' < g of ceil(rows_g' / 128),
+// routed groups first (rows = count), then S shared groups of T rows each.
+__device__ void write_schedule(int count, int E, int S, int T, int32_t* sched, int* warp_sums) {
+  const int e = threadIdx.x;
+  const int mt = (e < E) ? (count + kTileM - 1) / kTileM : 0;
+  const int incl = block_inclusive_scan(mt, warp_sums);
+  if (e < E) sched[e] = incl - mt;
+  if (e == E - 1) {
+    const int mts = (T + kTileM - 1) / kTileM;
+    for (int s = 0; s <= S; ++s) sched[E + s] = incl + s * mts;
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+    dispatch_scan_kernel(int32_t* __restrict__ blk_hist, int nblk, int E, int S, int T,
+                         int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                         int32_t* __restrict__ sched) {
+  __shared__ int warp_sums[32];
+  const int e = threadIdx.x;
+  int c = 0;
+  if (e < E) {
+    int run = 0;
+    for (int b = 0; b < nblk; ++b) {
+      const int h = blk_hist[size_t(b) * E + e];
+      blk_hist[size_t(b) * E + e] = run;
+      run += h;
+    }
+    c = run;
+    counts[e] = c;
+  }
+  const int incl = block_inclusive_scan(c, warp_sums);
+  const int excl = incl - c;
+  if (e < E) {
+    offsets[e] = excl;
+    for (int b = 0; b < nblk; ++b) blk_hist[size_t(b) * E + e] += excl;
+  }
+  if (e == E - 1) offsets[E] = incl;
+  write_schedule(c, E, S, T, sched, warp_sums);
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+    schedule_from_offsets_kernel(const int32_t* __restrict__ offsets, int E, int S, int T,
+                                 int32_t* __restrict__ sched) {
+  __shared__ int warp_sums[32];
+  const int e = threadIdx.x;
+  int c = 0;
+  // A group never holds more than T slots (a token picks an expert once).
+  if (e < E) c = min(T, max(0, offsets[e + 1] - offsets[e]));
+  write_schedule(c, E, S, T, sched, warp_sums);
+}
+
+__global__ void __launch_bounds__(kScatterWarps * 32)
+    dispatch_scatter_kernel(const int32_t* __restrict__ idx, int n, int E,
+                            const int32_t* __restrict__ blk_base, int32_t* __restrict__ perm,
+                            int32_t* __restrict__ pos) {
+  extern __shared__ int32_t cnt[];  // [kScatterWarps][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kScatterWarps * E; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  constexpr int kPerWarp = kDispatchChunk / kScatterWarps;
+  const int beg = blockIdx.x * kDispatchChunk + warp * kPerWarp;
+  const int end = min(n, beg + kPerWarp);
+  int32_t* my = cnt + warp * E;
+
+  for (int s0 = beg; s0 < end; s0 += 32) {
+    const int s = s0 + lane;
+    int e = (s < end) ? idx[s] : -1;
+    if (e < 0 || e >= E) e = -1;
+    const unsigned m = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(m) - 1) my[e] += __popc(m);
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = blk_base[size_t(blockIdx.x) * E + e];
+    for (int w = 0; w < kScatterWarps; ++w) {
+      const int c = cnt[w * E + e];
+      cnt[w * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  for (int s0 = beg; s0 < end; s0 += 32) {
+    const int s = s0 + lane;
+    int e = (s < end) ? idx[s] : -1;
+    if (e < 0 || e >= E) e = -1;
+    const unsigned m = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(m & ((1u << lane) - 1u));
+    const int base = (e >= 0) ? my[e] : 0;
+    __syncwarp();
+    if (e >= 0) {
+      const int p = base + rank;
+      perm[p] = s;
+      pos[s] = p;
+      if (lane == __ffs(m) - 1) my[e] = base + __popc(m);
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const Ctx& c, const int32_t* topk_idx, int T, int nblk,
+                            int32_t* blk_hist, int32_t* counts, int32_t* offsets, int32_t* perm,
+                            int32_t* pos, int32_t* sched, int* status, cudaStream_t st) {
+  const int n = T * c.k;
+  dispatch_count_kernel<<<nblk, kCountThreads, c.E * sizeof(int32_t), st>>>(topk_idx, n, c.E,
+                                                                            blk_hist, status);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(blk_hist, nblk, c.E, c.S, T, counts, offsets,
+                                                   sched);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  dispatch_scatter_kernel<<<nblk, kScatterWarps * 32, kScatterWarps * c.E * sizeof(int32_t),
+                            st>>>(topk_idx, n, c.E, blk_hist, perm, pos);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_schedule_from_offsets(const Ctx& c, const int32_t* offsets, int T,
+                                         int32_t* sched, cudaStream_t st) {
+  schedule_from_offsets_kernel<<<1, kScanThreads, 0, st>>>(offsets, c.E, c.S, T, sched);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

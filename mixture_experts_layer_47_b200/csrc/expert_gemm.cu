@@ -1,0 +1,472 @@
+// expert_gemm.cu -- grouped bf16 expert GEMMs on the sm_100a tensor cores.
+//
+// The expert FFN of the layer (m.xxqk.cn Hy4-preview MoE explainer, section
+// 2.1: every expert is an FFN sub-network standing in for the dense FFN; ZAKER
+// Hy4 Preview release news: 256 routed experts plus one shared expert) is, per
+// group g (a routed expert's token segment, or the shared expert over all T
+// tokens), two dense contractions:
+//   gate/up:  H_g = silu(X_g W_gate_g^T) * (X_g W_up_g^T)   -> bf16
+//   down:     Y_g = H_g W_down_g^T                           -> fp32
+// Both run in one persistent, warp-specialised kernel template:
+//   warp 0      TMA producer: 128x64 A tiles and 256x64 B tiles (128-byte
+//               swizzle) into a 4-stage shared-memory ring;
+//   warp 1      allocates 512 TMEM columns, one elected lane issues
+//               tcgen05.mma (M=128, N=256, K=16) into one of two fp32 TMEM
+//               accumulators and commits stage releases / tile completion to
+//               mbarriers;
+//   warps 2-5   epilogue: tcgen05.ld the accumulator (one TMEM lane per row),
+//               apply SwiGLU (gate/up) or pass fp32 through (down), store.
+// The gate/up B tile stacks 128 gate rows over the matching 128 up rows, so
+// one 256-wide accumulator holds both halves of 128 output features and the
+// SwiGLU product is formed in the epilogue without a second pass.
+// Tiles are enumerated group by group, N-tile-major inside a group, so CTAs
+// running at the same time share a weight tile through L2.  Every wait is
+// bounded; on expiry the kernel records the fault in the status word, drains
+// its own copies and MMAs, frees TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_TILE_BYTES = BM * BK * 2;
+constexpr int B_TILE_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_TILE_BYTES + B_TILE_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr int ACC_COLS = BN;           // fp32 columns per accumulator
+constexpr int TMEM_COLS = 2 * ACC_COLS;
+constexpr int MAX_GROUPS = 1024 + 8;   // E + S upper bound
+constexpr uint32_t IDESC = umma_idesc_bf16_f32(BM, BN);
+
+struct __align__(64) GemmParams {
+  CUtensorMap a_routed;  // gate/up: X_perm [T*k][d]; down: H [T*k+S*T][F]
+  CUtensorMap a_shared;  // gate/up: x [T][d];        down: same as a_routed
+  CUtensorMap b0;        // gate/up: W_gate [E*F][d]; down: W_down [E*d][F]
+  CUtensorMap b1;        // gate/up: W_up   [E*F][d]; down: unused
+  CUtensorMap s0;        // shared counterparts of b0 / b1
+  CUtensorMap s1;
+  const int32_t* offsets;  // [E+1]
+  const int32_t* sched;    // [E+S+1] prefix sums of M-tiles per group
+  void* out;               // gate/up: H bf16; down: Y fp32
+  int* status;
+  int T, E, S, k;
+  int K;          // reduction length (d or F)
+  int n_out;      // output features per group (F or d)
+  int b_rows;     // weight rows per expert in the B maps (F or d)
+  int out_rows;   // rows of the output buffer (T*k + S*T)
+};
+
+struct SharedStorage {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+  int sched[MAX_GROUPS + 1];
+  int offsets[MAX_GROUPS + 1];
+};
+
+constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + size_t(STAGES) * STAGE_BYTES +
+                              sizeof(SharedStorage);
+
+struct Tile {
+  int g, m_idx, n_idx;
+  int rows;      // valid rows of group g
+  int a_row;     // first A row of this tile
+  int out_row;   // first output row of this tile
+  int b_row;     // first weight row (in the per-group B map) of this tile
+  bool shared;
+};
+
+template <bool kGateUp>
+__device__ __forceinline__ Tile decode_tile(int t, int n_tiles, int G, const SharedStorage& ss,
+                                            const GemmParams& p) {
+  const int q = t / n_tiles;
+  int lo = 0, hi = G;  // largest g in [0, G) with sched[g] <= q
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (ss.sched[mid] <= q) lo = mid; else hi = mid;
+  }
+  Tile tl;
+  tl.g = lo;
+  const int mt = ss.sched[lo + 1] - ss.sched[lo];
+  const int local = t - ss.sched[lo] * n_tiles;
+  tl.n_idx = local / mt;
+  tl.m_idx = local - tl.n_idx * mt;
+  const int nslots = p.T * p.k;
+  constexpr int kOutCols = kGateUp ? BN / 2 : BN;
+  if (lo < p.E) {
+    tl.shared = false;
+    tl.rows = ss.offsets[lo + 1] - ss.offsets[lo];
+    tl.a_row = ss.offsets[lo] + tl.m_idx * BM;
+    tl.out_row = tl.a_row;
+    tl.b_row = lo * p.b_rows + tl.n_idx * kOutCols;
+  } else {
+    const int s = lo - p.E;
+    tl.shared = true;
+    tl.rows = p.T;
+    tl.out_row = nslots + s * p.T + tl.m_idx * BM;
+    tl.a_row = kGateUp ? tl.m_idx * BM : tl.out_row;
+    tl.b_row = s * p.b_rows + tl.n_idx * kOutCols;
+  }
+  return tl;
+}
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_TILE_BYTES;
+  SharedStorage& ss = *reinterpret_cast<SharedStorage*>(smem + STAGES * STAGE_BYTES);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = p.E + p.S;
+
+  for (int i = threadIdx.x; i <= G; i += NUM_THREADS) ss.sched[i] = p.sched[i];
+  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) ss.offsets[i] = p.offsets[i];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ss.full[s], 1);
+      mbar_init(&ss.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&ss.tmem_full[a], 1);
+      mbar_init(&ss.tmem_empty[a], 128);
+    }
+    mbar_init(&ss.mma_done, 1);
+    ss.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.a_routed);
+    tma_prefetch_desc(&p.a_shared);
+    tma_prefetch_desc(&p.b0);
+    tma_prefetch_desc(&p.s0);
+    if (kGateUp) {
+      tma_prefetch_desc(&p.b1);
+      tma_prefetch_desc(&p.s1);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(&ss.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ss.tmem_base;
+
+  constexpr int kOutCols = kGateUp ? BN / 2 : BN;
+  const int n_tiles = (p.n_out + kOutCols - 1) / kOutCols;
+  const int total = ss.sched[G] * n_tiles;
+  const int kblocks = p.K / BK;
+  volatile int* abort_flag = &ss.abort_flag;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        if (*abort_flag) break;
+        const Tile tl = decode_tile<kGateUp>(t, n_tiles, G, ss, p);
+        const CUtensorMap* mA = tl.shared ? &p.a_shared : &p.a_routed;
+        const CUtensorMap* mB0 = tl.shared ? &p.s0 : &p.b0;
+        const CUtensorMap* mB1 = tl.shared ? &p.s1 : &p.b1;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&ss.empty[stage], phase ^ 1)) {
+            report_error(p.status, kDevTimeout, kSiteProducer);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&ss.full[stage], STAGE_BYTES);
+          const int kc = kb * BK;
+          tma_load_2d_nohint(sA + stage * A_TILE_BYTES, mA, &ss.full[stage], kc, tl.a_row);
+          if (kGateUp) {
+            uint8_t* dst = sB + stage * B_TILE_BYTES;
+            tma_load_2d_nohint(dst, mB0, &ss.full[stage], kc, tl.b_row);
+            tma_load_2d_nohint(dst + B_TILE_BYTES / 2, mB1, &ss.full[stage], kc, tl.b_row);
+          } else {
+            tma_load_2d_nohint(sB + stage * B_TILE_BYTES, mB0, &ss.full[stage], kc, tl.b_row);
+          }
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Drain: every load this thread issued must have landed before the CTA
+      // may exit (normally they all have: the MMA warp consumed them).
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_mask & (1u << s))
+          if (!mbar_wait(&ss.full[s], (issued_parity >> s) & 1u, kDrainTimeoutNs))
+            report_error(p.status, kDevTimeout, kSiteDrain);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        if (*abort_flag) break;
+        if (!mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1)) {
+          report_error(p.status, kDevTimeout, kSiteMma);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + uint32_t(acc * ACC_COLS);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&ss.full[stage], phase)) {
+            report_error(p.status, kDevTimeout, kSiteMma);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a_desc = umma_desc_sw128_kmajor(smem_u32(sA + stage * A_TILE_BYTES));
+          const uint64_t b_desc = umma_desc_sw128_kmajor(smem_u32(sB + stage * B_TILE_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16(d_tmem, a_desc + uint64_t(2 * kk), b_desc + uint64_t(2 * kk), IDESC,
+                      (kb | kk) != 0 ? 1u : 0u);
+          umma_commit(&ss.empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&ss.tmem_full[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      // Drain: wait until every MMA issued here has completed.
+      umma_commit(&ss.mma_done);
+      if (!mbar_wait(&ss.mma_done, 0, kDrainTimeoutNs))
+        report_error(p.status, kDevTimeout, kSiteDrain);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5, one accumulator row per thread) --------
+    const int quarter = warp & 3;               // TMEM lanes [32*quarter, 32*quarter+32)
+    const int row_in_tile = quarter * 32 + lane;
+    const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      if (*abort_flag) break;
+      const Tile tl = decode_tile<kGateUp>(t, n_tiles, G, ss, p);
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&ss.tmem_full[acc], acc_phase));
+      if (!ok) {
+        if (lane == 0) report_error(p.status, kDevTimeout, kSiteEpilogue);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int r = tl.m_idx * BM + row_in_tile;
+      const int out_row = tl.out_row + row_in_tile;
+      const bool valid = r < tl.rows && out_row >= 0 && out_row < p.out_rows;
+      const uint32_t tbase = tmem_base + lane_addr + uint32_t(acc * ACC_COLS);
+      if (kGateUp) {
+        uint16_t* H = reinterpret_cast<uint16_t*>(p.out);
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld_32cols(tbase + uint32_t(c), g);
+          tmem_ld_32cols(tbase + uint32_t(BN / 2 + c), u);
+          tmem_ld_wait();
+          const int col0 = tl.n_idx * (BN / 2) + c;
+          if (valid && col0 < p.n_out) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
+              const float u0 = __uint_as_float(u[2 * j]), u1 = __uint_as_float(u[2 * j + 1]);
+              const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+              const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+              packed[j] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(H + size_t(out_row) * p.n_out + col0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2],
+                                  packed[4 * v + 3]);
+          }
+        }
+      } else {
+        float* Y = reinterpret_cast<float*>(p.out);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld_32cols(tbase + uint32_t(c), v);
+          tmem_ld_wait();
+          const int col0 = tl.n_idx * BN + c;
+          if (valid && col0 < p.n_out) {
+            float4* dst = reinterpret_cast<float4*>(Y + size_t(out_row) * p.n_out + col0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&ss.tmem_empty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launches.
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 2-D bf16 tensor [rows][cols] (cols contiguous), box [box_rows][64], 128-byte
+// swizzle, out-of-bounds elements read as zero.
+bool encode_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, int box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {uint32_t(BK), uint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool kGateUp>
+cudaError_t set_attrs() {
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+}
+
+}  // namespace
+
+moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
+                             cudaStream_t st) {
+  if (!get_encoder()) return MOE_ERR_CUDA;
+  static thread_local int attrs_device = -1;
+  if (attrs_device != dev.device) {
+    if (set_attrs<true>() != cudaSuccess || set_attrs<false>() != cudaSuccess)
+      return MOE_ERR_CUDA;
+    attrs_device = dev.device;
+  }
+  const int T = a.T;
+  const uint64_t nslots = uint64_t(T) * c.k;
+  const uint64_t rows = nslots + uint64_t(c.S) * T;
+
+  // ---- gate/up + SwiGLU ----
+  GemmParams gp;
+  memset(&gp, 0, sizeof gp);
+  bool ok = encode_2d(&gp.a_routed, a.x_perm, nslots, c.d, BM) &&
+            encode_2d(&gp.a_shared, a.x, uint64_t(T), c.d, BM) &&
+            encode_2d(&gp.b0, a.Wg, uint64_t(c.E) * c.F, c.d, BN / 2) &&
+            encode_2d(&gp.b1, a.Wu, uint64_t(c.E) * c.F, c.d, BN / 2);
+  if (c.S > 0)
+    ok = ok && encode_2d(&gp.s0, a.Sg, uint64_t(c.S) * c.F, c.d, BN / 2) &&
+         encode_2d(&gp.s1, a.Su, uint64_t(c.S) * c.F, c.d, BN / 2);
+  else {
+    gp.s0 = gp.b0;
+    gp.s1 = gp.b1;
+  }
+  if (!ok) return MOE_ERR_CUDA;
+  gp.offsets = a.offsets;
+  gp.sched = a.sched;
+  gp.out = a.h_act;
+  gp.status = a.status;
+  gp.T = T;
+  gp.E = c.E;
+  gp.S = c.S;
+  gp.k = c.k;
+  gp.K = c.d;
+  gp.n_out = c.F;
+  gp.b_rows = c.F;
+  gp.out_rows = int(rows);
+  const int grid = dev.num_sms;
+  grouped_gemm_kernel<true><<<grid, NUM_THREADS, kSmemBytes, st>>>(gp);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (a.after_gate_up && cudaEventRecord(a.after_gate_up, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // ---- down projection ----
+  GemmParams dp;
+  memset(&dp, 0, sizeof dp);
+  ok = encode_2d(&dp.a_routed, a.h_act, rows, c.F, BM) &&
+       encode_2d(&dp.b0, a.Wd, uint64_t(c.E) * c.d, c.F, BN);
+  if (c.S > 0)
+    ok = ok && encode_2d(&dp.s0, a.Sd, uint64_t(c.S) * c.d, c.F, BN);
+  else
+    dp.s0 = dp.b0;
+  if (!ok) return MOE_ERR_CUDA;
+  dp.a_shared = dp.a_routed;
+  dp.b1 = dp.b0;
+  dp.s1 = dp.s0;
+  dp.offsets = a.offsets;
+  dp.sched = a.sched;
+  dp.out = a.Y;
+  dp.status = a.status;
+  dp.T = T;
+  dp.E = c.E;
+  dp.S = c.S;
+  dp.k = c.k;
+  dp.K = c.F;
+  dp.n_out = c.d;
+  dp.b_rows = c.d;
+  dp.out_rows = int(rows);
+  grouped_gemm_kernel<false><<<grid, NUM_THREADS, kSmemBytes, st>>>(dp);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace moe

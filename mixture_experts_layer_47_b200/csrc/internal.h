@@ -1,0 +1,81 @@
+// internal.h -- host-side declarations shared by the translation units of
+// libmoe.so (not part of the public ABI; see include/moe.h for that).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+struct Ctx {
+  int d, E, k, F, S;
+};
+
+// Geometry of the router's split-K partial sums for T tokens.
+struct RouterPlan {
+  int bt;      // tokens per CTA tile (16 or 64)
+  int ksplit;  // number of K chunks
+  int kchunk;  // d / ksplit
+};
+RouterPlan router_plan(const Ctx& c, int T, int num_sms);
+
+// Workspace carve-up for T tokens (offsets from the 1024-aligned base).
+struct Layout {
+  size_t status, part, topk_idx, topk_w, counts, offsets, perm, pos, blk_hist, sched, x_perm,
+      h_act, y_rows, x_stage, y_stage, end;
+  int nblk;           // dispatch blocks
+  RouterPlan rplan;
+};
+Layout make_layout(const Ctx& c, int T, int num_sms);
+
+constexpr int kDispatchChunk = 4096;   // slots per dispatch block
+constexpr size_t kWsAlign = 1024;
+
+// Per-device state, filled at the first launch on that device.
+struct DeviceInfo {
+  int device = -1;
+  int num_sms = 0;
+  int cc_major = 0, cc_minor = 0;
+  bool ready = false;
+};
+moe_status ensure_device(DeviceInfo** out);
+
+// ---- launchers (each returns cudaSuccess or the launch error) ----
+cudaError_t launch_router(const Ctx& c, const RouterPlan& rp, const uint16_t* x, const float* Wr,
+                          const float* bias, int T, float* part, int32_t* topk_idx, float* topk_w,
+                          cudaStream_t st);
+
+cudaError_t launch_dispatch(const Ctx& c, const int32_t* topk_idx, int T, int nblk,
+                            int32_t* blk_hist, int32_t* counts, int32_t* offsets, int32_t* perm,
+                            int32_t* pos, int32_t* sched, int* status, cudaStream_t st);
+
+cudaError_t launch_schedule_from_offsets(const Ctx& c, const int32_t* offsets, int T,
+                                         int32_t* sched, cudaStream_t st);
+
+cudaError_t launch_gather(const Ctx& c, const uint16_t* x, const int32_t* perm,
+                          const int32_t* offsets, int T, uint16_t* x_perm, int num_sms,
+                          cudaStream_t st);
+
+cudaError_t launch_combine(const Ctx& c, const float* Y, const float* topk_w, const int32_t* pos,
+                           int T, uint16_t* y, cudaStream_t st);
+
+struct FfnArgs {
+  const uint16_t* x;        // [T][d]
+  const uint16_t* x_perm;   // [T*k][d]
+  const int32_t* offsets;   // [E+1]
+  const int32_t* sched;     // [E+S+1]
+  const uint16_t *Wg, *Wu, *Wd, *Sg, *Su, *Sd;
+  uint16_t* h_act;          // [T*k+S*T][F]
+  float* Y;                 // [T*k+S*T][d]
+  int* status;
+  int T;
+  cudaEvent_t after_gate_up;  // recorded between the two GEMMs when non-null
+};
+moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
+                             cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,458 @@
+// moe_api.cu -- the extern "C" entry points declared in include/moe.h.
+//
+// Host-side argument checks, the workspace carve-up, and the launch sequence
+// of the layer: router -> dispatch -> gather -> gate/up GEMM (+SwiGLU) ->
+// down GEMM -> combine, all on the caller's stream with no host
+// synchronisation.  The carve-up does not depend on the device, so the
+// workspace size and every result are the same on any sm_100 GPU.
+#include <cuda_runtime.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+#include <new>
+
+#include "common.cuh"
+#include "internal.h"
+
+struct moe_ctx {
+  moe::Ctx c;
+  cudaEvent_t stage_events[MOE_STAGE_EVENTS];
+  int n_stage_events;
+};
+
+namespace moe {
+namespace {
+
+constexpr int kPlanSms = 148;            // device-independent planning constant
+constexpr long long kMaxRows = 1ll << 24;  // T*k + S*T upper bound
+constexpr int kMaxDevices = 64;
+
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_dev_mu;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+uint8_t* aligned_base(void* ws) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws) + kWsAlign - 1) &
+                                    ~uintptr_t(kWsAlign - 1));
+}
+
+moe_status check_T(const Ctx& c, int T) {
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if ((long long)T * (c.k + c.S) > kMaxRows) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_ws(moe_handle h, int T, const void* ws, size_t ws_bytes) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_workspace_size(h, T)) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+moe_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  cudaGetLastError();  // clear a non-sticky error so the caller's context stays usable
+  return MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+Layout make_layout(const Ctx& c, int T, int num_sms) {
+  Layout L;
+  memset(&L, 0, sizeof L);
+  L.rplan = router_plan(c, T, num_sms);
+  const size_t nslots = size_t(T) * c.k;
+  const size_t rows = nslots + size_t(c.S) * T;
+  L.nblk = int(std::max<size_t>(1, (nslots + kDispatchChunk - 1) / kDispatchChunk));
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + std::max<size_t>(bytes, 16), kWsAlign);
+    return o;
+  };
+  L.status = take(256);
+  L.part = take(size_t(L.rplan.ksplit) * T * c.E * sizeof(float));
+  L.topk_idx = take(nslots * sizeof(int32_t));
+  L.topk_w = take(nslots * sizeof(float));
+  L.counts = take(size_t(c.E) * sizeof(int32_t));
+  L.offsets = take(size_t(c.E + 1) * sizeof(int32_t));
+  L.perm = take(nslots * sizeof(int32_t));
+  L.pos = take(nslots * sizeof(int32_t));
+  L.blk_hist = take(size_t(L.nblk) * c.E * sizeof(int32_t));
+  L.sched = take(size_t(c.E + c.S + 1) * sizeof(int32_t));
+  L.x_perm = take(nslots * c.d * sizeof(uint16_t));
+  L.h_act = take(rows * c.F * sizeof(uint16_t));
+  L.y_rows = take(rows * c.d * sizeof(float));
+  L.x_stage = take(size_t(T) * c.d * sizeof(uint16_t));
+  L.y_stage = take(size_t(T) * c.d * sizeof(uint16_t));
+  L.end = off;
+  return L;
+}
+
+moe_status ensure_device(DeviceInfo** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& di = g_devices[dev];
+  if (!di.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    // The kernels are built for sm_100a only (arch-specific tcgen05 / TMA).
+    if (major != 10 || minor != 0) return MOE_ERR_UNSUPPORTED;
+    di.device = dev;
+    di.cc_major = major;
+    di.cc_minor = minor;
+    di.num_sms = sms;
+    di.ready = true;
+  }
+  *out = &di;
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_create(int d_model, int n_experts, int top_k, int d_ff, int n_shared,
+                      moe_handle* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (d_model <= 0 || d_ff <= 0 || n_experts <= 0 || top_k < 1 || top_k > n_experts ||
+      n_shared < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (d_model % 64 || d_ff % 64 || d_model > 65536 || d_ff > 65536 || n_experts > 1024 ||
+      top_k > 32 || n_shared > 8)
+    return MOE_ERR_UNSUPPORTED;
+  moe_ctx* h = new (std::nothrow) moe_ctx;
+  if (!h) return MOE_ERR_INVALID_ARG;
+  h->c = Ctx{d_model, n_experts, top_k, d_ff, n_shared};
+  h->n_stage_events = 0;
+  *out = h;
+  return MOE_OK;
+}
+
+moe_status moe_destroy(moe_handle h) {
+  delete h;
+  return MOE_OK;
+}
+
+size_t moe_workspace_size(moe_handle h, int T) {
+  if (!h || T < 0) return 0;
+  if ((long long)T * (h->c.k + h->c.S) > kMaxRows) return 0;
+  return make_layout(h->c, T, kPlanSms).end + kWsAlign;
+}
+
+moe_status moe_get_workspace_layout(moe_handle h, int T, uintptr_t workspace_addr,
+                                    moe_workspace_layout* out) {
+  if (!h || !out) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_T(h->c, T);
+  if (s) return s;
+  const Layout L = make_layout(h->c, T, kPlanSms);
+  const size_t base = ((workspace_addr + kWsAlign - 1) & ~uintptr_t(kWsAlign - 1)) - workspace_addr;
+  out->status = base + L.status;
+  out->topk_idx = base + L.topk_idx;
+  out->topk_w = base + L.topk_w;
+  out->counts = base + L.counts;
+  out->offsets = base + L.offsets;
+  out->perm = base + L.perm;
+  out->pos = base + L.pos;
+  out->h_act = base + L.h_act;
+  out->y_rows = base + L.y_rows;
+  out->total = base + L.end;
+  return MOE_OK;
+}
+
+moe_status moe_route(moe_handle h, const uint16_t* x, const float* W_router, const float* bias,
+                     int T, int32_t* topk_idx, float* topk_w, void* workspace, size_t ws_bytes,
+                     void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_T(h->c, T);
+  if (s) return s;
+  if (T == 0) return MOE_OK;
+  if (!x || !W_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(W_router)) return MOE_ERR_ALIGNMENT;
+  if ((s = check_ws(h, T, workspace, ws_bytes))) return s;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Layout L = make_layout(h->c, T, kPlanSms);
+  uint8_t* ws = aligned_base(workspace);
+  if ((s = cuda_status(cudaMemsetAsync(ws + L.status, 0, sizeof(int), st)))) return s;
+  return cuda_status(launch_router(h->c, L.rplan, x, W_router, bias, T,
+                                   reinterpret_cast<float*>(ws + L.part), topk_idx, topk_w, st));
+}
+
+moe_status moe_dispatch(moe_handle h, const int32_t* topk_idx, int T, int32_t* counts,
+                        int32_t* offsets, int32_t* perm, int32_t* pos, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_T(h->c, T);
+  if (s) return s;
+  if (T == 0) return MOE_OK;
+  if (!topk_idx || !counts || !offsets || !perm || !pos) return MOE_ERR_INVALID_ARG;
+  if ((s = check_ws(h, T, workspace, ws_bytes))) return s;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Layout L = make_layout(h->c, T, kPlanSms);
+  uint8_t* ws = aligned_base(workspace);
+  int* status = reinterpret_cast<int*>(ws + L.status);
+  if ((s = cuda_status(cudaMemsetAsync(status, 0, sizeof(int), st)))) return s;
+  return cuda_status(launch_dispatch(h->c, topk_idx, T, L.nblk,
+                                     reinterpret_cast<int32_t*>(ws + L.blk_hist), counts, offsets,
+                                     perm, pos, reinterpret_cast<int32_t*>(ws + L.sched), status,
+                                     st));
+}
+
+static moe_status check_weights(const Ctx& c, const uint16_t* Wg, const uint16_t* Wu,
+                                const uint16_t* Wd, const uint16_t* Sg, const uint16_t* Su,
+                                const uint16_t* Sd) {
+  if (!Wg || !Wu || !Wd) return MOE_ERR_INVALID_ARG;
+  if (c.S > 0 && (!Sg || !Su || !Sd)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(Wg) || !aligned16(Wu) || !aligned16(Wd)) return MOE_ERR_ALIGNMENT;
+  if (c.S > 0 && (!aligned16(Sg) || !aligned16(Su) || !aligned16(Sd))) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+moe_status moe_expert_ffn(moe_handle h, const uint16_t* x, const int32_t* perm,
+                          const int32_t* offsets, int T, const uint16_t* W_gate,
+                          const uint16_t* W_up, const uint16_t* W_down, const uint16_t* Ws_gate,
+                          const uint16_t* Ws_up, const uint16_t* Ws_down, float* Y,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  moe_status s = check_T(c, T);
+  if (s) return s;
+  if (T == 0) return MOE_OK;
+  if (!x || !perm || !offsets || !Y) return MOE_ERR_INVALID_ARG;
+  if ((s = check_weights(c, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down))) return s;
+  if (!aligned16(x) || !aligned16(Y)) return MOE_ERR_ALIGNMENT;
+  if ((s = check_ws(h, T, workspace, ws_bytes))) return s;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Layout L = make_layout(c, T, kPlanSms);
+  uint8_t* ws = aligned_base(workspace);
+  int* status = reinterpret_cast<int*>(ws + L.status);
+  int32_t* sched = reinterpret_cast<int32_t*>(ws + L.sched);
+  uint16_t* x_perm = reinterpret_cast<uint16_t*>(ws + L.x_perm);
+  if ((s = cuda_status(cudaMemsetAsync(status, 0, sizeof(int), st)))) return s;
+  if ((s = cuda_status(launch_schedule_from_offsets(c, offsets, T, sched, st)))) return s;
+  if ((s = cuda_status(launch_gather(c, x, perm, offsets, T, x_perm, dev->num_sms, st)))) return s;
+  FfnArgs a;
+  a.x = x;
+  a.x_perm = x_perm;
+  a.offsets = offsets;
+  a.sched = sched;
+  a.Wg = W_gate;
+  a.Wu = W_up;
+  a.Wd = W_down;
+  a.Sg = Ws_gate;
+  a.Su = Ws_up;
+  a.Sd = Ws_down;
+  a.h_act = reinterpret_cast<uint16_t*>(ws + L.h_act);
+  a.Y = Y;
+  a.status = status;
+  a.T = T;
+  a.after_gate_up = nullptr;
+  return launch_expert_ffn(c, a, *dev, st);
+}
+
+moe_status moe_combine(moe_handle h, const float* Y, const float* topk_w, const int32_t* pos,
+                       int T, uint16_t* y, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_T(h->c, T);
+  if (s) return s;
+  if (T == 0) return MOE_OK;
+  if (!Y || !topk_w || !pos || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(Y) || !aligned16(y)) return MOE_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  return cuda_status(
+      launch_combine(h->c, Y, topk_w, pos, T, y, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W_router,
+                                 const float* bias, const uint16_t* W_gate, const uint16_t* W_up,
+                                 const uint16_t* W_down, const uint16_t* Ws_gate,
+                                 const uint16_t* Ws_up, const uint16_t* Ws_down, int T,
+                                 uint16_t* y, uint8_t* ws, const Layout& L, DeviceInfo* dev,
+                                 cudaStream_t st) {
+  const Ctx& c = h->c;
+  moe_status s;
+  int* status = reinterpret_cast<int*>(ws + L.status);
+  int32_t* topk_idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
+  float* topk_w = reinterpret_cast<float*>(ws + L.topk_w);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+  int32_t* pos = reinterpret_cast<int32_t*>(ws + L.pos);
+  int32_t* sched = reinterpret_cast<int32_t*>(ws + L.sched);
+  uint16_t* x_perm = reinterpret_cast<uint16_t*>(ws + L.x_perm);
+  float* Y = reinterpret_cast<float*>(ws + L.y_rows);
+  const bool prof = h->n_stage_events == MOE_STAGE_EVENTS;
+  auto mark = [&](int i) -> moe_status {
+    return prof ? cuda_status(cudaEventRecord(h->stage_events[i], st)) : MOE_OK;
+  };
+  if ((s = cuda_status(cudaMemsetAsync(status, 0, sizeof(int), st)))) return s;
+  if ((s = mark(0))) return s;
+  if ((s = cuda_status(launch_router(c, L.rplan, x, W_router, bias, T,
+                                     reinterpret_cast<float*>(ws + L.part), topk_idx, topk_w,
+                                     st))))
+    return s;
+  if ((s = mark(1))) return s;
+  if ((s = cuda_status(launch_dispatch(c, topk_idx, T, L.nblk,
+                                       reinterpret_cast<int32_t*>(ws + L.blk_hist), counts,
+                                       offsets, perm, pos, sched, status, st))))
+    return s;
+  if ((s = mark(2))) return s;
+  if ((s = cuda_status(launch_gather(c, x, perm, offsets, T, x_perm, dev->num_sms, st)))) return s;
+  if ((s = mark(3))) return s;
+  FfnArgs a;
+  a.x = x;
+  a.x_perm = x_perm;
+  a.offsets = offsets;
+  a.sched = sched;
+  a.Wg = W_gate;
+  a.Wu = W_up;
+  a.Wd = W_down;
+  a.Sg = Ws_gate;
+  a.Su = Ws_up;
+  a.Sd = Ws_down;
+  a.h_act = reinterpret_cast<uint16_t*>(ws + L.h_act);
+  a.Y = Y;
+  a.status = status;
+  a.T = T;
+  a.after_gate_up = prof ? h->stage_events[4] : nullptr;
+  if ((s = launch_expert_ffn(c, a, *dev, st))) return s;
+  if ((s = mark(5))) return s;
+  if ((s = cuda_status(launch_combine(c, Y, topk_w, pos, T, y, st)))) return s;
+  return mark(6);
+}
+
+static moe_status check_forward_args(moe_handle h, const uint16_t* x, const float* W_router,
+                                     const uint16_t* W_gate, const uint16_t* W_up,
+                                     const uint16_t* W_down, const uint16_t* Ws_gate,
+                                     const uint16_t* Ws_up, const uint16_t* Ws_down, int T,
+                                     const uint16_t* y, bool host_io, const void* workspace,
+                                     size_t ws_bytes) {
+  if (!x || !W_router || !y) return MOE_ERR_INVALID_ARG;
+  moe_status s;
+  if ((s = check_weights(h->c, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down))) return s;
+  if (!aligned16(W_router)) return MOE_ERR_ALIGNMENT;
+  if (!host_io && (!aligned16(x) || !aligned16(y))) return MOE_ERR_ALIGNMENT;
+  return check_ws(h, T, workspace, ws_bytes);
+}
+
+moe_status moe_forward(moe_handle h, const uint16_t* x, const float* W_router, const float* bias,
+                       const uint16_t* W_gate, const uint16_t* W_up, const uint16_t* W_down,
+                       const uint16_t* Ws_gate, const uint16_t* Ws_up, const uint16_t* Ws_down,
+                       int T, uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_T(h->c, T);
+  if (s) return s;
+  if (T == 0) return MOE_OK;
+  if ((s = check_forward_args(h, x, W_router, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, T,
+                              y, false, workspace, ws_bytes)))
+    return s;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  const Layout L = make_layout(h->c, T, kPlanSms);
+  return forward_device(h, x, W_router, bias, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, T,
+                        y, aligned_base(workspace), L, dev,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward_host(moe_handle h, const uint16_t* x_host, const float* W_router,
+                            const float* bias, const uint16_t* W_gate, const uint16_t* W_up,
+                            const uint16_t* W_down, const uint16_t* Ws_gate,
+                            const uint16_t* Ws_up, const uint16_t* Ws_down, int T,
+                            uint16_t* y_host, void* workspace, size_t ws_bytes, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_T(h->c, T);
+  if (s) return s;
+  if (T == 0) return MOE_OK;
+  if ((s = check_forward_args(h, x_host, W_router, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down,
+                              T, y_host, true, workspace, ws_bytes)))
+    return s;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Layout L = make_layout(h->c, T, kPlanSms);
+  uint8_t* ws = aligned_base(workspace);
+  const size_t bytes = size_t(T) * h->c.d * sizeof(uint16_t);
+  uint16_t* x_dev = reinterpret_cast<uint16_t*>(ws + L.x_stage);
+  uint16_t* y_dev = reinterpret_cast<uint16_t*>(ws + L.y_stage);
+  if ((s = cuda_status(cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st))))
+    return s;
+  if ((s = forward_device(h, x_dev, W_router, bias, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down,
+                          T, y_dev, ws, L, dev, st)))
+    return s;
+  return cuda_status(cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st));
+}
+
+moe_status moe_device_status(moe_handle h, int T, const void* workspace, void* stream,
+                             int32_t* device_detail) {
+  if (!h || !workspace) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_T(h->c, T);
+  if (s) return s;
+  if (device_detail) *device_detail = 0;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Layout L = make_layout(h->c, T, kPlanSms);
+  const uint8_t* ws = aligned_base(const_cast<void*>(workspace));
+  int32_t word = 0;
+  if ((s = cuda_status(cudaMemcpyAsync(&word, ws + L.status, sizeof word, cudaMemcpyDeviceToHost,
+                                       st))))
+    return s;
+  if ((s = cuda_status(cudaStreamSynchronize(st)))) return s;
+  if (device_detail) *device_detail = word;
+  if (word == 0) return MOE_OK;
+  return (word >> 16) == kDevBadIndex ? MOE_ERR_BAD_INDEX : MOE_ERR_TIMEOUT;
+}
+
+moe_status moe_set_stage_events(moe_handle h, void* const* events, int n_events) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (!events || n_events == 0) {
+    h->n_stage_events = 0;
+    return MOE_OK;
+  }
+  if (n_events != MOE_STAGE_EVENTS) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < MOE_STAGE_EVENTS; ++i) {
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+    h->stage_events[i] = reinterpret_cast<cudaEvent_t>(events[i]);
+  }
+  h->n_stage_events = MOE_STAGE_EVENTS;
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or device";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "bounded device wait expired";
+    case MOE_ERR_BAD_INDEX: return "expert index out of range";
+    case MOE_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

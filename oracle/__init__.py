@@ -63,8 +63,10 @@ def _load():
                                               P, I, P]
         lib.oracle_expert_one.argtypes = [P, I, I, P, P, P, P, P]
         lib.oracle_num_threads.argtypes = []
+        lib.oracle_combine.argtypes = [P, P, P, I, I, I, I, P]
         for f in ("oracle_router_logits", "oracle_route", "oracle_dispatch",
-                  "oracle_moe_ffn_tokens", "oracle_expert_one", "oracle_num_threads"):
+                  "oracle_moe_ffn_tokens", "oracle_expert_one", "oracle_num_threads",
+                  "oracle_combine"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -216,6 +218,18 @@ def expert_one(xrow, W_gate_e, W_up_e, W_down_e):
     _check(_load().oracle_expert_one(_ptr(xr), d, F, _ptr(Wg), _ptr(Wu), _ptr(Wd), _ptr(h),
                                      _ptr(y)), "expert_one")
     return h, y
+
+
+def combine(Y_rows, w, pos, T: int, k: int, S: int) -> np.ndarray:
+    """y[t] = sum_s Y_rows[T*k + s*T + t] + sum_i w[t, i] * Y_rows[pos[t*k + i]], fp64."""
+    Yr = np.ascontiguousarray(Y_rows, dtype=np.float64)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    pos = _np(pos, np.int32)
+    d = Yr.shape[1]
+    assert Yr.shape[0] == T * k + S * T and w.shape == (T, k) and pos.size == T * k
+    y = np.empty((T, d), np.float64)
+    _check(_load().oracle_combine(_ptr(Yr), _ptr(w), _ptr(pos), T, k, S, d, _ptr(y)), "combine")
+    return y
 
 
 def forward(inp, tokens: Optional[Sequence[int]] = None, idx_override=None,

@@ -275,6 +275,33 @@ int oracle_expert_one(const uint16_t *xrow, int d, int F, const uint16_t *Wg,
     return ORACLE_OK;
 }
 
+/* Step 7 alone -- merge per-(slot, expert) outputs into the layer output:
+ *   y[t] = sum_{s<S} Yrows[T*k + s*T + t] + sum_{i<k} w[t][i] * Yrows[pos[t*k+i]].
+ * Yrows: [T*k + S*T][d] (any fp64 values); w: [T][k]; pos: [T*k]; y: [T][d]. */
+int oracle_combine(const double *Yrows, const double *w, const int32_t *pos, int T, int k, int S,
+                   int d, double *y) {
+    if (T < 0 || k < 1 || S < 0 || d <= 0) return ORACLE_BAD_ARG;
+    if (T == 0) return ORACLE_OK;
+    if (!Yrows || !w || !pos || !y) return ORACLE_BAD_ARG;
+    const long nslots = (long)T * k;
+    for (long s = 0; s < nslots; ++s)
+        if (pos[s] < 0 || pos[s] >= nslots) return ORACLE_BAD_ARG;
+    for (int t = 0; t < T; ++t) {
+        double *yt = y + (size_t)t * d;
+        for (int j = 0; j < d; ++j) yt[j] = 0.0;
+        for (int s = 0; s < S; ++s) {
+            const double *row = Yrows + ((size_t)nslots + (size_t)s * T + t) * d;
+            for (int j = 0; j < d; ++j) yt[j] += row[j];
+        }
+        for (int i = 0; i < k; ++i) {
+            const double wi = w[(size_t)t * k + i];
+            const double *row = Yrows + (size_t)pos[(size_t)t * k + i] * d;
+            for (int j = 0; j < d; ++j) yt[j] += wi * row[j];
+        }
+    }
+    return ORACLE_OK;
+}
+
 /* Number of OpenMP threads a parallel region of this library uses. */
 int oracle_num_threads(void) {
     int n = 1;

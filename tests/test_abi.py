@@ -1,0 +1,159 @@
+"""Host-side checks of the C-ABI library: it builds for sm_100a, loads, exports
+every entry point include/moe.h declares, and rejects bad arguments on the host
+before anything reaches a device.  No kernel runs here."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import mixture_experts_layer_47_b200 as moe
+from mixture_experts_layer_47_b200 import build as moe_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moe_build.build()
+    return moe.load_library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:moe_status|size_t|const char \*)\s*(moe_\w+)\s*\(",
+                                 text, re.M)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 12, names
+    out = subprocess.run(["nm", "-D", "--defined-only", moe.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (moe_\w+)", out))
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n)
+    assert set(names) == set(moe.EXPORTS)
+
+
+def test_library_is_sm100a_only(lib):
+    out = subprocess.run(["cuobjdump", "--list-elf", moe.LIB_PATH], capture_output=True,
+                         text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    archs = set(re.findall(r"sm_(\d+a?)", out.stdout))
+    assert archs == {"100a"}, archs
+
+
+def test_status_strings(lib):
+    for code in range(0, 8):
+        assert moe.status_string(code)
+    assert moe.status_string(99) == "unknown status"
+
+
+def _create(d, E, k, F, S):
+    h = ctypes.c_void_p()
+    rc = moe.load_library().moe_create(d, E, k, F, S, ctypes.byref(h))
+    return rc, h
+
+
+@pytest.mark.parametrize("args,code", [
+    ((6144, 256, 8, 2048, 1), moe.MOE_OK),
+    ((256, 16, 2, 128, 1), moe.MOE_OK),
+    ((64, 1, 1, 64, 0), moe.MOE_OK),
+    ((256, 16, 17, 128, 1), moe.MOE_ERR_INVALID_ARG),   # k > E
+    ((256, 16, 0, 128, 1), moe.MOE_ERR_INVALID_ARG),    # k < 1
+    ((0, 16, 2, 128, 1), moe.MOE_ERR_INVALID_ARG),
+    ((256, 16, 2, 128, -1), moe.MOE_ERR_INVALID_ARG),
+    ((250, 16, 2, 128, 1), moe.MOE_ERR_UNSUPPORTED),    # d not a multiple of 64
+    ((256, 16, 2, 100, 1), moe.MOE_ERR_UNSUPPORTED),    # d_ff not a multiple of 64
+    ((256, 2048, 2, 128, 1), moe.MOE_ERR_UNSUPPORTED),  # E > 1024
+    ((256, 64, 33, 128, 1), moe.MOE_ERR_UNSUPPORTED),   # k > 32
+    ((256, 16, 2, 128, 9), moe.MOE_ERR_UNSUPPORTED),    # S > 8
+])
+def test_create_validates_shape(lib, args, code):
+    rc, h = _create(*args)
+    assert rc == code
+    assert (h.value is not None) == (code == moe.MOE_OK)
+    if h.value:
+        assert lib.moe_destroy(h) == moe.MOE_OK
+    assert lib.moe_create(1, 1, 1, 1, 1, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_workspace_size_and_layout(lib):
+    h = moe.moe_create(6144, 256, 8, 2048, 1)
+    assert moe.moe_workspace_size(h, -1) == 0
+    sizes = [moe.moe_workspace_size(h, T) for T in (1, 16, 256, 8192)]
+    assert all(s > 0 for s in sizes) and sizes == sorted(sizes)
+    # Hy4 prefill: X_perm 805 MB + H 302 MB + Y 1.81 GB + x/y staging 201 MB + small
+    assert 2.9e9 < sizes[-1] < 3.2e9
+    for addr in (0, 1, 1000, 4096 + 16):
+        L = moe.moe_get_workspace_layout(h, 16, addr)
+        assert L["total"] <= moe.moe_workspace_size(h, 16)
+        for key in ("status", "topk_idx", "topk_w", "counts", "offsets", "perm", "pos", "h_act",
+                    "y_rows"):
+            assert (addr + L[key]) % 1024 == 0, key
+    assert lib.moe_workspace_size(None, 16) == 0
+
+
+def test_host_side_argument_errors_need_no_device(lib):
+    """Bad arguments are rejected before any CUDA call, so these never touch a device."""
+    h = moe.moe_create(256, 16, 2, 128, 1)
+    hv = h.value
+    T = 64
+    ws_size = moe.moe_workspace_size(h, T)
+    A = 1 << 20  # a 16-byte aligned fake address; never dereferenced on these paths
+    L = moe.load_library()
+    # null handle / pointers
+    assert L.moe_route(None, A, A, None, T, A, A, A, ws_size, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route(hv, None, A, None, T, A, A, A, ws_size, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route(hv, A, A, None, -1, A, A, A, ws_size, None) == moe.MOE_ERR_INVALID_ARG
+    # misaligned x
+    assert L.moe_route(hv, A + 2, A, None, T, A, A, A, ws_size, None) == moe.MOE_ERR_ALIGNMENT
+    # workspace too small / missing
+    assert L.moe_route(hv, A, A, None, T, A, A, A, ws_size - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_route(hv, A, A, None, T, A, A, None, ws_size, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch(hv, None, T, A, A, A, A, A, ws_size, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch(hv, A, T, A, A, A, A, A, 10, None) == moe.MOE_ERR_WORKSPACE
+    # expert FFN: missing shared weights when S = 1, misaligned weights
+    assert L.moe_expert_ffn(hv, A, A, A, T, A, A, A, None, A, A, A, A, ws_size, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_ffn(hv, A, A, A, T, A + 8, A, A, A, A, A, A, A, ws_size, None) == \
+        moe.MOE_ERR_ALIGNMENT
+    assert L.moe_combine(hv, None, A, A, T, A, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(hv, A, A, A, T, A + 4, None) == moe.MOE_ERR_ALIGNMENT
+    assert L.moe_forward(hv, A, A, None, A, A, A, A, A, A, T, A, A, ws_size - 1, None) == \
+        moe.MOE_ERR_WORKSPACE
+    assert L.moe_forward(hv, A, None, None, A, A, A, A, A, A, T, A, A, ws_size, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    # T == 0 is a no-op that touches nothing
+    assert L.moe_forward(hv, None, None, None, None, None, None, None, None, None, 0, None, None,
+                         0, None) == moe.MOE_OK
+    assert L.moe_dispatch(hv, None, 0, None, None, None, None, None, 0, None) == moe.MOE_OK
+    # more rows than the supported envelope
+    assert L.moe_route(hv, A, A, None, 1 << 23, A, A, A, 1 << 40, None) == \
+        moe.MOE_ERR_UNSUPPORTED
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_valid_call_without_device_reports_cuda_error(lib):
+    """With valid arguments but no GPU, a launch returns MOE_ERR_CUDA instead of crashing."""
+    h = moe.moe_create(256, 16, 2, 128, 1)
+    T = 64
+    ws = moe.moe_workspace_size(h, T)
+    A = 1 << 20
+    L = moe.load_library()
+    assert L.moe_route(h.value, A, A, None, T, A, A, A, ws, None) == moe.MOE_ERR_CUDA
+
+
+def test_python_binding_validates_tensors(lib):
+    h = moe.moe_create(256, 16, 2, 128, 1)
+    ws = torch.empty(16, dtype=torch.uint8)
+    x = torch.zeros(4, 256, dtype=torch.float32)
+    with pytest.raises(TypeError):
+        moe.moe_route(h, x, torch.zeros(16, 256), None, torch.zeros(4, 2, dtype=torch.int32),
+                      torch.zeros(4, 2), ws)

@@ -1,0 +1,205 @@
+"""GPU parity of every step of the CUDA path against the fp64 oracle, through the C ABI.
+
+Sizes span several tiles and ragged tails (rows not a multiple of the 128-row
+M tile, d_ff not a multiple of the 128-feature gate/up tile, d not a multiple
+of the 256-feature down tile, dispatch runs over more than one 4096-slot
+block) plus the degenerate cases (one token, one expert, k = E, no shared
+expert, every token on one expert, an empty expert).
+"""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_layer_47_b200 as moe
+import oracle
+from gpu_helpers import (Y_REL_TOL, dispatch_parity, gpu_forward, oracle_rows, rel_err,
+                         route_parity)
+from workloads import WORKLOADS, Inputs, make_inputs, make_small, to_device
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [  # T, d, E, k, F, S, bias_scale
+    (1, 64, 1, 1, 64, 0, 0.0),
+    (7, 128, 3, 2, 64, 1, 0.0),
+    (64, 256, 16, 2, 128, 1, 0.0),
+    (300, 192, 64, 8, 192, 1, 0.5),
+    (130, 320, 5, 3, 384, 2, 0.0),
+    (513, 512, 64, 8, 256, 1, 0.2),
+    (40, 256, 8, 8, 128, 1, 0.0),      # k == E
+]
+
+
+def _ids(shapes):
+    return ["T{}_d{}_E{}_k{}_F{}_S{}".format(*s[:6]) for s in shapes]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=_ids(SHAPES))
+def test_route_stage(shape):
+    T, d, E, k, F, S, bs = shape
+    inp = make_small(T, d, E, k, F, S, seed=100 + T, bias_scale=bs)
+    dev = to_device(inp, "cuda")
+    h = moe.moe_create(d, E, k, F, S)
+    ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    moe.moe_route(h, dev.x, dev.W_router, dev.bias, idx, w, ws)
+    torch.cuda.synchronize()
+    logits = oracle.router_logits(inp.x, inp.W_router, inp.bias)
+    route_parity(logits, idx.cpu().numpy(), w.cpu().numpy(), k)
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 1, 1), (5, 3, 2), (64, 16, 2), (700, 64, 8),
+                                   (1500, 256, 8), (2000, 1024, 32), (8192, 256, 8)])
+def test_dispatch_stage(T, E, k):
+    g = torch.Generator().manual_seed(T * 7 + E)
+    idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
+    h = moe.moe_create(64, E, k, 64, 1)
+    ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    pos = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    moe.moe_dispatch(h, idx.cuda(), counts, offsets, perm, pos, ws)
+    st, _ = moe.moe_device_status(h, T, ws)
+    assert st == moe.MOE_OK
+    dispatch_parity(idx.numpy(), E, counts.cpu(), offsets.cpu(), perm.cpu(), pos.cpu())
+
+
+def test_dispatch_flags_out_of_range_index():
+    T, E, k = 10, 8, 2
+    idx = torch.tensor([[e % E, (e + 1) % E] for e in range(T)], dtype=torch.int32)
+    idx[3, 1] = E          # out of range
+    idx[7, 0] = -1         # out of range
+    h = moe.moe_create(64, E, k, 64, 1)
+    ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
+    out = [torch.full((n,), -7, dtype=torch.int32, device="cuda")
+           for n in (E, E + 1, T * k, T * k)]
+    moe.moe_dispatch(h, idx.cuda(), *out, ws)
+    st, detail = moe.moe_device_status(h, T, ws)
+    assert st == moe.MOE_ERR_BAD_INDEX and (detail >> 16) == 2
+    counts = out[0].cpu().numpy()
+    valid = idx.numpy().reshape(-1)
+    valid = valid[(valid >= 0) & (valid < E)]
+    np.testing.assert_array_equal(counts, np.bincount(valid, minlength=E))
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=_ids(SHAPES))
+def test_expert_ffn_stage(shape):
+    """Y rows (and the bf16 SwiGLU activations) against the oracle, given the oracle's dispatch."""
+    T, d, E, k, F, S, bs = shape
+    inp = make_small(T, d, E, k, F, S, seed=200 + T, bias_scale=bs)
+    dev = to_device(inp, "cuda")
+    logits = oracle.router_logits(inp.x, inp.W_router, inp.bias)
+    idx, w, _ = oracle.route(logits, k)
+    counts, offsets, perm, pos = oracle.dispatch(idx, E)
+    h = moe.moe_create(d, E, k, F, S)
+    ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
+    rows = T * k + S * T
+    Y = torch.full((rows, d), float("nan"), dtype=torch.float32, device="cuda")
+    moe.moe_expert_ffn(h, dev.x, torch.from_numpy(perm).cuda(), torch.from_numpy(offsets).cuda(),
+                       dev.W_gate, dev.W_up, dev.W_down, dev.Ws_gate, dev.Ws_up, dev.Ws_down, Y,
+                       ws)
+    st, detail = moe.moe_device_status(h, T, ws)
+    assert st == moe.MOE_OK, hex(detail)
+    views = moe.workspace_views(h, T, ws)
+    H_ref, Y_ref = oracle_rows(inp, idx, perm)
+    Yg = Y.cpu().numpy()
+    Hg = views["h_act"].float().cpu().numpy()
+    Yr = np.stack([Y_ref[r] for r in range(rows)])
+    Hr = np.stack([H_ref[r] for r in range(rows)])
+    assert np.isfinite(Yg).all()
+    assert rel_err(Hg, Hr) < Y_REL_TOL, rel_err(Hg, Hr)
+    assert rel_err(Yg, Yr) < Y_REL_TOL, rel_err(Yg, Yr)
+
+
+@pytest.mark.parametrize("T,k,S,d", [(1, 1, 0, 64), (64, 2, 1, 256), (33, 8, 2, 6144)])
+def test_combine_stage(T, k, S, d):
+    g = torch.Generator().manual_seed(T + k)
+    rows = T * k + S * T
+    Y = torch.randn(rows, d, generator=g)
+    w = torch.rand(T, k, generator=g)
+    w = w / w.sum(1, keepdim=True)
+    pos = torch.randperm(T * k, generator=g).to(torch.int32)
+    h = moe.moe_create(d, max(k, 2), k, 64, S)
+    y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(h, Y.cuda(), w.cuda(), pos.cuda(), y)
+    torch.cuda.synchronize()
+    ref = oracle.combine(Y.double().numpy(), w.double().numpy(), pos.numpy(), T, k, S)
+    got = y.float().cpu().numpy()
+    # fp32 accumulation then one bf16 rounding: within 2^-8 relative of each element
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6)
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=_ids(SHAPES))
+def test_forward_matches_oracle(shape):
+    T, d, E, k, F, S, bs = shape
+    inp = make_small(T, d, E, k, F, S, seed=300 + T, bias_scale=bs)
+    y, v = gpu_forward(to_device(inp, "cuda"))
+    logits = oracle.router_logits(inp.x, inp.W_router, inp.bias)
+    exempt, idx_o, _ = route_parity(logits, v["topk_idx"].numpy(), v["topk_w"].numpy(), k)
+    dispatch_parity(v["topk_idx"].numpy(), E, v["counts"], v["offsets"], v["perm"], v["pos"])
+    # exempt (near-tie) tokens are compared with the oracle rerun on the GPU's routing
+    idx_use = np.where(exempt[:, None], v["topk_idx"].numpy(), idx_o)
+    ref = oracle.forward(inp, idx_override=idx_use)
+    assert rel_err(y.float().numpy(), ref["y"]) < Y_REL_TOL
+
+
+def test_forward_tiny_workload():
+    """The tiny workload (T=64, d=256, 16 experts top-2 + 1 shared, d_ff=128, seed 0)."""
+    inp = make_inputs(WORKLOADS["tiny"], device="cpu")
+    y, v = gpu_forward(to_device(inp, "cuda"))
+    ref = oracle.forward(inp)
+    exempt, _, _ = route_parity(ref["logits"], v["topk_idx"].numpy(), v["topk_w"].numpy(), 2)
+    if not exempt.any():
+        np.testing.assert_array_equal(v["offsets"].numpy(), ref["offsets"])
+        np.testing.assert_array_equal(v["perm"].numpy(), ref["perm"])
+    err = rel_err(y.float().numpy(), ref["y"])
+    assert err < Y_REL_TOL, err
+
+
+def test_every_token_on_one_expert_and_empty_experts():
+    """A dominant bias sends all 300 tokens to expert 3 (3 M tiles); most experts stay empty."""
+    T, d, E, k, F, S = 300, 128, 16, 2, 128, 1
+    inp = make_small(T, d, E, k, F, S, seed=9)
+    bias = torch.zeros(E)
+    bias[3] = 50.0
+    inp = Inputs(inp.wl, inp.x, inp.W_router, bias, inp.W_gate, inp.W_up, inp.W_down,
+                 inp.Ws_gate, inp.Ws_up, inp.Ws_down)
+    y, v = gpu_forward(to_device(inp, "cuda"))
+    assert int(v["counts"][3]) == T
+    assert int((v["counts"] == 0).sum()) >= 1
+    ref = oracle.forward(inp)
+    route_parity(ref["logits"], v["topk_idx"].numpy(), v["topk_w"].numpy(), k)
+    assert rel_err(y.float().numpy(), ref["y"]) < Y_REL_TOL
+
+
+def test_forward_is_deterministic_and_host_io_matches():
+    inp = to_device(make_small(200, 256, 32, 4, 128, 1, seed=5), "cuda")
+    wl = inp.wl
+    h = moe.moe_create(wl.d, wl.E, wl.k, wl.F, wl.S)
+    ws = torch.empty(moe.moe_workspace_size(h, wl.T), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(2):
+        y = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda")
+        moe.moe_forward(h, inp.x, inp.W_router, inp.bias, inp.W_gate, inp.W_up, inp.W_down,
+                        inp.Ws_gate, inp.Ws_up, inp.Ws_down, y, ws)
+        outs.append(y.cpu())
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    x_host = inp.x.cpu().pin_memory()
+    y_host = torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory()
+    moe.moe_forward_host(h, x_host, inp.W_router, inp.bias, inp.W_gate, inp.W_up, inp.W_down,
+                         inp.Ws_gate, inp.Ws_up, inp.Ws_down, y_host, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y_host.view(torch.int16), outs[0].view(torch.int16))
+
+
+def test_zero_tokens_is_a_no_op():
+    h = moe.moe_create(256, 16, 2, 128, 1)
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    x = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    W = make_small(1, 256, 16, 2, 128, 1)
+    dev = to_device(W, "cuda")
+    y = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    moe.moe_forward(h, x, dev.W_router, None, dev.W_gate, dev.W_up, dev.W_down, dev.Ws_gate,
+                    dev.Ws_up, dev.Ws_down, y, ws)
+    torch.cuda.synchronize()

@@ -57,6 +57,19 @@ def test_hand_worked_example():
     h, y = oracle.expert_one(inp.x[0], inp.W_gate[1], inp.W_up[1], inp.W_down[1])
     np.testing.assert_allclose(h, [_ev(v) for v in ex["h_token0_e1"]], rtol=1e-14)
     np.testing.assert_allclose(y, [_ev(v) for v in ex["y_token0_e1"]], rtol=1e-14)
+    # the combine step alone, fed the per-(slot, expert) rows in dispatch order
+    T, k, S = fx["T"], fx["k"], fx["S"]
+    rows = np.zeros((T * k + S * T, fx["d"]))
+    for p, s in enumerate(ex["perm"]):
+        t, i = divmod(s, k)
+        e = ex["idx"][t][i]
+        rows[p] = oracle.expert_one(inp.x[t], inp.W_gate[e], inp.W_up[e], inp.W_down[e])[1]
+    for t in range(T):
+        rows[T * k + t] = oracle.expert_one(inp.x[t], inp.Ws_gate[0], inp.Ws_up[0],
+                                            inp.Ws_down[0])[1]
+    yc = oracle.combine(rows, out["w"], out["pos"], T, k, S)
+    np.testing.assert_allclose(yc, [[_ev(v) for v in r] for r in ex["y"]], rtol=1e-14,
+                               atol=1e-15)
 
 
 def test_router_logits_equal_float64_matmul():
