@@ -32,7 +32,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import WORKLOADS, Workload, make_inputs  # noqa: E402
+from workloads import ALL_WORKLOADS, Workload, make_inputs  # noqa: E402
 
 DEFAULT_WORKLOAD = "decode"
 
@@ -136,6 +136,13 @@ def barrier(world: int):
         torch.distributed.barrier()
 
 
+def rank_batch(wl: Workload, rank: int) -> torch.Tensor:
+    """The token batch of a replica rank > 0 (rank 0 uses the workload's own x): every rank
+    holds the same weights and draws its own T tokens from seed + 1000 * rank."""
+    g = torch.Generator().manual_seed(wl.seed + 1000 * rank)
+    return torch.randn(wl.T, wl.d, generator=g).to(torch.bfloat16)
+
+
 def max_over_ranks(value: float, world: int, device) -> float:
     if world == 1:
         return value
@@ -174,6 +181,25 @@ def algorithmic_work(wl: Workload, counts: np.ndarray) -> dict:
     }
 
 
+def measured_traffic(kernel: str, bound: str, units: int):
+    """DRAM bytes per launch of ``kernel`` scaled from the committed ncu capture
+    (profiles/traffic.json), or None when there is none or the kernel source has
+    changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        entry = json.load(f).get(kernel)
+    if not entry or entry.get("bound") != bound:
+        return None
+    src = os.path.join(ROOT, "mixture_experts_layer_47_b200", "csrc", "expert_gemm.cu")
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != entry["kernel_source_sha256"]:
+            return None
+    return int(entry["bytes_per_touched_expert"] * units)
+
+
 def hbm_bound(wl: Workload, work: dict, peaks: dict) -> bool:
     """Arithmetic intensity of the gate/up GEMM against the machine balance."""
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
@@ -188,12 +214,10 @@ def run_ours(args, rank, local, world):
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    wl = WORKLOADS[args.workload]
+    wl = ALL_WORKLOADS[args.workload]
     inp = make_inputs(wl, device=device)
-    if world > 1 and rank > 0:
-        # every rank holds the same weights (one replica each) and its own batch of tokens
-        g = torch.Generator().manual_seed(wl.seed + 1000 * rank)
-        inp.x = torch.randn(wl.T, wl.d, generator=g).to(torch.bfloat16).to(device)
+    if rank > 0:
+        inp.x = rank_batch(wl, rank).to(device)
     h = moe.moe_create(wl.d, wl.E, wl.k, wl.F, wl.S)
     ws = torch.empty(moe.moe_workspace_size(h, wl.T), dtype=torch.uint8, device=device)
     y = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=device)
@@ -282,7 +306,8 @@ def run_ours(args, rank, local, world):
         peak = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4)}
-    roof.update({"kernel": dominant, "traffic": None, "peak_source": peaks["source"],
+    traffic = measured_traffic(dominant, roof["bound"], work["touched_experts"] + wl.S)
+    roof.update({"kernel": dominant, "traffic": traffic, "peak_source": peaks["source"],
                  "algorithmic_per_launch": work[key + ("_bytes" if roof["bound"] == "hbm"
                                                        else "_flops")],
                  "launch_ms": round(dom_ms, 4)})
@@ -379,7 +404,7 @@ def run_reference(args, rank, local, world):
     if rank != 0:
         return
     import oracle
-    wl = WORKLOADS[args.workload]
+    wl = ALL_WORKLOADS[args.workload]
     device = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     inp = make_inputs(wl, device=device)
     tokens = _sample_tokens(wl)
@@ -416,7 +441,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ALL_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()

@@ -158,16 +158,18 @@ def test_forward_tiny_workload():
 
 
 def test_every_token_on_one_expert_and_empty_experts():
-    """A dominant bias sends all 300 tokens to expert 3 (3 M tiles); most experts stay empty."""
+    """Dominant biases send all 300 tokens to experts 3 and 7 (3 M tiles each); the other
+    14 experts stay empty."""
     T, d, E, k, F, S = 300, 128, 16, 2, 128, 1
     inp = make_small(T, d, E, k, F, S, seed=9)
     bias = torch.zeros(E)
     bias[3] = 50.0
+    bias[7] = 40.0
     inp = Inputs(inp.wl, inp.x, inp.W_router, bias, inp.W_gate, inp.W_up, inp.W_down,
                  inp.Ws_gate, inp.Ws_up, inp.Ws_down)
     y, v = gpu_forward(to_device(inp, "cuda"))
-    assert int(v["counts"][3]) == T
-    assert int((v["counts"] == 0).sum()) >= 1
+    assert int(v["counts"][3]) == T and int(v["counts"][7]) == T
+    assert int((v["counts"] == 0).sum()) == E - 2
     ref = oracle.forward(inp)
     route_parity(ref["logits"], v["topk_idx"].numpy(), v["topk_w"].numpy(), k)
     assert rel_err(y.float().numpy(), ref["y"]) < Y_REL_TOL

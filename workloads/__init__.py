@@ -83,6 +83,19 @@ WORKLOADS = {
                     "calibrated so expert popularity follows Zipf s=1.2"),
 }
 
+# Reduced cases of the same kernels for profiler captures that must stay a few GB on the
+# device: the Hy4 hidden and expert widths with 32 routed experts (2.4 GB of weights).
+PROFILE_WORKLOADS = {
+    "profile_decode_e32": Workload(
+        "profile_decode_e32", T=16, d=6144, E=32, k=8, F=2048, S=1, router="normal", seed=0,
+        description="decode-shaped profiling case: T=16, d=6144, 32 experts top-8 + 1 shared"),
+    "profile_prefill_e32": Workload(
+        "profile_prefill_e32", T=1024, d=6144, E=32, k=8, F=2048, S=1, router="uniform", seed=0,
+        description="prefill-shaped profiling case: T=1024 (256 rows per expert), d=6144, "
+                    "32 experts top-8 + 1 shared"),
+}
+ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS}
+
 
 def zipf_bias_path(wl: Workload) -> str:
     return os.path.join(
