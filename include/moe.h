@@ -206,6 +206,31 @@ moe_status moe_device_status(moe_handle h, int T, const void *workspace, void *s
 #define MOE_STAGE_EVENTS 7
 moe_status moe_set_stage_events(moe_handle h, void *const *events, int n_events);
 
+/*
+ * moe_dispatch without a workspace, for callers that cannot allocate device
+ * memory -- for example a plug-in inside a host application that owns every
+ * device allocation through its own pool, or a latency-critical loop where a
+ * cudaMalloc (which can synchronise the device) is not allowed.  (The pages
+ * describe the layer only; they have no counterpart to this entry point.)
+ * Same arguments and results as moe_dispatch, minus the workspace: the
+ * scratch it needs (per-block histograms, the GEMM tile schedule, a status
+ * word) lives in a fixed array of about 70 KB compiled into the library,
+ * which every GPU that loads the library keeps until the process exits.
+ * Limits: T * k <= 65536 slots and E <= 1024; larger calls return
+ * MOE_ERR_WORKSPACE and enqueue nothing.  It allocates nothing: no
+ * cudaMalloc / cudaFree or allocating library routine.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any
+ * stream capture.  All calls share the one array and it keeps the last
+ * call's contents (each call clears what must start at zero), so calls that
+ * overlap on the GPU -- on different streams without ordering between them
+ * -- race and corrupt each other's results.  Out-of-range expert indices are
+ * skipped as in moe_dispatch, but the status word is not readable through
+ * this entry point.
+ */
+moe_status moe_dispatch_noalloc(moe_handle h, const int32_t *topk_idx, int T, int32_t *counts,
+                                int32_t *offsets, int32_t *perm, int32_t *pos, void *stream);
+
 /* Static text for a status code. */
 const char *moe_status_string(moe_status s);
 

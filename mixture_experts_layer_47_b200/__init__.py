@@ -36,7 +36,7 @@ MOE_ERR_ALIGNMENT = 7
 EXPORTS = ("moe_create", "moe_destroy", "moe_workspace_size", "moe_get_workspace_layout",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_host", "moe_device_status", "moe_set_stage_events",
-           "moe_status_string")
+           "moe_dispatch_noalloc", "moe_status_string")
 MOE_STAGE_EVENTS = 7
 STAGE_NAMES = ("router", "dispatch", "gather", "gate_up_gemm", "down_gemm", "combine")
 
@@ -80,6 +80,7 @@ def load_library() -> ctypes.CDLL:
         "moe_forward_host": ([P, P, P, P, P, P, P, P, P, P, I, P, P, Z, P], I),
         "moe_device_status": ([P, I, P, P, ctypes.POINTER(ctypes.c_int32)], I),
         "moe_set_stage_events": ([P, ctypes.POINTER(P), I], I),
+        "moe_dispatch_noalloc": ([P, P, I, P, P, P, P, P], I),
         "moe_status_string": ([I], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -197,6 +198,19 @@ def moe_dispatch(h: Handle, topk_idx, counts, offsets, perm, pos, workspace, str
         _ptr(offsets, torch.int32, "offsets", (h.E + 1,)),
         _ptr(perm, torch.int32, "perm", (n,)), _ptr(pos, torch.int32, "pos", (n,)), wp, wn,
         _stream(stream)), "moe_dispatch")
+
+
+def moe_dispatch_noalloc(h: Handle, topk_idx, counts, offsets, perm, pos, stream=None) -> None:
+    """moe_dispatch without a workspace, for callers that cannot allocate device memory
+    (the library's fixed scratch is used instead; see include/moe.h for its limits)."""
+    T = topk_idx.shape[0]
+    n = T * h.k
+    _check(load_library().moe_dispatch_noalloc(
+        h.value, _ptr(topk_idx, torch.int32, "topk_idx", (T, h.k)), T,
+        _ptr(counts, torch.int32, "counts", (h.E,)),
+        _ptr(offsets, torch.int32, "offsets", (h.E + 1,)),
+        _ptr(perm, torch.int32, "perm", (n,)), _ptr(pos, torch.int32, "pos", (n,)),
+        _stream(stream)), "moe_dispatch_noalloc")
 
 
 def _weights(h: Handle, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down):

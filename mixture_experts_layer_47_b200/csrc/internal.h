@@ -43,6 +43,8 @@ struct DeviceInfo {
   bool ready = false;
 };
 moe_status ensure_device(DeviceInfo** out);
+// The layer shape a context was created with.
+moe_status moe_internal_shape(moe_handle h, Ctx* out);
 
 // ---- launchers (each returns cudaSuccess or the launch error) ----
 cudaError_t launch_router(const Ctx& c, const RouterPlan& rp, const uint16_t* x, const float* Wr,

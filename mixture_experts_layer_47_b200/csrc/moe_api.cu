@@ -121,6 +121,12 @@ moe_status ensure_device(DeviceInfo** out) {
   return MOE_OK;
 }
 
+moe_status moe_internal_shape(moe_handle h, Ctx* out) {
+  if (!h || !out) return MOE_ERR_INVALID_ARG;
+  *out = h->c;
+  return MOE_OK;
+}
+
 }  // namespace moe
 
 using namespace moe;
