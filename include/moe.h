@@ -97,7 +97,7 @@ typedef struct {
     size_t perm;      /* int32 [T*k]                                         */
     size_t pos;       /* int32 [T*k]                                         */
     size_t h_act;     /* bf16  [T*k + S*T][F]  SwiGLU activations            */
-    size_t y_rows;    /* fp32  [T*k + S*T][d]  per-(slot, expert) outputs    */
+    size_t y_rows;    /* bf16  [T*k + S*T][d]  per-(slot, expert) outputs    */
     size_t total;     /* bytes used, including the alignment slack           */
 } moe_workspace_layout;
 moe_status moe_get_workspace_layout(moe_handle h, int T, uintptr_t workspace_addr,
@@ -164,7 +164,10 @@ moe_status moe_combine(moe_handle h, const float *Y, const float *topk_w, const 
 /*
  * The whole layer: moe_route, moe_dispatch, moe_expert_ffn and moe_combine
  * in one call, intermediates kept in the workspace (moe_get_workspace_layout).
- * Arguments as in those calls; y: bf16 [T][d] (output).
+ * Arguments as in those calls; y: bf16 [T][d] (output).  One difference from
+ * chaining the four calls: the per-(slot, expert) rows Y are kept in bf16
+ * (rounded once from the fp32 accumulator) instead of fp32, halving their
+ * write and read; the combine still sums in fp32.
  */
 moe_status moe_forward(moe_handle h, const uint16_t *x, const float *W_router, const float *bias,
                        const uint16_t *W_gate, const uint16_t *W_up, const uint16_t *W_down,
@@ -214,7 +217,7 @@ moe_status moe_set_stage_events(moe_handle h, void *const *events, int n_events)
  * describe the layer only; they have no counterpart to this entry point.)
  * Same arguments and results as moe_dispatch, minus the workspace: the
  * scratch it needs (per-block histograms, the GEMM tile schedule, a status
- * word) lives in a fixed array of about 70 KB compiled into the library,
+ * word) lives in a fixed array of about 74 KB compiled into the library,
  * which every GPU that loads the library keeps until the process exits.
  * Limits: T * k <= 65536 slots and E <= 1024; larger calls return
  * MOE_ERR_WORKSPACE and enqueue nothing.  It allocates nothing: no

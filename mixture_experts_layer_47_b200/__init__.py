@@ -313,7 +313,7 @@ def workspace_views(h: Handle, T: int, workspace: torch.Tensor) -> dict:
         perm=view(L["perm"], T * h.k, torch.int32),
         pos=view(L["pos"], T * h.k, torch.int32),
         h_act=view(L["h_act"], rows * h.F, torch.bfloat16).view(rows, h.F),
-        y_rows=view(L["y_rows"], rows * h.d, torch.float32).view(rows, h.d),
+        y_rows=view(L["y_rows"], rows * h.d, torch.bfloat16).view(rows, h.d),
     )
 
 

@@ -14,6 +14,8 @@
 //                     __match_any_sync gives each slot its rank among equal
 //                     experts in the warp; per-warp, per-expert running
 //                     counts make the order ascending in slot index.
+// Up to 4096 slots and 256 experts the three steps run in one CTA
+// (dispatch_single).
 #include "common.cuh"
 #include "internal.h"
 
@@ -71,16 +73,23 @@ __device__ int block_inclusive_scan(int v, int* warp_sums) {
   return r;
 }
 
-// Grouped-GEMM schedule: sched[g] = sum over groups g' < g of ceil(rows_g' / 128),
-// routed groups first (rows = count), then S shared groups of T rows each.
+// Grouped-GEMM schedules: sched[g] = sum over groups g' < g of ceil(rows_g' / 128),
+// routed groups first (rows = count), then S shared groups of T rows each; the
+// same for 256-row tiles (the 2-SM GEMM) at sched[G + 1 + g], G = E + S.
 __device__ void write_schedule(int count, int E, int S, int T, int32_t* sched, int* warp_sums) {
   const int e = threadIdx.x;
-  const int mt = (e < E) ? (count + kTileM - 1) / kTileM : 0;
-  const int incl = block_inclusive_scan(mt, warp_sums);
-  if (e < E) sched[e] = incl - mt;
-  if (e == E - 1) {
-    const int mts = (T + kTileM - 1) / kTileM;
-    for (int s = 0; s <= S; ++s) sched[E + s] = incl + s * mts;
+  const int G1 = E + S + 1;
+#pragma unroll
+  for (int which = 0; which < 2; ++which) {
+    const int tm = which == 0 ? kTileM : 2 * kTileM;
+    int32_t* out = sched + which * G1;
+    const int mt = (e < E) ? (count + tm - 1) / tm : 0;
+    const int incl = block_inclusive_scan(mt, warp_sums);
+    if (e < E) out[e] = incl - mt;
+    if (e == E - 1) {
+      const int mts = (T + tm - 1) / tm;
+      for (int s = 0; s <= S; ++s) out[E + s] = incl + s * mts;
+    }
   }
 }
 
@@ -171,12 +180,89 @@ __global__ void __launch_bounds__(kScatterWarps * 32)
   }
 }
 
+// Small dispatches (n <= 4096 slots, E <= 256) in one CTA of 1024 threads:
+// per-warp counts (as in dispatch_scatter), then per expert the prefix over
+// warps and the totals, the exclusive scan over experts and the schedules,
+// then the stable scatter.  One launch instead of three.
+constexpr int kSingleWarps = kScanThreads / 32;
+constexpr int kSingleMaxExperts = 256;
+
+__global__ void __launch_bounds__(kScanThreads)
+    dispatch_single_kernel(const int32_t* __restrict__ idx, int n, int E, int S, int T,
+                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                           int32_t* __restrict__ perm, int32_t* __restrict__ pos,
+                           int32_t* __restrict__ sched, int* status) {
+  extern __shared__ int32_t cnt[];  // [kSingleWarps][E]
+  __shared__ int warp_sums[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kSingleWarps * E; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  constexpr int kPerWarp = kDispatchChunk / kSingleWarps;
+  const int beg = warp * kPerWarp;
+  const int end = min(n, beg + kPerWarp);
+  int32_t* my = cnt + warp * E;
+  bool bad = false;
+  for (int s0 = beg; s0 < end; s0 += 32) {
+    const int s = s0 + lane;
+    int e = (s < end) ? idx[s] : -1;
+    if (s < end && (e < 0 || e >= E)) bad = true;
+    if (e < 0 || e >= E) e = -1;
+    const unsigned m = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(m) - 1) my[e] += __popc(m);
+    __syncwarp();
+  }
+  if (bad) report_error(status, kDevBadIndex, kSiteDispatch);
+  __syncthreads();
+  const int e = threadIdx.x;
+  int c = 0;
+  if (e < E) {
+    int run = 0;
+    for (int w = 0; w < kSingleWarps; ++w) {
+      const int v = cnt[w * E + e];
+      cnt[w * E + e] = run;
+      run += v;
+    }
+    c = run;
+    counts[e] = c;
+  }
+  const int incl = block_inclusive_scan(c, warp_sums);
+  const int excl = incl - c;
+  if (e < E) {
+    offsets[e] = excl;
+    for (int w = 0; w < kSingleWarps; ++w) cnt[w * E + e] += excl;
+  }
+  if (e == E - 1) offsets[E] = incl;
+  write_schedule(c, E, S, T, sched, warp_sums);
+  __syncthreads();
+  for (int s0 = beg; s0 < end; s0 += 32) {
+    const int s = s0 + lane;
+    int e2 = (s < end) ? idx[s] : -1;
+    if (e2 < 0 || e2 >= E) e2 = -1;
+    const unsigned m = __match_any_sync(0xffffffffu, e2);
+    const int rank = __popc(m & ((1u << lane) - 1u));
+    const int base = (e2 >= 0) ? my[e2] : 0;
+    __syncwarp();
+    if (e2 >= 0) {
+      const int p = base + rank;
+      perm[p] = s;
+      pos[s] = p;
+      if (lane == __ffs(m) - 1) my[e2] = base + __popc(m);
+    }
+    __syncwarp();
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_dispatch(const Ctx& c, const int32_t* topk_idx, int T, int nblk,
                             int32_t* blk_hist, int32_t* counts, int32_t* offsets, int32_t* perm,
                             int32_t* pos, int32_t* sched, int* status, cudaStream_t st) {
   const int n = T * c.k;
+  if (n <= kDispatchChunk && c.E <= kSingleMaxExperts) {
+    dispatch_single_kernel<<<1, kScanThreads, kSingleWarps * c.E * sizeof(int32_t), st>>>(
+        topk_idx, n, c.E, c.S, T, counts, offsets, perm, pos, sched, status);
+    return cudaGetLastError();
+  }
   dispatch_count_kernel<<<nblk, kCountThreads, c.E * sizeof(int32_t), st>>>(topk_idx, n, c.E,
                                                                             blk_hist, status);
   cudaError_t err = cudaGetLastError();

@@ -11,7 +11,7 @@
 // library instead of a workspace.
 //
 // The scratch is a file-scope __device__ array: every GPU on which the
-// library's kernels are loaded holds its own copy (about 70 KB) until the
+// library's kernels are loaded holds its own copy (about 74 KB) until the
 // process exits.  Host code cannot use the array's name as a device pointer;
 // the device address is obtained once per device with cudaGetSymbolAddress
 // (on the first call made with that device current) and cached.
@@ -32,7 +32,7 @@ constexpr int kNoAllocMaxBlocks = kNoAllocMaxSlots / kDispatchChunk;  // 16
 constexpr int kNoAllocMaxExperts = 1024;
 constexpr int kStatusInts = 64;  // status word, padded to 256 bytes
 constexpr int kHistInts = kNoAllocMaxBlocks * kNoAllocMaxExperts;
-constexpr int kSchedInts = kNoAllocMaxExperts + 8 + 1 + 63;  // E + S + 1, padded
+constexpr int kSchedInts = 2 * (kNoAllocMaxExperts + 8 + 1) + 62;  // two schedules, padded
 constexpr int kScratchInts = kStatusInts + kHistInts + kSchedInts;
 
 static __device__ __align__(256) int32_t g_dispatch_scratch[kScratchInts];

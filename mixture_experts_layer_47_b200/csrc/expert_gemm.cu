@@ -25,6 +25,9 @@
 // its own copies and MMAs, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
+#include <stdlib.h>
+#include <string.h>
+
 #include <algorithm>
 #include <mutex>
 
@@ -34,18 +37,27 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
 constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int A_TILE_BYTES = BM * BK * 2;
-constexpr int B_TILE_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_TILE_BYTES + B_TILE_BYTES;
+constexpr int BN = 256;                // MMA N: output features of a tile (gate|up halves or down)
+constexpr int A_TILE_BYTES = 128 * BK * 2;
 constexpr int NUM_THREADS = 192;
-constexpr int ACC_COLS = BN;           // fp32 columns per accumulator
+constexpr int ACC_COLS = BN;           // fp32 TMEM columns per accumulator
 constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int MAX_GROUPS = 1024 + 8;   // E + S upper bound
-constexpr uint32_t IDESC = umma_idesc_bf16_f32(BM, BN);
+
+// kPair = false: one CTA computes a 128 x 256 tile (tcgen05 M=128), loading all 256 B rows.
+// kPair = true:  a cluster of two CTAs computes a 256 x 256 tile with the 2-SM MMA
+//                (M=256); each CTA loads its own 128 A rows and 128 of the 256 B rows,
+//                so each weight byte read from HBM feeds 256 token rows.
+template <bool kPair>
+struct Cfg {
+  static constexpr int TILE_M = kPair ? 256 : 128;
+  static constexpr int B_ROWS = kPair ? 128 : 256;  // B rows held by one CTA
+  static constexpr int B_TILE_BYTES = B_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = A_TILE_BYTES + B_TILE_BYTES;
+  static constexpr int STAGES = kPair ? 6 : 4;
+  static constexpr uint32_t IDESC = umma_idesc_bf16_f32(TILE_M, BN);
+};
 
 struct __align__(64) GemmParams {
   CUtensorMap a_routed;  // gate/up: X_perm [T*k][d]; down: H [T*k+S*T][F]
@@ -55,9 +67,10 @@ struct __align__(64) GemmParams {
   CUtensorMap s0;        // shared counterparts of b0 / b1
   CUtensorMap s1;
   const int32_t* offsets;  // [E+1]
-  const int32_t* sched;    // [E+S+1] prefix sums of M-tiles per group
-  void* out;               // gate/up: H bf16; down: Y fp32
+  const int32_t* sched;    // [E+S+1] prefix sums of M tiles (of TILE_M rows) per group
+  void* out;               // gate/up: H bf16; down: Y fp32, or bf16 when out_bf16
   int* status;
+  int out_bf16;            // down only: store Y rounded to bf16
   int T, E, S, k;
   int K;          // reduction length (d or F)
   int n_out;      // output features per group (F or d)
@@ -66,8 +79,8 @@ struct __align__(64) GemmParams {
 };
 
 struct SharedStorage {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[6];
+  uint64_t empty[6];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t mma_done;
@@ -77,21 +90,25 @@ struct SharedStorage {
   int offsets[MAX_GROUPS + 1];
 };
 
-constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + size_t(STAGES) * STAGE_BYTES +
-                              sizeof(SharedStorage);
+template <bool kPair>
+constexpr size_t smem_bytes() {
+  return 1024 /*alignment slack*/ + size_t(Cfg<kPair>::STAGES) * Cfg<kPair>::STAGE_BYTES +
+         sizeof(SharedStorage);
+}
 
 struct Tile {
   int g, m_idx, n_idx;
   int rows;      // valid rows of group g
-  int a_row;     // first A row of this tile
+  int a_row;     // first A row of this tile (pair: of the pair's 256 rows)
   int out_row;   // first output row of this tile
-  int b_row;     // first weight row (in the per-group B map) of this tile
+  int b_row;     // first weight row (in the per-group B maps) of this tile
   bool shared;
 };
 
-template <bool kGateUp>
+template <bool kGateUp, bool kPair>
 __device__ __forceinline__ Tile decode_tile(int t, int n_tiles, int G, const SharedStorage& ss,
                                             const GemmParams& p) {
+  constexpr int TM = Cfg<kPair>::TILE_M;
   const int q = t / n_tiles;
   int lo = 0, hi = G;  // largest g in [0, G) with sched[g] <= q
   while (hi - lo > 1) {
@@ -109,44 +126,49 @@ __device__ __forceinline__ Tile decode_tile(int t, int n_tiles, int G, const Sha
   if (lo < p.E) {
     tl.shared = false;
     tl.rows = ss.offsets[lo + 1] - ss.offsets[lo];
-    tl.a_row = ss.offsets[lo] + tl.m_idx * BM;
+    tl.a_row = ss.offsets[lo] + tl.m_idx * TM;
     tl.out_row = tl.a_row;
     tl.b_row = lo * p.b_rows + tl.n_idx * kOutCols;
   } else {
     const int s = lo - p.E;
     tl.shared = true;
     tl.rows = p.T;
-    tl.out_row = nslots + s * p.T + tl.m_idx * BM;
-    tl.a_row = kGateUp ? tl.m_idx * BM : tl.out_row;
+    tl.out_row = nslots + s * p.T + tl.m_idx * TM;
+    tl.a_row = kGateUp ? tl.m_idx * TM : tl.out_row;
     tl.b_row = s * p.b_rows + tl.n_idx * kOutCols;
   }
   return tl;
 }
 
-template <bool kGateUp>
+template <bool kGateUp, bool kPair>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
+  using C = Cfg<kPair>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_TILE_BYTES;
-  SharedStorage& ss = *reinterpret_cast<SharedStorage*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* sB = smem + C::STAGES * A_TILE_BYTES;
+  SharedStorage& ss = *reinterpret_cast<SharedStorage*>(smem + C::STAGES * C::STAGE_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = p.E + p.S;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;   // CTA rank inside the pair
+  const bool leader = rank == 0;
+  const int unit = kPair ? int(blockIdx.x >> 1) : int(blockIdx.x);        // this pair / CTA
+  const int n_units = kPair ? int(gridDim.x >> 1) : int(gridDim.x);
 
   for (int i = threadIdx.x; i <= G; i += NUM_THREADS) ss.sched[i] = p.sched[i];
   for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) ss.offsets[i] = p.offsets[i];
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&ss.full[s], 1);
       mbar_init(&ss.empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&ss.tmem_full[a], 1);
-      mbar_init(&ss.tmem_empty[a], 128);
+      mbar_init(&ss.tmem_empty[a], kPair ? 256 : 128);
     }
     mbar_init(&ss.mma_done, 1);
     ss.abort_flag = 0;
@@ -163,11 +185,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(&ss.tmem_base, TMEM_COLS);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(&ss.tmem_base, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&ss.tmem_base, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (kPair) cluster_sync_all(); else __syncthreads();   // barriers of both CTAs initialised
   tc_fence_after();
   const uint32_t tmem_base = ss.tmem_base;
 
@@ -176,66 +203,81 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int total = ss.sched[G] * n_tiles;
   const int kblocks = p.K / BK;
   volatile int* abort_flag = &ss.abort_flag;
+  bool aborted = false;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (both CTAs of a pair load their own halves) ----------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        if (*abort_flag) break;
-        const Tile tl = decode_tile<kGateUp>(t, n_tiles, G, ss, p);
+      for (int t = unit; t < total && !aborted; t += n_units) {
+        if (*abort_flag) { aborted = true; break; }
+        const Tile tl = decode_tile<kGateUp, kPair>(t, n_tiles, G, ss, p);
         const CUtensorMap* mA = tl.shared ? &p.a_shared : &p.a_routed;
         const CUtensorMap* mB0 = tl.shared ? &p.s0 : &p.b0;
         const CUtensorMap* mB1 = tl.shared ? &p.s1 : &p.b1;
+        const int a_row = tl.a_row + int(rank) * 128;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&ss.empty[stage], phase ^ 1)) {
             report_error(p.status, kDevTimeout, kSiteProducer);
             *abort_flag = 1;
-            ok = false;
+            aborted = true;
             break;
           }
-          mbar_arrive_expect_tx(&ss.full[stage], STAGE_BYTES);
+          uint8_t* dA = sA + stage * A_TILE_BYTES;
+          uint8_t* dB = sB + stage * C::B_TILE_BYTES;
           const int kc = kb * BK;
-          tma_load_2d_nohint(sA + stage * A_TILE_BYTES, mA, &ss.full[stage], kc, tl.a_row);
-          if (kGateUp) {
-            uint8_t* dst = sB + stage * B_TILE_BYTES;
-            tma_load_2d_nohint(dst, mB0, &ss.full[stage], kc, tl.b_row);
-            tma_load_2d_nohint(dst + B_TILE_BYTES / 2, mB1, &ss.full[stage], kc, tl.b_row);
+          if (kPair) {
+            // The leader's full barrier counts the bytes of both CTAs' loads.
+            const uint32_t bar = mapa_shared(smem_u32(&ss.full[stage]), 0);
+            if (leader) mbar_arrive_expect_tx(&ss.full[stage], 2 * C::STAGE_BYTES);
+            tma_load_2d_pair(dA, mA, bar, kc, a_row);
+            if (kGateUp)   // CTA 0 holds the gate rows, CTA 1 the matching up rows
+              tma_load_2d_pair(dB, rank == 0 ? mB0 : mB1, bar, kc, tl.b_row);
+            else           // CTA r holds W_down rows [b_row + 128 r, b_row + 128 r + 128)
+              tma_load_2d_pair(dB, mB0, bar, kc, tl.b_row + int(rank) * 128);
           } else {
-            tma_load_2d_nohint(sB + stage * B_TILE_BYTES, mB0, &ss.full[stage], kc, tl.b_row);
+            mbar_arrive_expect_tx(&ss.full[stage], C::STAGE_BYTES);
+            tma_load_2d_nohint(dA, mA, &ss.full[stage], kc, a_row);
+            if (kGateUp) {
+              tma_load_2d_nohint(dB, mB0, &ss.full[stage], kc, tl.b_row);
+              tma_load_2d_nohint(dB + C::B_TILE_BYTES / 2, mB1, &ss.full[stage], kc, tl.b_row);
+            } else {
+              tma_load_2d_nohint(dB, mB0, &ss.full[stage], kc, tl.b_row);
+            }
           }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
-      // Drain: every load this thread issued must have landed before the CTA
-      // may exit (normally they all have: the MMA warp consumed them).
-      for (int s = 0; s < STAGES; ++s)
-        if (issued_mask & (1u << s))
-          if (!mbar_wait(&ss.full[s], (issued_parity >> s) & 1u, kDrainTimeoutNs))
-            report_error(p.status, kDevTimeout, kSiteDrain);
+      // Drain: loads counted on this CTA's own full barriers must have landed
+      // before the CTA may exit (in the normal path the MMA consumed them all).
+      if (!kPair || leader) {
+        for (int s = 0; s < C::STAGES; ++s)
+          if (issued_mask & (1u << s))
+            if (!mbar_wait(&ss.full[s], (issued_parity >> s) & 1u, kDrainTimeoutNs))
+              report_error(p.status, kDevTimeout, kSiteDrain);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
+    // ---------------- MMA issuer (the pair's leader only) ----------------
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        if (*abort_flag) break;
+      for (int t = unit; t < total && !aborted; t += n_units) {
+        if (*abort_flag) { aborted = true; break; }
         if (!mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1)) {
           report_error(p.status, kDevTimeout, kSiteMma);
           *abort_flag = 1;
+          aborted = true;
           break;
         }
         tc_fence_after();
@@ -244,31 +286,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!mbar_wait(&ss.full[stage], phase)) {
             report_error(p.status, kDevTimeout, kSiteMma);
             *abort_flag = 1;
-            ok = false;
+            aborted = true;
             break;
           }
           tc_fence_after();
           const uint64_t a_desc = umma_desc_sw128_kmajor(smem_u32(sA + stage * A_TILE_BYTES));
-          const uint64_t b_desc = umma_desc_sw128_kmajor(smem_u32(sB + stage * B_TILE_BYTES));
+          const uint64_t b_desc = umma_desc_sw128_kmajor(smem_u32(sB + stage * C::B_TILE_BYTES));
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16(d_tmem, a_desc + uint64_t(2 * kk), b_desc + uint64_t(2 * kk), IDESC,
-                      (kb | kk) != 0 ? 1u : 0u);
-          umma_commit(&ss.empty[stage]);
-          if (++stage == STAGES) {
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            if (kPair)
+              umma_bf16_pair(d_tmem, a_desc + uint64_t(2 * kk), b_desc + uint64_t(2 * kk),
+                             C::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            else
+              umma_bf16(d_tmem, a_desc + uint64_t(2 * kk), b_desc + uint64_t(2 * kk), C::IDESC,
+                        (kb | kk) != 0 ? 1u : 0u);
+          }
+          if (kPair) umma_commit_pair(&ss.empty[stage], 0x3); else umma_commit(&ss.empty[stage]);
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
-        if (!ok) break;
-        umma_commit(&ss.tmem_full[acc]);
+        if (aborted) break;
+        if (kPair) umma_commit_pair(&ss.tmem_full[acc], 0x3); else umma_commit(&ss.tmem_full[acc]);
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1;
         }
       }
       // Drain: wait until every MMA issued here has completed.
-      umma_commit(&ss.mma_done);
+      if (kPair) umma_commit_pair(&ss.mma_done, 0x1); else umma_commit(&ss.mma_done);
       if (!mbar_wait(&ss.mma_done, 0, kDrainTimeoutNs))
         report_error(p.status, kDevTimeout, kSiteDrain);
     }
@@ -276,21 +323,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------- epilogue (warps 2..5, one accumulator row per thread) --------
     const int quarter = warp & 3;               // TMEM lanes [32*quarter, 32*quarter+32)
-    const int row_in_tile = quarter * 32 + lane;
+    const int row_in_cta = quarter * 32 + lane;
     const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      if (*abort_flag) break;
-      const Tile tl = decode_tile<kGateUp>(t, n_tiles, G, ss, p);
+    for (int t = unit; t < total; t += n_units) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) { aborted = true; break; }  // warp-uniform
+      const Tile tl = decode_tile<kGateUp, kPair>(t, n_tiles, G, ss, p);
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&ss.tmem_full[acc], acc_phase));
       if (!ok) {
         if (lane == 0) report_error(p.status, kDevTimeout, kSiteEpilogue);
         *abort_flag = 1;
+        aborted = true;
         break;
       }
       tc_fence_after();
-      const int r = tl.m_idx * BM + row_in_tile;
+      const int row_in_tile = int(rank) * 128 + row_in_cta;
+      const int r = tl.m_idx * C::TILE_M + row_in_tile;
       const int out_row = tl.out_row + row_in_tile;
       const bool valid = r < tl.rows && out_row >= 0 && out_row < p.out_rows;
       const uint32_t tbase = tmem_base + lane_addr + uint32_t(acc * ACC_COLS);
@@ -321,7 +370,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       } else {
-        float* Y = reinterpret_cast<float*>(p.out);
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t v[32];
@@ -329,16 +377,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_ld_wait();
           const int col0 = tl.n_idx * BN + c;
           if (valid && col0 < p.n_out) {
-            float4* dst = reinterpret_cast<float4*>(Y + size_t(out_row) * p.n_out + col0);
+            if (p.out_bf16) {
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) +
+                                                    size_t(out_row) * p.n_out + col0);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+              for (int j = 0; j < 4; ++j)
+                dst[j] = make_uint4(
+                    pack_bf16x2(__uint_as_float(v[8 * j]), __uint_as_float(v[8 * j + 1])),
+                    pack_bf16x2(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3])),
+                    pack_bf16x2(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5])),
+                    pack_bf16x2(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7])));
+            } else {
+              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) +
+                                                      size_t(out_row) * p.n_out + col0);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                dst[j] =
+                    make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+            }
           }
         }
       }
       tc_fence_before();
-      mbar_arrive(&ss.tmem_empty[acc]);
+      if (kPair)
+        mbar_arrive_cluster(mapa_shared(smem_u32(&ss.tmem_empty[acc]), 0));
+      else
+        mbar_arrive(&ss.tmem_empty[acc]);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -346,11 +411,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
 
+  if (kPair && aborted) {
+    // A CTA of a pair cannot observe its own loads' completion (they are
+    // counted on the leader's barrier): give copies in flight time to land.
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 100000ull) {
+    }
+  }
   tc_fence_before();
-  __syncthreads();
+  if (kPair) cluster_sync_all(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (kPair) tmem_dealloc_pair(tmem_base, TMEM_COLS); else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -386,32 +458,73 @@ bool encode_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
   return r == CUDA_SUCCESS;
 }
 
-template <bool kGateUp>
+template <bool kGateUp, bool kPair>
 cudaError_t set_attrs() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kGateUp, kPair>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              int(smem_bytes<kPair>()));
+}
+
+template <bool kGateUp, bool kPair>
+cudaError_t launch_gemm(const GemmParams& gp, int num_sms, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kPair ? unsigned(num_sms & ~1) : unsigned(num_sms));
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem_bytes<kPair>();
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  if (kPair) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kGateUp, kPair>, gp);
 }
 
 }  // namespace
+
+// Tile choice.  A group of c rows costs ceil(c / M) tiles of M rows of tensor work;
+// with M = 256 (2-SM pairs) the padding averages ~128 rows per group against ~64
+// for M = 128, which outweighs the pair kernel's higher MMA rate until groups
+// average about 1024 rows.  MOE_GEMM_TILES=single|pair overrides the choice
+// (both compute the same result; for tuning and tests).
+bool use_pair_tiles(const Ctx& c, int T) {
+  static const int forced = [] {
+    const char* v = getenv("MOE_GEMM_TILES");
+    if (v && strcmp(v, "pair") == 0) return 1;
+    if (v && strcmp(v, "single") == 0) return 0;
+    return -1;
+  }();
+  if (forced >= 0) return forced == 1;
+  return int64_t(T) * c.k >= int64_t(1024) * c.E;
+}
 
 moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                              cudaStream_t st) {
   if (!get_encoder()) return MOE_ERR_CUDA;
   static thread_local int attrs_device = -1;
   if (attrs_device != dev.device) {
-    if (set_attrs<true>() != cudaSuccess || set_attrs<false>() != cudaSuccess)
+    if (set_attrs<true, false>() != cudaSuccess || set_attrs<false, false>() != cudaSuccess ||
+        set_attrs<true, true>() != cudaSuccess || set_attrs<false, true>() != cudaSuccess)
       return MOE_ERR_CUDA;
     attrs_device = dev.device;
   }
   const int T = a.T;
+  const bool pair = use_pair_tiles(c, T);
+  const int b_box = pair ? 128 : 256;   // B rows one CTA loads per stage (down GEMM)
   const uint64_t nslots = uint64_t(T) * c.k;
   const uint64_t rows = nslots + uint64_t(c.S) * T;
+  // schedules of 128-row tiles at sched[0..G], of 256-row tiles at sched[G+1..2G+1]
+  const int32_t* sched = a.sched + (pair ? (c.E + c.S + 1) : 0);
 
   // ---- gate/up + SwiGLU ----
   GemmParams gp;
   memset(&gp, 0, sizeof gp);
-  bool ok = encode_2d(&gp.a_routed, a.x_perm, nslots, c.d, BM) &&
-            encode_2d(&gp.a_shared, a.x, uint64_t(T), c.d, BM) &&
+  bool ok = encode_2d(&gp.a_routed, a.x_perm, nslots, c.d, 128) &&
+            encode_2d(&gp.a_shared, a.x, uint64_t(T), c.d, 128) &&
             encode_2d(&gp.b0, a.Wg, uint64_t(c.E) * c.F, c.d, BN / 2) &&
             encode_2d(&gp.b1, a.Wu, uint64_t(c.E) * c.F, c.d, BN / 2);
   if (c.S > 0)
@@ -423,7 +536,7 @@ moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& d
   }
   if (!ok) return MOE_ERR_CUDA;
   gp.offsets = a.offsets;
-  gp.sched = a.sched;
+  gp.sched = sched;
   gp.out = a.h_act;
   gp.status = a.status;
   gp.T = T;
@@ -434,18 +547,18 @@ moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& d
   gp.n_out = c.F;
   gp.b_rows = c.F;
   gp.out_rows = int(rows);
-  const int grid = dev.num_sms;
-  grouped_gemm_kernel<true><<<grid, NUM_THREADS, kSmemBytes, st>>>(gp);
-  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  cudaError_t err = pair ? launch_gemm<true, true>(gp, dev.num_sms, st)
+                         : launch_gemm<true, false>(gp, dev.num_sms, st);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
   if (a.after_gate_up && cudaEventRecord(a.after_gate_up, st) != cudaSuccess) return MOE_ERR_CUDA;
 
   // ---- down projection ----
   GemmParams dp;
   memset(&dp, 0, sizeof dp);
-  ok = encode_2d(&dp.a_routed, a.h_act, rows, c.F, BM) &&
-       encode_2d(&dp.b0, a.Wd, uint64_t(c.E) * c.d, c.F, BN);
+  ok = encode_2d(&dp.a_routed, a.h_act, rows, c.F, 128) &&
+       encode_2d(&dp.b0, a.Wd, uint64_t(c.E) * c.d, c.F, b_box);
   if (c.S > 0)
-    ok = ok && encode_2d(&dp.s0, a.Sd, uint64_t(c.S) * c.d, c.F, BN);
+    ok = ok && encode_2d(&dp.s0, a.Sd, uint64_t(c.S) * c.d, c.F, b_box);
   else
     dp.s0 = dp.b0;
   if (!ok) return MOE_ERR_CUDA;
@@ -453,8 +566,9 @@ moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& d
   dp.b1 = dp.b0;
   dp.s1 = dp.s0;
   dp.offsets = a.offsets;
-  dp.sched = a.sched;
+  dp.sched = sched;
   dp.out = a.Y;
+  dp.out_bf16 = a.y_bf16 ? 1 : 0;
   dp.status = a.status;
   dp.T = T;
   dp.E = c.E;
@@ -464,8 +578,9 @@ moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& d
   dp.n_out = c.d;
   dp.b_rows = c.d;
   dp.out_rows = int(rows);
-  grouped_gemm_kernel<false><<<grid, NUM_THREADS, kSmemBytes, st>>>(dp);
-  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  err = pair ? launch_gemm<false, true>(dp, dev.num_sms, st)
+             : launch_gemm<false, false>(dp, dev.num_sms, st);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

@@ -9,7 +9,8 @@
 //           expert of the ZAKER release news is added with weight 1):
 //             y[t] = sum_s Y[T*k + s*T + t] + sum_i w[t][i] * Y[pos[t*k + i]]
 //           in fp32, in that fixed order, then rounded once to bf16.  Each
-//           thread owns 8 consecutive features of one token.
+//           thread owns 8 consecutive features of one token.  Y is fp32 for
+//           moe_combine and bf16 inside moe_forward (half the traffic).
 #include "common.cuh"
 #include "internal.h"
 
@@ -46,21 +47,30 @@ __global__ void __launch_bounds__(kGatherThreads)
   }
 }
 
-__device__ __forceinline__ void fma8(float (&acc)[8], float w, const float* __restrict__ row) {
-  const float4 a = *reinterpret_cast<const float4*>(row);
-  const float4 b = *reinterpret_cast<const float4*>(row + 4);
-  acc[0] = fmaf(w, a.x, acc[0]);
-  acc[1] = fmaf(w, a.y, acc[1]);
-  acc[2] = fmaf(w, a.z, acc[2]);
-  acc[3] = fmaf(w, a.w, acc[3]);
-  acc[4] = fmaf(w, b.x, acc[4]);
-  acc[5] = fmaf(w, b.y, acc[5]);
-  acc[6] = fmaf(w, b.z, acc[6]);
-  acc[7] = fmaf(w, b.w, acc[7]);
-}
+struct RowF32 {
+  __device__ static void load8(const float* __restrict__ row, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(row);
+    const float4 b = *reinterpret_cast<const float4*>(row + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+struct RowBF16 {
+  __device__ static void load8(const uint16_t* __restrict__ row, float (&v)[8]) {
+    const uint4 a = *reinterpret_cast<const uint4*>(row);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      v[2 * q] = bf16_bits_to_float(w[q] & 0xFFFFu);
+      v[2 * q + 1] = bf16_bits_to_float(w[q] >> 16);
+    }
+  }
+};
 
+// TY = float (Y in fp32) or uint16_t (Y in bf16); the sums are fp32 either way.
+template <typename TY, typename Row>
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_kernel(const float* __restrict__ Y, const float* __restrict__ topk_w,
+    combine_kernel(const TY* __restrict__ Y, const float* __restrict__ topk_w,
                    const int32_t* __restrict__ pos, int T, int k, int S, int d,
                    uint16_t* __restrict__ y) {
   const int t = blockIdx.x;
@@ -68,17 +78,19 @@ __global__ void __launch_bounds__(kCombineThreads)
   if (c >= d) return;
   const size_t nslots = size_t(T) * k;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float v[8];
   for (int s = 0; s < S; ++s) {
-    const float* row = Y + (nslots + size_t(s) * T + t) * d + c;
-    const float4 a = *reinterpret_cast<const float4*>(row);
-    const float4 b = *reinterpret_cast<const float4*>(row + 4);
-    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    Row::load8(Y + (nslots + size_t(s) * T + t) * d + c, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] += v[j];
   }
   for (int i = 0; i < k; ++i) {
     const int p = pos[size_t(t) * k + i];
     if (p < 0 || size_t(p) >= nslots) continue;
-    fma8(acc, topk_w[size_t(t) * k + i], Y + size_t(p) * d + c);
+    const float w = topk_w[size_t(t) * k + i];
+    Row::load8(Y + size_t(p) * d + c, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = fmaf(w, v[j], acc[j]);
   }
   uint4 out;
   out.x = pack_bf16x2(acc[0], acc[1]);
@@ -106,7 +118,16 @@ cudaError_t launch_gather(const Ctx& c, const uint16_t* x, const int32_t* perm,
 cudaError_t launch_combine(const Ctx& c, const float* Y, const float* topk_w, const int32_t* pos,
                            int T, uint16_t* y, cudaStream_t st) {
   dim3 grid(T, (c.d / 8 + kCombineThreads - 1) / kCombineThreads);
-  combine_kernel<<<grid, kCombineThreads, 0, st>>>(Y, topk_w, pos, T, c.k, c.S, c.d, y);
+  combine_kernel<float, RowF32><<<grid, kCombineThreads, 0, st>>>(Y, topk_w, pos, T, c.k, c.S,
+                                                                 c.d, y);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_bf16(const Ctx& c, const uint16_t* Y, const float* topk_w,
+                                const int32_t* pos, int T, uint16_t* y, cudaStream_t st) {
+  dim3 grid(T, (c.d / 8 + kCombineThreads - 1) / kCombineThreads);
+  combine_kernel<uint16_t, RowBF16><<<grid, kCombineThreads, 0, st>>>(Y, topk_w, pos, T, c.k,
+                                                                      c.S, c.d, y);
   return cudaGetLastError();
 }
 

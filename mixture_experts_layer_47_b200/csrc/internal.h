@@ -64,6 +64,8 @@ cudaError_t launch_gather(const Ctx& c, const uint16_t* x, const int32_t* perm,
 
 cudaError_t launch_combine(const Ctx& c, const float* Y, const float* topk_w, const int32_t* pos,
                            int T, uint16_t* y, cudaStream_t st);
+cudaError_t launch_combine_bf16(const Ctx& c, const uint16_t* Y, const float* topk_w,
+                                const int32_t* pos, int T, uint16_t* y, cudaStream_t st);
 
 struct FfnArgs {
   const uint16_t* x;        // [T][d]
@@ -72,7 +74,8 @@ struct FfnArgs {
   const int32_t* sched;     // [E+S+1]
   const uint16_t *Wg, *Wu, *Wd, *Sg, *Su, *Sd;
   uint16_t* h_act;          // [T*k+S*T][F]
-  float* Y;                 // [T*k+S*T][d]
+  void* Y;                  // [T*k+S*T][d], fp32 or (y_bf16) bf16
+  bool y_bf16;
   int* status;
   int T;
   cudaEvent_t after_gate_up;  // recorded between the two GEMMs when non-null

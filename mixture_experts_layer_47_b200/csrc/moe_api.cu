@@ -83,10 +83,10 @@ Layout make_layout(const Ctx& c, int T, int num_sms) {
   L.perm = take(nslots * sizeof(int32_t));
   L.pos = take(nslots * sizeof(int32_t));
   L.blk_hist = take(size_t(L.nblk) * c.E * sizeof(int32_t));
-  L.sched = take(size_t(c.E + c.S + 1) * sizeof(int32_t));
+  L.sched = take(2 * size_t(c.E + c.S + 1) * sizeof(int32_t));  // 128- and 256-row tiles
   L.x_perm = take(nslots * c.d * sizeof(uint16_t));
   L.h_act = take(rows * c.F * sizeof(uint16_t));
-  L.y_rows = take(rows * c.d * sizeof(float));
+  L.y_rows = take(rows * c.d * sizeof(float));  // fp32 for moe_expert_ffn, bf16 in moe_forward
   L.x_stage = take(size_t(T) * c.d * sizeof(uint16_t));
   L.y_stage = take(size_t(T) * c.d * sizeof(uint16_t));
   L.end = off;
@@ -272,6 +272,7 @@ moe_status moe_expert_ffn(moe_handle h, const uint16_t* x, const int32_t* perm,
   a.Sd = Ws_down;
   a.h_act = reinterpret_cast<uint16_t*>(ws + L.h_act);
   a.Y = Y;
+  a.y_bf16 = false;
   a.status = status;
   a.T = T;
   a.after_gate_up = nullptr;
@@ -309,7 +310,7 @@ static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W
   int32_t* pos = reinterpret_cast<int32_t*>(ws + L.pos);
   int32_t* sched = reinterpret_cast<int32_t*>(ws + L.sched);
   uint16_t* x_perm = reinterpret_cast<uint16_t*>(ws + L.x_perm);
-  float* Y = reinterpret_cast<float*>(ws + L.y_rows);
+  uint16_t* Y = reinterpret_cast<uint16_t*>(ws + L.y_rows);  // bf16 rows
   const bool prof = h->n_stage_events == MOE_STAGE_EVENTS;
   auto mark = [&](int i) -> moe_status {
     return prof ? cuda_status(cudaEventRecord(h->stage_events[i], st)) : MOE_OK;
@@ -343,10 +344,11 @@ static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W
   a.Y = Y;
   a.status = status;
   a.T = T;
+  a.y_bf16 = true;
   a.after_gate_up = prof ? h->stage_events[4] : nullptr;
   if ((s = launch_expert_ffn(c, a, *dev, st))) return s;
   if ((s = mark(5))) return s;
-  if ((s = cuda_status(launch_combine(c, Y, topk_w, pos, T, y, st)))) return s;
+  if ((s = cuda_status(launch_combine_bf16(c, Y, topk_w, pos, T, y, st)))) return s;
   return mark(6);
 }
 

@@ -9,14 +9,17 @@
 // Two kernels:
 //  router_partial  logits over a K-chunk, fp32 FFMA (no TF32: the index parity
 //                  needs logits accurate to well below 1e-5), x widened from
-//                  bf16 exactly.  A CTA computes a BT x 64 tile of
-//                  (tokens x experts) for one K-chunk; the chunk count is
-//                  chosen so the grid fills the GPU even for 16 tokens.
-//  router_topk     one warp per token adds the chunk partials in a fixed
-//                  order, then k rounds of a warp arg-max (value desc, expert
-//                  asc) select the experts; the gate of choice i is
+//                  bf16 exactly.  A CTA computes a (tokens x experts) tile --
+//                  16 x 64, 64 x 64 or 128 x 128 by batch size -- for one
+//                  K-chunk; the chunk count is chosen so the grid fills the GPU
+//                  even for 16 tokens.
+//  router_topk     one CTA per token adds the chunk partials in a fixed order,
+//                  then k rounds of a warp arg-max (value desc, expert asc)
+//                  select the experts; the gate of choice i is
 //                  exp(l_i - l_0) / sum_j exp(l_j - l_0).
 #include <math.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "internal.h"
@@ -25,21 +28,83 @@ namespace moe {
 namespace {
 
 constexpr int kRouterThreads = 256;
-constexpr int kBE = 64;   // experts per CTA tile
-constexpr int kBK = 32;   // K per shared-memory stage
+constexpr int kBK = 16;   // K per shared-memory stage
 
-template <int BT>
+// Partial logits of a BT x BE (tokens x experts) tile over one K chunk, fp32
+// FFMA.  256 threads, each owning TT tokens x TE experts (split in two halves
+// of the tile for conflict-free 16-byte shared loads when TT, TE = 8); the K
+// loop is double-buffered: the next stage's global loads are issued before
+// the current stage's FMAs.
+template <int BT, int BE, int TT, int TE>
 __global__ void __launch_bounds__(kRouterThreads)
     router_partial_kernel(const uint16_t* __restrict__ x, const float* __restrict__ Wr, int T,
                           int d, int E, int kchunk, float* __restrict__ part) {
-  constexpr int TT = BT / 16;  // tokens per thread
-  constexpr int TE = 4;        // experts per thread
-  __shared__ __align__(16) float xs[kBK][BT + 4];
-  __shared__ __align__(16) float ws[kBK][kBE + 4];
+  static_assert((BT / TT) * (BE / TE) == kRouterThreads, "thread tiling");
+  static_assert(TE == 4 || TE == 8, "experts per thread");
+  constexpr int NTX = BE / TE;                 // threads along experts
+  constexpr int HT = (TT == 8) ? TT / 2 : TT;  // tokens per half
+  constexpr int HE = (TE == 8) ? TE / 2 : TE;
+  constexpr int X_LOADS = BT * kBK / 8;        // 16-byte loads of x per stage
+  constexpr int W_LOADS = BE * kBK / 4;        // 16-byte loads of W per stage
+  constexpr int XL = (X_LOADS + kRouterThreads - 1) / kRouterThreads;
+  constexpr int WL = (W_LOADS + kRouterThreads - 1) / kRouterThreads;
+  __shared__ __align__(16) float xs[2][kBK][BT + 4];
+  __shared__ __align__(16) float ws[2][kBK][BE + 4];
+
   const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
-  const int t0 = blockIdx.x * BT, e0 = blockIdx.y * kBE, ks = blockIdx.z;
-  const int kbeg = ks * kchunk;
+  const int tx = tid % NTX, ty = tid / NTX;
+  const int t0 = blockIdx.x * BT, e0 = blockIdx.y * BE;
+  const int kbeg = blockIdx.z * kchunk;
+  const int nk = kchunk / kBK;
+
+  uint4 xr[XL];
+  float4 wr[WL][1];
+  auto load_global = [&](int k0) {
+#pragma unroll
+    for (int l = 0; l < XL; ++l) {
+      const int i = tid + l * kRouterThreads;
+      xr[l] = make_uint4(0, 0, 0, 0);
+      if (i < X_LOADS) {
+        const int r = i / (kBK / 8), c8 = (i % (kBK / 8)) * 8;
+        if (t0 + r < T) xr[l] = *reinterpret_cast<const uint4*>(x + size_t(t0 + r) * d + k0 + c8);
+      }
+    }
+#pragma unroll
+    for (int l = 0; l < WL; ++l) {
+      const int i = tid + l * kRouterThreads;
+      wr[l][0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < W_LOADS) {
+        const int r = i / (kBK / 4), c4 = (i % (kBK / 4)) * 4;
+        if (e0 + r < E) wr[l][0] = *reinterpret_cast<const float4*>(Wr + size_t(e0 + r) * d + k0 + c4);
+      }
+    }
+  };
+  auto store_smem = [&](int buf) {
+#pragma unroll
+    for (int l = 0; l < XL; ++l) {
+      const int i = tid + l * kRouterThreads;
+      if (i < X_LOADS) {
+        const int r = i / (kBK / 8), c8 = (i % (kBK / 8)) * 8;
+        const uint32_t w4[4] = {xr[l].x, xr[l].y, xr[l].z, xr[l].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          xs[buf][c8 + 2 * q][r] = bf16_bits_to_float(w4[q] & 0xFFFFu);
+          xs[buf][c8 + 2 * q + 1][r] = bf16_bits_to_float(w4[q] >> 16);
+        }
+      }
+    }
+#pragma unroll
+    for (int l = 0; l < WL; ++l) {
+      const int i = tid + l * kRouterThreads;
+      if (i < W_LOADS) {
+        const int r = i / (kBK / 4), c4 = (i % (kBK / 4)) * 4;
+        ws[buf][c4][r] = wr[l][0].x;
+        ws[buf][c4 + 1][r] = wr[l][0].y;
+        ws[buf][c4 + 2][r] = wr[l][0].z;
+        ws[buf][c4 + 3][r] = wr[l][0].w;
+      }
+    }
+  };
 
   float acc[TT][TE];
 #pragma unroll
@@ -47,57 +112,48 @@ __global__ void __launch_bounds__(kRouterThreads)
 #pragma unroll
     for (int j = 0; j < TE; ++j) acc[i][j] = 0.f;
 
-  for (int k0 = kbeg; k0 < kbeg + kchunk; k0 += kBK) {
-    // x tile: BT tokens x 32 bf16, 16-byte loads, widened to fp32, stored K-major.
-    for (int i = tid; i < BT * (kBK / 8); i += kRouterThreads) {
-      const int r = i / (kBK / 8), c8 = (i % (kBK / 8)) * 8;
-      const int t = t0 + r;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t < T) v = *reinterpret_cast<const uint4*>(x + size_t(t) * d + k0 + c8);
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+  load_global(kbeg);
+  store_smem(0);
+  __syncthreads();
+  for (int kt = 0; kt < nk; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < nk) load_global(kbeg + (kt + 1) * kBK);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        xs[c8 + 2 * q][r] = bf16_bits_to_float(w4[q] & 0xFFFFu);
-        xs[c8 + 2 * q + 1][r] = bf16_bits_to_float(w4[q] >> 16);
-      }
-    }
-    // W tile: 64 experts x 32 fp32.
-    for (int i = tid; i < kBE * (kBK / 4); i += kRouterThreads) {
-      const int r = i / (kBK / 4), c4 = (i % (kBK / 4)) * 4;
-      const int e = e0 + r;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < E) v = *reinterpret_cast<const float4*>(Wr + size_t(e) * d + k0 + c4);
-      ws[c4][r] = v.x;
-      ws[c4 + 1][r] = v.y;
-      ws[c4 + 2][r] = v.z;
-      ws[c4 + 3][r] = v.w;
-    }
-    __syncthreads();
-#pragma unroll 8
     for (int kk = 0; kk < kBK; ++kk) {
       float a[TT], b[TE];
+      if constexpr (HT == 4) {   // 16-byte shared loads: a float4 per half tile
 #pragma unroll
-      for (int i = 0; i < TT; ++i) a[i] = xs[kk][ty * TT + i];
-      const float4 bv = *reinterpret_cast<const float4*>(&ws[kk][tx * TE]);
-      b[0] = bv.x;
-      b[1] = bv.y;
-      b[2] = bv.z;
-      b[3] = bv.w;
+        for (int h = 0; h < TT / 4; ++h) {
+          const float4 v =
+              *reinterpret_cast<const float4*>(&xs[buf][kk][h * (BT / 2) * (TT / 4 - 1) + ty * 4]);
+          a[4 * h] = v.x; a[4 * h + 1] = v.y; a[4 * h + 2] = v.z; a[4 * h + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < TT; ++i) a[i] = xs[buf][kk][ty * TT + i];
+      }
+#pragma unroll
+      for (int h = 0; h < TE / 4; ++h) {
+        const float4 v =
+            *reinterpret_cast<const float4*>(&ws[buf][kk][h * (BE / 2) * (TE / 4 - 1) + tx * 4]);
+        b[4 * h] = v.x; b[4 * h + 1] = v.y; b[4 * h + 2] = v.z; b[4 * h + 3] = v.w;
+      }
 #pragma unroll
       for (int i = 0; i < TT; ++i)
 #pragma unroll
         for (int j = 0; j < TE; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
     }
+    if (kt + 1 < nk) store_smem(buf ^ 1);
     __syncthreads();
   }
 #pragma unroll
   for (int i = 0; i < TT; ++i) {
-    const int t = t0 + ty * TT + i;
+    const int t = t0 + (i / HT) * (BT / 2) * (TT / HT - 1) + ty * HT + (i % HT);
     if (t >= T) continue;
 #pragma unroll
     for (int j = 0; j < TE; ++j) {
-      const int e = e0 + tx * TE + j;
-      if (e < E) part[(size_t(ks) * T + t) * E + e] = acc[i][j];
+      const int e = e0 + (j / HE) * (BE / 2) * (TE / HE - 1) + tx * HE + (j % HE);
+      if (e < E) part[(size_t(blockIdx.z) * T + t) * E + e] = acc[i][j];
     }
   }
 }
@@ -106,40 +162,44 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
   return v > bv || (v == bv && e < be);
 }
 
-// EPL = experts per lane (E <= 32 * EPL); expert e lives in lane e % 32, slot e / 32.
-template <int EPL>
-__global__ void __launch_bounds__(kRouterThreads)
+// One CTA per token: thread e adds the K-chunk partials of expert e in chunk
+// order (plus the bias) into shared memory; warp 0 then takes k rounds of a
+// warp arg-max (value desc, expert asc) over the E logits and writes the
+// experts and their renormalised softmax gates.
+__global__ void __launch_bounds__(1024)
     router_topk_kernel(const float* __restrict__ part, const float* __restrict__ bias, int T, int E,
                        int k, int ksplit, int32_t* __restrict__ topk_idx,
                        float* __restrict__ topk_w) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (kRouterThreads / 32) + (threadIdx.x >> 5);
-  if (t >= T) return;
-  float v[EPL];
-  uint32_t taken = 0;
+  extern __shared__ float logit[];  // [E]
+  const int t = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float s = 0.f;
+    const float* p = part + size_t(t) * E + e;
+    const size_t stride = size_t(T) * E;
+    int ks = 0;
+    for (; ks + 8 <= ksplit; ks += 8) {   // eight independent loads in flight, added in order
+      float v[8];
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) {
-    const int e = lane + 32 * j;
-    if (e < E) {
-      float s = 0.f;
-      for (int ks = 0; ks < ksplit; ++ks) s += part[(size_t(ks) * T + t) * E + e];
-      if (bias) s += bias[e];
-      v[j] = (s == s) ? s : -INFINITY;  // a NaN score is never preferred
-    } else {
-      v[j] = -INFINITY;
-      taken |= 1u << j;
+      for (int q = 0; q < 8; ++q) v[q] = p[(ks + q) * stride];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) s += v[q];
     }
+    for (; ks < ksplit; ++ks) s += p[ks * stride];
+    if (bias) s += bias[e];
+    logit[e] = (s == s) ? s : -INFINITY;  // a NaN score is never preferred
   }
+  __syncthreads();
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
   float my_l = 0.f, l0 = 0.f;
   int my_e = 0;
   for (int i = 0; i < k; ++i) {
     float bv = -INFINITY;
     int be = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = lane + 32 * j;
-      if (!((taken >> j) & 1u) && better(v[j], e, bv, be)) {
-        bv = v[j];
+    for (int e = lane; e < E; e += 32) {
+      const float v = logit[e];
+      if (better(v, e, bv, be)) {
+        bv = v;
         be = e;
       }
     }
@@ -152,7 +212,9 @@ __global__ void __launch_bounds__(kRouterThreads)
         be = oe;
       }
     }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    // every lane holds the winner; its owner removes it from further rounds
+    if ((be & 31) == lane) logit[be] = __int_as_float(0xff800001u);  // NaN: never 'better'
+    __syncwarp();
     if (i == 0) l0 = bv;
     if (lane == i) {
       my_l = bv;
@@ -169,52 +231,60 @@ __global__ void __launch_bounds__(kRouterThreads)
   }
 }
 
+template <int BT, int BE, int TT, int TE>
+cudaError_t launch_partial(const Ctx& c, const RouterPlan& rp, const uint16_t* x, const float* Wr,
+                           int T, float* part, cudaStream_t st) {
+  dim3 grid((T + BT - 1) / BT, (c.E + BE - 1) / BE, rp.ksplit);
+  router_partial_kernel<BT, BE, TT, TE><<<grid, kRouterThreads, 0, st>>>(x, Wr, T, c.d, c.E,
+                                                                         rp.kchunk, part);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
+// Tile shape by batch size; the K split is chosen so the grid fills the GPU
+// (about two CTAs per SM, counted for a 148-SM part so that the plan, and with
+// it the summation order, is the same on every device).
 RouterPlan router_plan(const Ctx& c, int T, int num_sms) {
   RouterPlan rp;
-  rp.bt = T <= 16 ? 16 : 64;
-  const int tiles = ((T + rp.bt - 1) / rp.bt) * ((c.E + kBE - 1) / kBE);
+  rp.bt = T <= 16 ? 16 : (T <= 256 ? 64 : 128);
+  const int be = rp.bt == 128 ? 128 : 64;
+  const int tiles = ((T + rp.bt - 1) / rp.bt) * ((c.E + be - 1) / be);
   const int kblocks = c.d / kBK;
-  const int want = (2 * (num_sms > 0 ? num_sms : 148) + tiles - 1) / tiles;
-  int ks = 1;
-  for (int cand = 1; cand <= kblocks && cand <= 64; ++cand)
-    if (kblocks % cand == 0 && cand <= want) ks = cand;
-  rp.ksplit = ks;
-  rp.kchunk = c.d / ks;
+  const int slots = 2 * (num_sms > 0 ? num_sms : 148);
+  int best = 1;
+  double best_eff = -1.0;
+  const int max_split = rp.bt == 128 ? 8 : 64;
+  for (int cand = 1; cand <= kblocks && cand <= max_split; ++cand) {
+    if (kblocks % cand) continue;
+    const int n = tiles * cand;
+    const int waves = (n + slots - 1) / slots;
+    double eff = double(n) / double(waves * slots);
+    if (n < slots / 2) eff *= 0.5;   // too few CTAs to cover the SMs
+    if (eff > best_eff + 0.02) {
+      best_eff = eff;
+      best = cand;
+    }
+  }
+  rp.ksplit = best;
+  rp.kchunk = c.d / best;
   return rp;
 }
 
 cudaError_t launch_router(const Ctx& c, const RouterPlan& rp, const uint16_t* x, const float* Wr,
                           const float* bias, int T, float* part, int32_t* topk_idx, float* topk_w,
                           cudaStream_t st) {
-  dim3 grid((T + rp.bt - 1) / rp.bt, (c.E + kBE - 1) / kBE, rp.ksplit);
+  cudaError_t err;
   if (rp.bt == 16)
-    router_partial_kernel<16><<<grid, kRouterThreads, 0, st>>>(x, Wr, T, c.d, c.E, rp.kchunk,
-                                                              part);
+    err = launch_partial<16, 64, 1, 4>(c, rp, x, Wr, T, part, st);
+  else if (rp.bt == 64)
+    err = launch_partial<64, 64, 4, 4>(c, rp, x, Wr, T, part, st);
   else
-    router_partial_kernel<64><<<grid, kRouterThreads, 0, st>>>(x, Wr, T, c.d, c.E, rp.kchunk,
-                                                              part);
-  cudaError_t err = cudaGetLastError();
+    err = launch_partial<128, 128, 8, 8>(c, rp, x, Wr, T, part, st);
   if (err != cudaSuccess) return err;
-  const int blocks = (T + kRouterThreads / 32 - 1) / (kRouterThreads / 32);
-  const int epl = (c.E + 31) / 32;
-#define MOE_TOPK_CASE(N)                                                                       \
-  case N:                                                                                      \
-    router_topk_kernel<N><<<blocks, kRouterThreads, 0, st>>>(part, bias, T, c.E, c.k,          \
-                                                             rp.ksplit, topk_idx, topk_w);     \
-    break;
-  const int epl_p2 = epl <= 1 ? 1 : epl <= 2 ? 2 : epl <= 4 ? 4 : epl <= 8 ? 8 : epl <= 16 ? 16
-                                                                                         : 32;
-  switch (epl_p2) {
-    MOE_TOPK_CASE(1)
-    MOE_TOPK_CASE(2)
-    MOE_TOPK_CASE(4)
-    MOE_TOPK_CASE(8)
-    MOE_TOPK_CASE(16)
-    MOE_TOPK_CASE(32)
-  }
-#undef MOE_TOPK_CASE
+  const int threads = std::min(1024, std::max(32, (c.E + 31) / 32 * 32));
+  router_topk_kernel<<<T, threads, c.E * sizeof(float), st>>>(part, bias, T, c.E, c.k, rp.ksplit,
+                                                              topk_idx, topk_w);
   return cudaGetLastError();
 }
 

@@ -26,6 +26,10 @@ SHAPES = [  # T, d, E, k, F, S, bias_scale
     (130, 320, 5, 3, 384, 2, 0.0),
     (513, 512, 64, 8, 256, 1, 0.2),
     (40, 256, 8, 8, 128, 1, 0.0),      # k == E
+    # T*k >= 128*E: the 2-SM (cta_group::2, 256-row tile) GEMM path
+    (600, 256, 4, 2, 128, 1, 0.0),     # ~300 rows per expert: two pair tiles, ragged tail
+    (200, 320, 2, 2, 192, 2, 0.0),     # k == E, every group 200 rows; two shared experts
+    (1000, 128, 8, 2, 64, 1, 0.3),     # d_ff = 64: half of each gate/up tile masked
 ]
 
 
@@ -170,6 +174,21 @@ def test_every_token_on_one_expert_and_empty_experts():
     y, v = gpu_forward(to_device(inp, "cuda"))
     assert int(v["counts"][3]) == T and int(v["counts"][7]) == T
     assert int((v["counts"] == 0).sum()) == E - 2
+    ref = oracle.forward(inp)
+    route_parity(ref["logits"], v["topk_idx"].numpy(), v["topk_w"].numpy(), k)
+    assert rel_err(y.float().numpy(), ref["y"]) < Y_REL_TOL
+
+
+def test_pair_tiles_hot_experts_and_empty_experts():
+    """2-SM path: two experts take all 700 tokens (3 pair tiles of 256, 256, 188 rows) and
+    the other two stay empty."""
+    T, d, E, k, F, S = 700, 256, 4, 2, 128, 1
+    inp = make_small(T, d, E, k, F, S, seed=19)
+    bias = torch.tensor([0.0, 50.0, 0.0, 40.0])
+    inp = Inputs(inp.wl, inp.x, inp.W_router, bias, inp.W_gate, inp.W_up, inp.W_down,
+                 inp.Ws_gate, inp.Ws_up, inp.Ws_down)
+    y, v = gpu_forward(to_device(inp, "cuda"))
+    assert v["counts"].tolist() == [0, T, 0, T]
     ref = oracle.forward(inp)
     route_parity(ref["logits"], v["topk_idx"].numpy(), v["topk_w"].numpy(), k)
     assert rel_err(y.float().numpy(), ref["y"]) < Y_REL_TOL
