@@ -99,15 +99,20 @@ typedef struct {
     size_t h_act;     /* bf16  [T*k + S*T][F]  SwiGLU activations            */
     size_t y_rows;    /* bf16  [T*k + S*T][d]  per-(slot, expert) outputs    */
     size_t total;     /* bytes used, including the alignment slack           */
+    size_t router_partials; /* fp32 [router_ksplit][T][E] partial logits     */
+    size_t router_ksplit;   /* their count; the logits are their in-order sum */
 } moe_workspace_layout;
 moe_status moe_get_workspace_layout(moe_handle h, int T, uintptr_t workspace_addr,
                                     moe_workspace_layout *out);
 
 /*
  * Router: score, top-k select and gate (explainer section 2.2).
- *   logits[t][e] = sum_j x[t][j] * W_router[e][j] + bias[e]     (fp32 FMA on
- *                  CUDA cores, no TF32; split-K partial sums added in a fixed
- *                  order)
+ *   logits[t][e] = sum_j x[t][j] * W_router[e][j] + bias[e]     (fp32-accurate:
+ *                  on the tensor cores with W_router split exactly into three
+ *                  bf16 parts and every 64-wide K chunk accumulated separately
+ *                  and added in fp32 (T > 32), or with fp32 FMA on the CUDA
+ *                  cores (T <= 32); MOE_ROUTER=tc|ffma in the environment forces
+ *                  one; split-K partial sums added in a fixed order)
  *   topk_idx[t][i] = the i-th largest logit's expert (ties: lower index)
  *   topk_w[t][i]   = exp(l_i - l_0) / sum_{j<k} exp(l_j - l_0)
  * x: bf16 [T][d]; W_router: fp32 [E][d]; bias: fp32 [E] or NULL;

@@ -50,7 +50,7 @@ class MoEError(RuntimeError):
 class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("status", "topk_idx", "topk_w", "counts", "offsets", "perm", "pos", "h_act",
-                 "y_rows", "total")]
+                 "y_rows", "total", "router_partials", "router_ksplit")]
 
 
 _lib = None
@@ -304,8 +304,10 @@ def workspace_views(h: Handle, T: int, workspace: torch.Tensor) -> dict:
         nbytes = n * torch.empty((), dtype=dtype).element_size()
         return workspace[off:off + nbytes].view(dtype)
 
+    ks = L["router_ksplit"]
     return dict(
         status=view(L["status"], 1, torch.int32),
+        router_partials=view(L["router_partials"], ks * T * h.E, torch.float32).view(ks, T, h.E),
         topk_idx=view(L["topk_idx"], T * h.k, torch.int32).view(T, h.k),
         topk_w=view(L["topk_w"], T * h.k, torch.float32).view(T, h.k),
         counts=view(L["counts"], h.E, torch.int32),

@@ -492,13 +492,9 @@ cudaError_t launch_gemm(const GemmParams& gp, int num_sms, cudaStream_t st) {
 // average about 1024 rows.  MOE_GEMM_TILES=single|pair overrides the choice
 // (both compute the same result; for tuning and tests).
 bool use_pair_tiles(const Ctx& c, int T) {
-  static const int forced = [] {
-    const char* v = getenv("MOE_GEMM_TILES");
-    if (v && strcmp(v, "pair") == 0) return 1;
-    if (v && strcmp(v, "single") == 0) return 0;
-    return -1;
-  }();
-  if (forced >= 0) return forced == 1;
+  const char* v = getenv("MOE_GEMM_TILES");
+  if (v && strcmp(v, "pair") == 0) return true;
+  if (v && strcmp(v, "single") == 0) return false;
   return int64_t(T) * c.k >= int64_t(1024) * c.E;
 }
 

@@ -17,16 +17,17 @@ struct Ctx {
 
 // Geometry of the router's split-K partial sums for T tokens.
 struct RouterPlan {
-  int bt;      // tokens per CTA tile (16 or 64)
-  int ksplit;  // number of K chunks
+  bool tc;     // tensor-core score GEMM (router_tc.cu) rather than fp32 FFMA tiles
+  int bt;      // FFMA: tokens per CTA tile (16, 64 or 128)
+  int ksplit;  // number of K chunks (partial logits added in order by the top-k)
   int kchunk;  // d / ksplit
 };
 RouterPlan router_plan(const Ctx& c, int T, int num_sms);
 
 // Workspace carve-up for T tokens (offsets from the 1024-aligned base).
 struct Layout {
-  size_t status, part, topk_idx, topk_w, counts, offsets, perm, pos, blk_hist, sched, x_perm,
-      h_act, y_rows, x_stage, y_stage, end;
+  size_t status, part, wparts, topk_idx, topk_w, counts, offsets, perm, pos, blk_hist, sched,
+      x_perm, h_act, y_rows, x_stage, y_stage, end;
   int nblk;           // dispatch blocks
   RouterPlan rplan;
 };
@@ -48,8 +49,13 @@ moe_status moe_internal_shape(moe_handle h, Ctx* out);
 
 // ---- launchers (each returns cudaSuccess or the launch error) ----
 cudaError_t launch_router(const Ctx& c, const RouterPlan& rp, const uint16_t* x, const float* Wr,
-                          const float* bias, int T, float* part, int32_t* topk_idx, float* topk_w,
-                          cudaStream_t st);
+                          const float* bias, int T, float* part, uint16_t* wparts, int* status,
+                          int num_sms, int32_t* topk_idx, float* topk_w, cudaStream_t st);
+int router_tc_ksplit(const Ctx& c, int T, int num_sms);
+cudaError_t launch_router_tc(const Ctx& c, int ksplit, const uint16_t* x, const float* Wr, int T,
+                             uint16_t* wparts, float* part, int* status, int num_sms,
+                             cudaStream_t st);
+bool use_pair_tiles(const Ctx& c, int T);
 
 cudaError_t launch_dispatch(const Ctx& c, const int32_t* topk_idx, int T, int nblk,
                             int32_t* blk_hist, int32_t* counts, int32_t* offsets, int32_t* perm,

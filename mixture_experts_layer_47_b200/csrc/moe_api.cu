@@ -76,6 +76,7 @@ Layout make_layout(const Ctx& c, int T, int num_sms) {
   };
   L.status = take(256);
   L.part = take(size_t(L.rplan.ksplit) * T * c.E * sizeof(float));
+  L.wparts = take(L.rplan.tc ? 3 * size_t(c.E) * c.d * sizeof(uint16_t) : 0);
   L.topk_idx = take(nslots * sizeof(int32_t));
   L.topk_w = take(nslots * sizeof(float));
   L.counts = take(size_t(c.E) * sizeof(int32_t));
@@ -170,6 +171,8 @@ moe_status moe_get_workspace_layout(moe_handle h, int T, uintptr_t workspace_add
   const Layout L = make_layout(h->c, T, kPlanSms);
   const size_t base = ((workspace_addr + kWsAlign - 1) & ~uintptr_t(kWsAlign - 1)) - workspace_addr;
   out->status = base + L.status;
+  out->router_partials = base + L.part;
+  out->router_ksplit = size_t(L.rplan.ksplit);
   out->topk_idx = base + L.topk_idx;
   out->topk_w = base + L.topk_w;
   out->counts = base + L.counts;
@@ -199,7 +202,10 @@ moe_status moe_route(moe_handle h, const uint16_t* x, const float* W_router, con
   uint8_t* ws = aligned_base(workspace);
   if ((s = cuda_status(cudaMemsetAsync(ws + L.status, 0, sizeof(int), st)))) return s;
   return cuda_status(launch_router(h->c, L.rplan, x, W_router, bias, T,
-                                   reinterpret_cast<float*>(ws + L.part), topk_idx, topk_w, st));
+                                   reinterpret_cast<float*>(ws + L.part),
+                                   reinterpret_cast<uint16_t*>(ws + L.wparts),
+                                   reinterpret_cast<int*>(ws + L.status), dev->num_sms, topk_idx,
+                                   topk_w, st));
 }
 
 moe_status moe_dispatch(moe_handle h, const int32_t* topk_idx, int T, int32_t* counts,
@@ -318,8 +324,9 @@ static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W
   if ((s = cuda_status(cudaMemsetAsync(status, 0, sizeof(int), st)))) return s;
   if ((s = mark(0))) return s;
   if ((s = cuda_status(launch_router(c, L.rplan, x, W_router, bias, T,
-                                     reinterpret_cast<float*>(ws + L.part), topk_idx, topk_w,
-                                     st))))
+                                     reinterpret_cast<float*>(ws + L.part),
+                                     reinterpret_cast<uint16_t*>(ws + L.wparts), status,
+                                     dev->num_sms, topk_idx, topk_w, st))))
     return s;
   if ((s = mark(1))) return s;
   if ((s = cuda_status(launch_dispatch(c, topk_idx, T, L.nblk,

@@ -19,6 +19,9 @@
 //                  exp(l_i - l_0) / sum_j exp(l_j - l_0).
 #include <math.h>
 
+#include <stdlib.h>
+#include <string.h>
+
 #include <algorithm>
 
 #include "common.cuh"
@@ -242,11 +245,26 @@ cudaError_t launch_partial(const Ctx& c, const RouterPlan& rp, const uint16_t* x
 
 }  // namespace
 
-// Tile shape by batch size; the K split is chosen so the grid fills the GPU
-// (about two CTAs per SM, counted for a 148-SM part so that the plan, and with
-// it the summation order, is the same on every device).
+// Path and tile shape by batch size.  The score GEMM runs on the tensor cores
+// (router_tc.cu) for more than 32 tokens and on fp32 FFMA tiles otherwise;
+// MOE_ROUTER=tc|ffma forces one.  Both compute fp32-accurate logits.  The FFMA K split is chosen so the grid
+// fills the GPU (about two CTAs per SM, counted for a 148-SM part so that the
+// plan, and with it the summation order, is the same on every device).
 RouterPlan router_plan(const Ctx& c, int T, int num_sms) {
   RouterPlan rp;
+  const char* env = getenv("MOE_ROUTER");
+  if (env && strcmp(env, "ffma") == 0)
+    rp.tc = false;
+  else if (env && strcmp(env, "tc") == 0)
+    rp.tc = true;
+  else
+    rp.tc = T > 32;   // below that the FFMA tiles finish first (measured on B200)
+  if (rp.tc) {
+    rp.bt = 128;
+    rp.ksplit = router_tc_ksplit(c, T, num_sms);
+    rp.kchunk = c.d / rp.ksplit;
+    return rp;
+  }
   rp.bt = T <= 16 ? 16 : (T <= 256 ? 64 : 128);
   const int be = rp.bt == 128 ? 128 : 64;
   const int tiles = ((T + rp.bt - 1) / rp.bt) * ((c.E + be - 1) / be);
@@ -272,10 +290,12 @@ RouterPlan router_plan(const Ctx& c, int T, int num_sms) {
 }
 
 cudaError_t launch_router(const Ctx& c, const RouterPlan& rp, const uint16_t* x, const float* Wr,
-                          const float* bias, int T, float* part, int32_t* topk_idx, float* topk_w,
-                          cudaStream_t st) {
+                          const float* bias, int T, float* part, uint16_t* wparts, int* status,
+                          int num_sms, int32_t* topk_idx, float* topk_w, cudaStream_t st) {
   cudaError_t err;
-  if (rp.bt == 16)
+  if (rp.tc)
+    err = launch_router_tc(c, rp.ksplit, x, Wr, T, wparts, part, status, num_sms, st);
+  else if (rp.bt == 16)
     err = launch_partial<16, 64, 1, 4>(c, rp, x, Wr, T, part, st);
   else if (rp.bt == 64)
     err = launch_partial<64, 64, 4, 4>(c, rp, x, Wr, T, part, st);

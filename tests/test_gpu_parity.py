@@ -52,6 +52,58 @@ def test_route_stage(shape):
     route_parity(logits, idx.cpu().numpy(), w.cpu().numpy(), k)
 
 
+ROUTER_SHAPES = [  # T, d, E, router init, bias scale
+    (16, 6144, 256, "normal", 0.0),
+    (513, 6144, 256, "uniform", 0.0),
+    (300, 192, 64, "normal", 0.5),
+    (70, 320, 5, "uniform", 0.0),
+]
+
+
+@pytest.mark.parametrize("path", ["tc", "ffma"])
+@pytest.mark.parametrize("shape", ROUTER_SHAPES, ids=lambda s: "T{}_d{}_E{}_{}".format(*s[:4]))
+def test_router_logit_accuracy(shape, path, monkeypatch):
+    """Both score-GEMM paths (tensor cores with exact three-way bf16 split of W_r, and fp32
+    FFMA) against the fp64 logits.  The bar is half the 1e-5 margin below which a token's
+    routing is exempt, so no non-exempt token can change its experts through logit error."""
+    monkeypatch.setenv("MOE_ROUTER", path)
+    T, d, E, router, bs = shape
+    inp = make_small(T, d, E, min(8, E), 64, 1, seed=400 + T, router=router, bias_scale=bs)
+    dev = to_device(inp, "cuda")
+    h = moe.moe_create(d, E, min(8, E), 64, 1)
+    ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
+    idx = torch.empty(T, h.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, h.k, dtype=torch.float32, device="cuda")
+    moe.moe_route(h, dev.x, dev.W_router, dev.bias, idx, w, ws)
+    st, detail = moe.moe_device_status(h, T, ws)
+    assert st == moe.MOE_OK, hex(detail)
+    parts = moe.workspace_views(h, T, ws)["router_partials"].cpu().double().numpy()
+    got = parts.sum(0)
+    ref = oracle.router_logits(inp.x, inp.W_router, None)   # the bias is added by the top-k
+    err = np.abs(got - ref).max()
+    print(f"{path} T={T} d={d} E={E}: max |logit err| {err:.3e}, ksplit {parts.shape[0]}")
+    assert err < 5e-6, err
+    route_parity(oracle.router_logits(inp.x, inp.W_router, inp.bias), idx.cpu().numpy(),
+                 w.cpu().numpy(), h.k)
+
+
+@pytest.mark.parametrize("tiles", ["single", "pair"])
+@pytest.mark.parametrize("shape", [(64, 256, 16, 2, 128, 1, 0.0), (600, 256, 4, 2, 128, 1, 0.0),
+                                   (130, 320, 5, 3, 384, 2, 0.0)],
+                         ids=lambda s: "T{}_d{}_E{}_k{}_F{}_S{}".format(*s[:6]))
+def test_forward_both_gemm_tilings(shape, tiles, monkeypatch):
+    """The 1-SM (128-row) and 2-SM (256-row, cta_group::2) GEMM paths on the same inputs."""
+    monkeypatch.setenv("MOE_GEMM_TILES", tiles)
+    T, d, E, k, F, S, bs = shape
+    inp = make_small(T, d, E, k, F, S, seed=500 + T, bias_scale=bs)
+    y, v = gpu_forward(to_device(inp, "cuda"))
+    logits = oracle.router_logits(inp.x, inp.W_router, inp.bias)
+    exempt, idx_o, _ = route_parity(logits, v["topk_idx"].numpy(), v["topk_w"].numpy(), k)
+    idx_use = np.where(exempt[:, None], v["topk_idx"].numpy(), idx_o)
+    ref = oracle.forward(inp, idx_override=idx_use)
+    assert rel_err(y.float().numpy(), ref["y"]) < Y_REL_TOL
+
+
 @pytest.mark.parametrize("T,E,k", [(1, 1, 1), (5, 3, 2), (64, 16, 2), (700, 64, 8),
                                    (1500, 256, 8), (2000, 1024, 32), (8192, 256, 8)])
 def test_dispatch_stage(T, E, k):
