@@ -239,6 +239,20 @@ moe_status moe_set_stage_events(moe_handle h, void *const *events, int n_events)
 moe_status moe_dispatch_noalloc(moe_handle h, const int32_t *topk_idx, int T, int32_t *counts,
                                 int32_t *offsets, int32_t *perm, int32_t *pos, void *stream);
 
+/*
+ * Self-test of the failure path.  Every wait inside the library's kernels is
+ * bounded: when it expires the kernel records MOE_ERR_TIMEOUT in the
+ * workspace's status word and returns instead of hanging.  This call runs a
+ * one-CTA kernel that waits, through the same bounded wait, on a barrier that
+ * nothing completes, so the wait expires after timeout_ns (1 ns .. 2 s).
+ * Afterwards moe_device_status on this workspace (with any handle and
+ * T >= 0 whose layout starts at the same status word -- every layout does)
+ * reports MOE_ERR_TIMEOUT, and the device stays usable.  workspace: at least
+ * 1028 bytes of device memory.  Asynchronous on the stream.
+ */
+moe_status moe_selftest_wait_timeout(void *workspace, size_t ws_bytes,
+                                     unsigned long long timeout_ns, void *stream);
+
 /* Static text for a status code. */
 const char *moe_status_string(moe_status s);
 

@@ -36,7 +36,7 @@ MOE_ERR_ALIGNMENT = 7
 EXPORTS = ("moe_create", "moe_destroy", "moe_workspace_size", "moe_get_workspace_layout",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_host", "moe_device_status", "moe_set_stage_events",
-           "moe_dispatch_noalloc", "moe_status_string")
+           "moe_dispatch_noalloc", "moe_selftest_wait_timeout", "moe_status_string")
 MOE_STAGE_EVENTS = 7
 STAGE_NAMES = ("router", "dispatch", "gather", "gate_up_gemm", "down_gemm", "combine")
 
@@ -81,6 +81,7 @@ def load_library() -> ctypes.CDLL:
         "moe_device_status": ([P, I, P, P, ctypes.POINTER(ctypes.c_int32)], I),
         "moe_set_stage_events": ([P, ctypes.POINTER(P), I], I),
         "moe_dispatch_noalloc": ([P, P, I, P, P, P, P, P], I),
+        "moe_selftest_wait_timeout": ([P, Z, ctypes.c_ulonglong, P], I),
         "moe_status_string": ([I], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -289,6 +290,13 @@ def moe_set_stage_events(h: Handle, events) -> None:
         return
     arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
     _check(lib.moe_set_stage_events(h.value, arr, len(events)), "moe_set_stage_events")
+
+
+def moe_selftest_wait_timeout(workspace, timeout_ns: int, stream=None) -> None:
+    """Run a kernel whose bounded wait is made to expire (see include/moe.h)."""
+    wp, wn = _ws(workspace)
+    _check(load_library().moe_selftest_wait_timeout(wp, wn, int(timeout_ns), _stream(stream)),
+           "moe_selftest_wait_timeout")
 
 
 def moe_status_string(status: int) -> str:

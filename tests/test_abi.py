@@ -134,6 +134,9 @@ def test_host_side_argument_errors_need_no_device(lib):
     assert L.moe_forward(hv, None, None, None, None, None, None, None, None, None, 0, None, None,
                          0, None) == moe.MOE_OK
     assert L.moe_dispatch(hv, None, 0, None, None, None, None, None, 0, None) == moe.MOE_OK
+    assert L.moe_selftest_wait_timeout(None, 4096, 1000, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_wait_timeout(A, 4096, 0, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_wait_timeout(A, 4096, 3_000_000_000, None) == moe.MOE_ERR_INVALID_ARG
     # more rows than the supported envelope
     assert L.moe_route(hv, A, A, None, 1 << 23, A, A, A, 1 << 40, None) == \
         moe.MOE_ERR_UNSUPPORTED

@@ -266,6 +266,21 @@ def test_forward_is_deterministic_and_host_io_matches():
     assert torch.equal(y_host.view(torch.int16), outs[0].view(torch.int16))
 
 
+def test_bounded_wait_expires_with_a_status_and_the_device_stays_usable():
+    """Failure detection without a GPU fault: a wait that nothing completes gives up after
+    its limit (50 ms here), the host reads MOE_ERR_TIMEOUT, and the next forward is correct."""
+    h = moe.moe_create(256, 16, 2, 128, 1)
+    T = 64
+    ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
+    moe.moe_selftest_wait_timeout(ws, 50_000_000)
+    st, detail = moe.moe_device_status(h, T, ws)
+    assert st == moe.MOE_ERR_TIMEOUT and (detail >> 16) == 1, (st, hex(detail))
+    inp = make_inputs(WORKLOADS["tiny"], device="cpu")
+    y, v = gpu_forward(to_device(inp, "cuda"))          # status cleared, results correct
+    ref = oracle.forward(inp)
+    assert rel_err(y.float().numpy(), ref["y"]) < Y_REL_TOL
+
+
 def test_zero_tokens_is_a_no_op():
     h = moe.moe_create(256, 16, 2, 128, 1)
     ws = torch.empty(16, dtype=torch.uint8, device="cuda")
