@@ -253,6 +253,10 @@ moe_status moe_dispatch_noalloc(moe_handle h, const int32_t *topk_idx, int T, in
 moe_status moe_selftest_wait_timeout(void *workspace, size_t ws_bytes,
                                      unsigned long long timeout_ns, void *stream);
 
+/* Number of kernels one moe_forward call with T tokens launches (for launch
+ * accounting), or -1 for invalid arguments. */
+int moe_forward_kernel_count(moe_handle h, int T);
+
 /* Static text for a status code. */
 const char *moe_status_string(moe_status s);
 

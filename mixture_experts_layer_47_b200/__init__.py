@@ -36,7 +36,8 @@ MOE_ERR_ALIGNMENT = 7
 EXPORTS = ("moe_create", "moe_destroy", "moe_workspace_size", "moe_get_workspace_layout",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_host", "moe_device_status", "moe_set_stage_events",
-           "moe_dispatch_noalloc", "moe_selftest_wait_timeout", "moe_status_string")
+           "moe_dispatch_noalloc", "moe_selftest_wait_timeout", "moe_forward_kernel_count",
+           "moe_status_string")
 MOE_STAGE_EVENTS = 7
 STAGE_NAMES = ("router", "dispatch", "gather", "gate_up_gemm", "down_gemm", "combine")
 
@@ -82,6 +83,7 @@ def load_library() -> ctypes.CDLL:
         "moe_set_stage_events": ([P, ctypes.POINTER(P), I], I),
         "moe_dispatch_noalloc": ([P, P, I, P, P, P, P, P], I),
         "moe_selftest_wait_timeout": ([P, Z, ctypes.c_ulonglong, P], I),
+        "moe_forward_kernel_count": ([P, I], I),
         "moe_status_string": ([I], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -297,6 +299,10 @@ def moe_selftest_wait_timeout(workspace, timeout_ns: int, stream=None) -> None:
     wp, wn = _ws(workspace)
     _check(load_library().moe_selftest_wait_timeout(wp, wn, int(timeout_ns), _stream(stream)),
            "moe_selftest_wait_timeout")
+
+
+def moe_forward_kernel_count(h: Handle, T: int) -> int:
+    return int(load_library().moe_forward_kernel_count(h.value, int(T)))
 
 
 def moe_status_string(status: int) -> str:

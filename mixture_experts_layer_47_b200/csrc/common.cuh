@@ -295,6 +295,19 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mas
       : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the forward is launched with
+// programmatic stream serialisation, so it may start while its predecessor on
+// the stream is still running.  pdl_wait() blocks until the predecessor has
+// completed and its writes are visible: call it before reading any global data
+// (a no-op when the kernel was launched without the attribute).
+// pdl_launch_dependents() lets the successor start launching.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

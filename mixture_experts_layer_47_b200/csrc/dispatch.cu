@@ -31,6 +31,8 @@ __global__ void __launch_bounds__(kCountThreads)
     dispatch_count_kernel(const int32_t* __restrict__ idx, int n, int E,
                           int32_t* __restrict__ blk_hist, int* status) {
   extern __shared__ int32_t hist[];
+  pdl_wait();
+  pdl_launch_dependents();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   const int beg = blockIdx.x * kDispatchChunk;
@@ -98,6 +100,8 @@ __global__ void __launch_bounds__(kScanThreads)
                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                          int32_t* __restrict__ sched) {
   __shared__ int warp_sums[32];
+  pdl_wait();
+  pdl_launch_dependents();
   const int e = threadIdx.x;
   int c = 0;
   if (e < E) {
@@ -124,6 +128,8 @@ __global__ void __launch_bounds__(kScanThreads)
     schedule_from_offsets_kernel(const int32_t* __restrict__ offsets, int E, int S, int T,
                                  int32_t* __restrict__ sched) {
   __shared__ int warp_sums[32];
+  pdl_wait();
+  pdl_launch_dependents();
   const int e = threadIdx.x;
   int c = 0;
   // A group never holds more than T slots (a token picks an expert once).
@@ -136,6 +142,8 @@ __global__ void __launch_bounds__(kScatterWarps * 32)
                             const int32_t* __restrict__ blk_base, int32_t* __restrict__ perm,
                             int32_t* __restrict__ pos) {
   extern __shared__ int32_t cnt[];  // [kScatterWarps][E]
+  pdl_wait();
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kScatterWarps * E; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
@@ -194,6 +202,8 @@ __global__ void __launch_bounds__(kScanThreads)
                            int32_t* __restrict__ sched, int* status) {
   extern __shared__ int32_t cnt[];  // [kSingleWarps][E]
   __shared__ int warp_sums[32];
+  pdl_wait();
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kSingleWarps * E; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
@@ -259,27 +269,25 @@ cudaError_t launch_dispatch(const Ctx& c, const int32_t* topk_idx, int T, int nb
                             int32_t* pos, int32_t* sched, int* status, cudaStream_t st) {
   const int n = T * c.k;
   if (n <= kDispatchChunk && c.E <= kSingleMaxExperts) {
-    dispatch_single_kernel<<<1, kScanThreads, kSingleWarps * c.E * sizeof(int32_t), st>>>(
-        topk_idx, n, c.E, c.S, T, counts, offsets, perm, pos, sched, status);
-    return cudaGetLastError();
+    return launch_pdl(dispatch_single_kernel, dim3(1), dim3(kScanThreads),
+                      kSingleWarps * c.E * sizeof(int32_t), st, 1, topk_idx, n, c.E, c.S, T,
+                      counts, offsets, perm, pos, sched, status);
   }
-  dispatch_count_kernel<<<nblk, kCountThreads, c.E * sizeof(int32_t), st>>>(topk_idx, n, c.E,
-                                                                            blk_hist, status);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_pdl(dispatch_count_kernel, dim3(nblk), dim3(kCountThreads),
+                               c.E * sizeof(int32_t), st, 1, topk_idx, n, c.E, blk_hist, status);
   if (err != cudaSuccess) return err;
-  dispatch_scan_kernel<<<1, kScanThreads, 0, st>>>(blk_hist, nblk, c.E, c.S, T, counts, offsets,
-                                                   sched);
-  err = cudaGetLastError();
+  err = launch_pdl(dispatch_scan_kernel, dim3(1), dim3(kScanThreads), 0, st, 1, blk_hist, nblk,
+                   c.E, c.S, T, counts, offsets, sched);
   if (err != cudaSuccess) return err;
-  dispatch_scatter_kernel<<<nblk, kScatterWarps * 32, kScatterWarps * c.E * sizeof(int32_t),
-                            st>>>(topk_idx, n, c.E, blk_hist, perm, pos);
-  return cudaGetLastError();
+  return launch_pdl(dispatch_scatter_kernel, dim3(nblk), dim3(kScatterWarps * 32),
+                    kScatterWarps * c.E * sizeof(int32_t), st, 1, topk_idx, n, c.E,
+                    static_cast<const int32_t*>(blk_hist), perm, pos);
 }
 
 cudaError_t launch_schedule_from_offsets(const Ctx& c, const int32_t* offsets, int T,
                                          int32_t* sched, cudaStream_t st) {
-  schedule_from_offsets_kernel<<<1, kScanThreads, 0, st>>>(offsets, c.E, c.S, T, sched);
-  return cudaGetLastError();
+  return launch_pdl(schedule_from_offsets_kernel, dim3(1), dim3(kScanThreads), 0, st, 1, offsets,
+                    c.E, c.S, T, sched);
 }
 
 }  // namespace moe

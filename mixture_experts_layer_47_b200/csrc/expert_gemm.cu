@@ -159,8 +159,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int unit = kPair ? int(blockIdx.x >> 1) : int(blockIdx.x);        // this pair / CTA
   const int n_units = kPair ? int(gridDim.x >> 1) : int(gridDim.x);
 
-  for (int i = threadIdx.x; i <= G; i += NUM_THREADS) ss.sched[i] = p.sched[i];
-  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) ss.offsets[i] = p.offsets[i];
+  // Prologue that reads no global data (overlaps the previous kernel under PDL).
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&ss.full[s], 1);
@@ -193,6 +192,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_relinquish();
     }
   }
+  pdl_wait();   // the schedule, offsets and A operands come from earlier kernels
+  pdl_launch_dependents();
+  for (int i = threadIdx.x; i <= G; i += NUM_THREADS) ss.sched[i] = p.sched[i];
+  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) ss.offsets[i] = p.offsets[i];
   tc_fence_before();
   if (kPair) cluster_sync_all(); else __syncthreads();   // barriers of both CTAs initialised
   tc_fence_after();
@@ -467,21 +470,9 @@ cudaError_t set_attrs() {
 
 template <bool kGateUp, bool kPair>
 cudaError_t launch_gemm(const GemmParams& gp, int num_sms, cudaStream_t st) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kPair ? unsigned(num_sms & ~1) : unsigned(num_sms));
-  cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = smem_bytes<kPair>();
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  if (kPair) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kGateUp, kPair>, gp);
+  const unsigned grid = kPair ? unsigned(num_sms & ~1) : unsigned(num_sms);
+  return launch_pdl(grouped_gemm_kernel<kGateUp, kPair>, dim3(grid), dim3(NUM_THREADS),
+                    smem_bytes<kPair>(), st, kPair ? 2 : 1, gp);
 }
 
 }  // namespace

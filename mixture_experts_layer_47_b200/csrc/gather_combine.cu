@@ -24,6 +24,8 @@ __global__ void __launch_bounds__(kGatherThreads)
     gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
                        const int32_t* __restrict__ offsets, int T, int k, int E, int d,
                        uint16_t* __restrict__ x_perm) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int nslots = T * k;
   const int nrows = min(nslots, max(0, offsets[E]));
   const int warps_total = gridDim.x * (kGatherThreads / 32);
@@ -73,6 +75,8 @@ __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const TY* __restrict__ Y, const float* __restrict__ topk_w,
                    const int32_t* __restrict__ pos, int T, int k, int S, int d,
                    uint16_t* __restrict__ y) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int t = blockIdx.x;
   const int c = (blockIdx.y * kCombineThreads + threadIdx.x) * 8;
   if (c >= d) return;
@@ -110,25 +114,22 @@ cudaError_t launch_gather(const Ctx& c, const uint16_t* x, const int32_t* perm,
   int blocks = (rows + warps_per_block - 1) / warps_per_block;
   blocks = blocks < num_sms * 8 ? blocks : num_sms * 8;
   if (blocks < 1) blocks = 1;
-  gather_rows_kernel<<<blocks, kGatherThreads, 0, st>>>(x, perm, offsets, T, c.k, c.E, c.d,
-                                                        x_perm);
-  return cudaGetLastError();
+  return launch_pdl(gather_rows_kernel, dim3(blocks), dim3(kGatherThreads), 0, st, 1, x, perm,
+                    offsets, T, c.k, c.E, c.d, x_perm);
 }
 
 cudaError_t launch_combine(const Ctx& c, const float* Y, const float* topk_w, const int32_t* pos,
                            int T, uint16_t* y, cudaStream_t st) {
   dim3 grid(T, (c.d / 8 + kCombineThreads - 1) / kCombineThreads);
-  combine_kernel<float, RowF32><<<grid, kCombineThreads, 0, st>>>(Y, topk_w, pos, T, c.k, c.S,
-                                                                 c.d, y);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel<float, RowF32>, grid, dim3(kCombineThreads), 0, st, 1, Y,
+                    topk_w, pos, T, c.k, c.S, c.d, y);
 }
 
 cudaError_t launch_combine_bf16(const Ctx& c, const uint16_t* Y, const float* topk_w,
                                 const int32_t* pos, int T, uint16_t* y, cudaStream_t st) {
   dim3 grid(T, (c.d / 8 + kCombineThreads - 1) / kCombineThreads);
-  combine_kernel<uint16_t, RowBF16><<<grid, kCombineThreads, 0, st>>>(Y, topk_w, pos, T, c.k,
-                                                                      c.S, c.d, y);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel<uint16_t, RowBF16>, grid, dim3(kCombineThreads), 0, st, 1, Y,
+                    topk_w, pos, T, c.k, c.S, c.d, y);
 }
 
 }  // namespace moe

@@ -441,6 +441,16 @@ moe_status moe_device_status(moe_handle h, int T, const void* workspace, void* s
   return (word >> 16) == kDevBadIndex ? MOE_ERR_BAD_INDEX : MOE_ERR_TIMEOUT;
 }
 
+int moe_forward_kernel_count(moe_handle h, int T) {
+  if (!h || T < 0 || check_T(h->c, T) != MOE_OK) return -1;
+  if (T == 0) return 0;
+  const Ctx& c = h->c;
+  const RouterPlan rp = router_plan(c, T, kPlanSms);
+  const int router = rp.tc ? 3 : 2;  // [weight split +] score GEMM + top-k
+  const int dispatch = (int64_t(T) * c.k <= kDispatchChunk && c.E <= 256) ? 1 : 3;
+  return router + dispatch + 1 /*gather*/ + 2 /*GEMMs*/ + 1 /*combine*/;
+}
+
 moe_status moe_set_stage_events(moe_handle h, void* const* events, int n_events) {
   if (!h) return MOE_ERR_INVALID_ARG;
   if (!events || n_events == 0) {

@@ -54,6 +54,8 @@ __global__ void __launch_bounds__(kRouterThreads)
   __shared__ __align__(16) float xs[2][kBK][BT + 4];
   __shared__ __align__(16) float ws[2][kBK][BE + 4];
 
+  pdl_wait();
+  pdl_launch_dependents();
   const int tid = threadIdx.x;
   const int tx = tid % NTX, ty = tid / NTX;
   const int t0 = blockIdx.x * BT, e0 = blockIdx.y * BE;
@@ -174,6 +176,8 @@ __global__ void __launch_bounds__(1024)
                        int k, int ksplit, int32_t* __restrict__ topk_idx,
                        float* __restrict__ topk_w) {
   extern __shared__ float logit[];  // [E]
+  pdl_wait();
+  pdl_launch_dependents();
   const int t = blockIdx.x;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     float s = 0.f;
@@ -238,9 +242,8 @@ template <int BT, int BE, int TT, int TE>
 cudaError_t launch_partial(const Ctx& c, const RouterPlan& rp, const uint16_t* x, const float* Wr,
                            int T, float* part, cudaStream_t st) {
   dim3 grid((T + BT - 1) / BT, (c.E + BE - 1) / BE, rp.ksplit);
-  router_partial_kernel<BT, BE, TT, TE><<<grid, kRouterThreads, 0, st>>>(x, Wr, T, c.d, c.E,
-                                                                         rp.kchunk, part);
-  return cudaGetLastError();
+  return launch_pdl(router_partial_kernel<BT, BE, TT, TE>, grid, dim3(kRouterThreads), 0, st, 1,
+                    x, Wr, T, c.d, c.E, rp.kchunk, part);
 }
 
 }  // namespace
@@ -303,9 +306,9 @@ cudaError_t launch_router(const Ctx& c, const RouterPlan& rp, const uint16_t* x,
     err = launch_partial<128, 128, 8, 8>(c, rp, x, Wr, T, part, st);
   if (err != cudaSuccess) return err;
   const int threads = std::min(1024, std::max(32, (c.E + 31) / 32 * 32));
-  router_topk_kernel<<<T, threads, c.E * sizeof(float), st>>>(part, bias, T, c.E, c.k, rp.ksplit,
-                                                              topk_idx, topk_w);
-  return cudaGetLastError();
+  return launch_pdl(router_topk_kernel, dim3(T), dim3(threads), c.E * sizeof(float), st, 1,
+                    static_cast<const float*>(part), bias, T, c.E, c.k, rp.ksplit, topk_idx,
+                    topk_w);
 }
 
 }  // namespace moe

@@ -95,6 +95,8 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     tmem_alloc(&ss.tmem_base, RT_RING * RT_BN);
     tmem_relinquish();
   }
+  pdl_wait();   // x and the split weights come from earlier work on the stream
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -257,6 +259,8 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
 __global__ void __launch_bounds__(256)
     split_router_weights_kernel(const float* __restrict__ Wr, size_t n,
                                 uint16_t* __restrict__ parts) {
+  pdl_wait();
+  pdl_launch_dependents();
   for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n;
        i += size_t(gridDim.x) * blockDim.x) {
     const float w = Wr[i];
@@ -320,9 +324,9 @@ cudaError_t launch_router_tc(const Ctx& c, int ksplit, const uint16_t* x, const 
     attr_device = dev;
   }
   const size_t n = size_t(c.E) * c.d;
-  split_router_weights_kernel<<<(unsigned)std::min<size_t>((n + 255) / 256, 4096), 256, 0, st>>>(
-      Wr, n, wparts);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_pdl(split_router_weights_kernel,
+                               dim3((unsigned)std::min<size_t>((n + 255) / 256, 4096)), dim3(256),
+                               0, st, 1, Wr, n, wparts);
   if (err != cudaSuccess) return err;
   RouterTcParams p;
   memset(&p, 0, sizeof p);
@@ -337,8 +341,7 @@ cudaError_t launch_router_tc(const Ctx& c, int ksplit, const uint16_t* x, const 
   p.ksplit = ksplit;
   const int tiles = ((T + RT_BM - 1) / RT_BM) * ((c.E + RT_BN - 1) / RT_BN) * ksplit;
   const int grid = std::min(tiles, num_sms > 0 ? num_sms : 148);
-  router_tc_kernel<<<grid, RT_THREADS, kRtSmem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(router_tc_kernel, dim3(grid), dim3(RT_THREADS), kRtSmem, st, 1, p);
 }
 
 }  // namespace moe

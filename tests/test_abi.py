@@ -24,7 +24,7 @@ def lib():
 
 def declared_symbols():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:moe_status|size_t|const char \*)\s*(moe_\w+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:moe_status|size_t|int|const char \*)\s*(moe_\w+)\s*\(",
                                  text, re.M)))
 
 
