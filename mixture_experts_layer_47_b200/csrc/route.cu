@@ -167,19 +167,26 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
   return v > bv || (v == bv && e < be);
 }
 
-// One CTA per token: thread e adds the K-chunk partials of expert e in chunk
-// order (plus the bias) into shared memory; warp 0 then takes k rounds of a
-// warp arg-max (value desc, expert asc) over the E logits and writes the
-// experts and their renormalised softmax gates.
+// TPC tokens per CTA.  The threads of a token add the K-chunk partials of its
+// experts in chunk order (plus the bias) into shared memory; the token's first
+// warp then takes k rounds of a warp arg-max (value desc, expert asc) over the E
+// logits and writes the experts and their renormalised softmax gates.
+// TPC = 1 (all of a CTA's threads per token) suits many partials per logit (the
+// small-batch split); TPC = 8 (a warp per token) suits few.
+template <int TPC>
 __global__ void __launch_bounds__(1024)
     router_topk_kernel(const float* __restrict__ part, const float* __restrict__ bias, int T, int E,
                        int k, int ksplit, int32_t* __restrict__ topk_idx,
                        float* __restrict__ topk_w) {
-  extern __shared__ float logit[];  // [E]
+  extern __shared__ float logit_all[];  // [TPC][E]
   pdl_wait();
   pdl_launch_dependents();
-  const int t = blockIdx.x;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+  const int per_tok = blockDim.x / TPC;                 // threads per token
+  const int grp = threadIdx.x / per_tok, tid = threadIdx.x % per_tok;
+  const int t = blockIdx.x * TPC + grp;
+  if (t >= T) return;   // whole token groups (warps) leave together
+  float* logit = logit_all + grp * E;
+  for (int e = tid; e < E; e += per_tok) {
     float s = 0.f;
     const float* p = part + size_t(t) * E + e;
     const size_t stride = size_t(T) * E;
@@ -195,9 +202,9 @@ __global__ void __launch_bounds__(1024)
     if (bias) s += bias[e];
     logit[e] = (s == s) ? s : -INFINITY;  // a NaN score is never preferred
   }
-  __syncthreads();
-  if (threadIdx.x >= 32) return;
-  const int lane = threadIdx.x;
+  if (TPC == 1) __syncthreads(); else __syncwarp();
+  if (tid >= 32) return;
+  const int lane = tid;
   float my_l = 0.f, l0 = 0.f;
   int my_e = 0;
   for (int i = 0; i < k; ++i) {
@@ -305,8 +312,12 @@ cudaError_t launch_router(const Ctx& c, const RouterPlan& rp, const uint16_t* x,
   else
     err = launch_partial<128, 128, 8, 8>(c, rp, x, Wr, T, part, st);
   if (err != cudaSuccess) return err;
+  if (rp.ksplit <= 4)   // a warp per token, 8 tokens per CTA
+    return launch_pdl(router_topk_kernel<8>, dim3((T + 7) / 8), dim3(256), 8 * c.E * sizeof(float),
+                      st, 1, static_cast<const float*>(part), bias, T, c.E, c.k, rp.ksplit,
+                      topk_idx, topk_w);
   const int threads = std::min(1024, std::max(32, (c.E + 31) / 32 * 32));
-  return launch_pdl(router_topk_kernel, dim3(T), dim3(threads), c.E * sizeof(float), st, 1,
+  return launch_pdl(router_topk_kernel<1>, dim3(T), dim3(threads), c.E * sizeof(float), st, 1,
                     static_cast<const float*>(part), bias, T, c.E, c.k, rp.ksplit, topk_idx,
                     topk_w);
 }

@@ -10,7 +10,7 @@
 //    lo = bf16(W_r - hi - mid); the residual is below 2^-24 |W_r|).  Every
 //    product of a bf16 x with a bf16 part is exact in fp32.
 //  * Whatever rounding the tensor core's fp32 accumulation applies, it is
-//    confined to one 64-wide K chunk: each chunk's 12 MMAs (4 K16 steps x 3
+//    confined to one 128-wide K chunk: each chunk's 24 MMAs (8 K16 steps x 3
 //    parts) go into a fresh TMEM accumulator, and the epilogue warps add the
 //    chunk results in fp32 on the CUDA cores, in chunk order (deterministic).
 // Layout: a persistent kernel, one CTA per SM, 192 threads.  Warp 0 issues TMA
@@ -38,6 +38,7 @@ constexpr int RT_A_BYTES = RT_BM * RT_BK * 2;
 constexpr int RT_B_BYTES = RT_BN * RT_BK * 2;
 constexpr int RT_STAGE_BYTES = RT_A_BYTES + 3 * RT_B_BYTES;
 constexpr int RT_RING = 8;          // accumulators of RT_BN columns
+constexpr int RT_CHUNK_KB = 2;      // 64-wide K blocks accumulated per chunk (K = 128)
 constexpr int RT_THREADS = 192;
 constexpr uint32_t RT_IDESC = umma_idesc_bf16_f32(RT_BM, RT_BN);
 
@@ -72,7 +73,8 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
   const int tiles_m = (p.T + RT_BM - 1) / RT_BM;
   const int tiles_n = (p.E + RT_BN - 1) / RT_BN;
   const int total = tiles_m * tiles_n * p.ksplit;
-  const int kblocks = p.d / RT_BK / p.ksplit;   // K chunks per tile
+  const int kblocks = p.d / RT_BK / p.ksplit;   // K blocks per tile
+  const int nchunks = (kblocks + RT_CHUNK_KB - 1) / RT_CHUNK_KB;   // chunks per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < RT_STAGES; ++s) {
@@ -157,35 +159,44 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
       bool stop = false;
       for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
         if (*abort_flag) break;
-        for (int kb = 0; kb < kblocks; ++kb, ++chunk) {
+        int kb = 0;
+        for (int ch = 0; ch < nchunks && !stop; ++ch, ++chunk) {
           const uint32_t slot = chunk % RT_RING;
           const uint32_t use = chunk / RT_RING;
-          if (!mbar_wait(&ss.chunk_free[slot], (use & 1u) ^ 1u) ||
-              !mbar_wait(&ss.full[stage], phase)) {
+          if (!mbar_wait(&ss.chunk_free[slot], (use & 1u) ^ 1u)) {
             report_error(p.status, kDevTimeout, kSiteMma);
             *abort_flag = 1;
             stop = true;
             break;
           }
-          tc_fence_after();
-          const uint32_t st = smem_u32(smem + stage * RT_STAGE_BYTES);
-          const uint64_t a_desc = umma_desc_sw128_kmajor(st);
           const uint32_t d_tmem = tmem_base + slot * RT_BN;
-#pragma unroll
-          for (int kk = 0; kk < RT_BK / 16; ++kk)
-#pragma unroll
-            for (int part = 0; part < 3; ++part) {
-              const uint64_t b_desc =
-                  umma_desc_sw128_kmajor(st + RT_A_BYTES + part * RT_B_BYTES);
-              umma_bf16(d_tmem, a_desc + uint64_t(2 * kk), b_desc + uint64_t(2 * kk), RT_IDESC,
-                        (kk | part) != 0 ? 1u : 0u);
+          for (int sub = 0; sub < RT_CHUNK_KB && kb < kblocks; ++sub, ++kb) {
+            if (!mbar_wait(&ss.full[stage], phase)) {
+              report_error(p.status, kDevTimeout, kSiteMma);
+              *abort_flag = 1;
+              stop = true;
+              break;
             }
-          umma_commit(&ss.empty[stage]);
-          umma_commit(&ss.chunk_full[slot]);
-          if (++stage == RT_STAGES) {
-            stage = 0;
-            phase ^= 1;
+            tc_fence_after();
+            const uint32_t st = smem_u32(smem + stage * RT_STAGE_BYTES);
+            const uint64_t a_desc = umma_desc_sw128_kmajor(st);
+#pragma unroll
+            for (int kk = 0; kk < RT_BK / 16; ++kk)
+#pragma unroll
+              for (int part = 0; part < 3; ++part) {
+                const uint64_t b_desc =
+                    umma_desc_sw128_kmajor(st + RT_A_BYTES + part * RT_B_BYTES);
+                umma_bf16(d_tmem, a_desc + uint64_t(2 * kk), b_desc + uint64_t(2 * kk),
+                          RT_IDESC, (sub | kk | part) != 0 ? 1u : 0u);
+              }
+            umma_commit(&ss.empty[stage]);
+            if (++stage == RT_STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
+          if (stop) break;
+          umma_commit(&ss.chunk_full[slot]);
         }
       }
       umma_commit(&ss.mma_done);
@@ -205,7 +216,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
       float sum[RT_BN];
 #pragma unroll
       for (int j = 0; j < RT_BN; ++j) sum[j] = 0.f;
-      for (int kb = 0; kb < kblocks; ++kb, ++chunk) {
+      for (int ch = 0; ch < nchunks; ++ch, ++chunk) {
         if (__any_sync(0xffffffffu, *abort_flag != 0)) { stop = true; break; }
         const uint32_t slot = chunk % RT_RING;
         const uint32_t use = chunk / RT_RING;
@@ -217,13 +228,14 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + lane_addr + slot * RT_BN;
+        uint32_t v0[32], v1[32];   // both halves in flight, one wait
+        tmem_ld_32cols(taddr, v0);
+        tmem_ld_32cols(taddr + 32u, v1);
+        tmem_ld_wait();
 #pragma unroll
-        for (int h = 0; h < RT_BN / 32; ++h) {
-          uint32_t v[32];
-          tmem_ld_32cols(taddr + uint32_t(32 * h), v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) sum[32 * h + j] += __uint_as_float(v[j]);
+        for (int j = 0; j < 32; ++j) {
+          sum[j] += __uint_as_float(v0[j]);
+          sum[32 + j] += __uint_as_float(v1[j]);
         }
         tc_fence_before();
         mbar_arrive(&ss.chunk_free[slot]);
