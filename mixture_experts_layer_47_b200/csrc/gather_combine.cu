@@ -2,8 +2,10 @@
 //
 //  gather   X_perm[p] = x[perm[p] / k] for every routed slot position p, so each
 //           expert's tokens form one contiguous run of rows for the grouped
-//           GEMM's TMA loads (the shared expert reads x directly).  One warp
-//           copies one row with 16-byte loads and stores.
+//           GEMM's TMA loads (the shared expert reads x directly).  Inside
+//           moe_forward a warp takes a token, reads its row once and writes it
+//           to its k positions (pos); moe_expert_ffn, given perm only, copies
+//           position by position.
 //  combine  the merge of the chosen experts' results into the layer output
 //           (m.xxqk.cn Hy4-preview MoE explainer, section 2.2; the shared
 //           expert of the ZAKER release news is added with weight 1):
@@ -46,6 +48,43 @@ __global__ void __launch_bounds__(kGatherThreads)
       dst[i + 96] = e;
     }
     for (; i < vec; i += 32) dst[i] = src[i];
+  }
+}
+
+// Token-major gather: one warp reads a token's row of x once (in chunks held in
+// registers) and writes it to the token's k positions pos[t*k + i].  x is read
+// once instead of k times, so the X_perm write stream cannot push it out of L2.
+__global__ void __launch_bounds__(kGatherThreads)
+    gather_tokens_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ pos, int T,
+                         int k, int d, uint16_t* __restrict__ x_perm) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int nslots = T * k;
+  const int warps_total = gridDim.x * (kGatherThreads / 32);
+  const int lane = threadIdx.x & 31;
+  const int vec = d / 8;  // 16-byte vectors per row
+  constexpr int kChunk = 8;  // vectors per lane held at once
+  for (int t = blockIdx.x * (kGatherThreads / 32) + (threadIdx.x >> 5); t < T;
+       t += warps_total) {
+    const uint4* __restrict__ src = reinterpret_cast<const uint4*>(x + size_t(t) * d);
+    for (int base = 0; base < vec; base += 32 * kChunk) {
+      uint4 v[kChunk];
+#pragma unroll
+      for (int j = 0; j < kChunk; ++j) {
+        const int i = base + lane + 32 * j;
+        if (i < vec) v[j] = src[i];
+      }
+      for (int c = 0; c < k; ++c) {
+        const int p = pos[size_t(t) * k + c];
+        if (p < 0 || p >= nslots) continue;
+        uint4* __restrict__ dst = reinterpret_cast<uint4*>(x_perm + size_t(p) * d);
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) {
+          const int i = base + lane + 32 * j;
+          if (i < vec) dst[i] = v[j];
+        }
+      }
+    }
   }
 }
 
@@ -116,6 +155,16 @@ cudaError_t launch_gather(const Ctx& c, const uint16_t* x, const int32_t* perm,
   if (blocks < 1) blocks = 1;
   return launch_pdl(gather_rows_kernel, dim3(blocks), dim3(kGatherThreads), 0, st, 1, x, perm,
                     offsets, T, c.k, c.E, c.d, x_perm);
+}
+
+cudaError_t launch_gather_tokens(const Ctx& c, const uint16_t* x, const int32_t* pos, int T,
+                                 uint16_t* x_perm, int num_sms, cudaStream_t st) {
+  const int warps_per_block = kGatherThreads / 32;
+  int blocks = (T + warps_per_block - 1) / warps_per_block;
+  blocks = blocks < num_sms * 8 ? blocks : num_sms * 8;
+  if (blocks < 1) blocks = 1;
+  return launch_pdl(gather_tokens_kernel, dim3(blocks), dim3(kGatherThreads), 0, st, 1, x, pos,
+                    T, c.k, c.d, x_perm);
 }
 
 cudaError_t launch_combine(const Ctx& c, const float* Y, const float* topk_w, const int32_t* pos,

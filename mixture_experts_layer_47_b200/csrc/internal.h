@@ -97,6 +97,9 @@ cudaError_t launch_gather(const Ctx& c, const uint16_t* x, const int32_t* perm,
                           const int32_t* offsets, int T, uint16_t* x_perm, int num_sms,
                           cudaStream_t st);
 
+cudaError_t launch_gather_tokens(const Ctx& c, const uint16_t* x, const int32_t* pos, int T,
+                                 uint16_t* x_perm, int num_sms, cudaStream_t st);
+
 cudaError_t launch_combine(const Ctx& c, const float* Y, const float* topk_w, const int32_t* pos,
                            int T, uint16_t* y, cudaStream_t st);
 cudaError_t launch_combine_bf16(const Ctx& c, const uint16_t* Y, const float* topk_w,

@@ -334,7 +334,7 @@ static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W
                                        offsets, perm, pos, sched, status, st))))
     return s;
   if ((s = mark(2))) return s;
-  if ((s = cuda_status(launch_gather(c, x, perm, offsets, T, x_perm, dev->num_sms, st)))) return s;
+  if ((s = cuda_status(launch_gather_tokens(c, x, pos, T, x_perm, dev->num_sms, st)))) return s;
   if ((s = mark(3))) return s;
   FfnArgs a;
   a.x = x;
