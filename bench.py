@@ -190,10 +190,13 @@ def measured_traffic(kernel: str, bound: str, units: int):
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        entry = json.load(f).get(kernel)
+        entry = json.load(f).get(f"{kernel}/{bound}")
     if not entry or entry.get("bound") != bound:
         return None
-    src = os.path.join(ROOT, "mixture_experts_layer_47_b200", "csrc", "expert_gemm.cu")
+    src = os.path.join(ROOT, "mixture_experts_layer_47_b200", "csrc",
+                       entry.get("kernel_source", "expert_gemm.cu"))
+    if not os.path.exists(src):
+        return None
     with open(src, "rb") as f:
         if hashlib.sha256(f.read()).hexdigest() != entry["kernel_source_sha256"]:
             return None

@@ -9,7 +9,7 @@
 //                     (integer atomics: the counts do not depend on order);
 //   dispatch_scan     one CTA: for every expert the exclusive prefix over
 //                     blocks, counts, the exclusive scan over experts
-//                     (offsets), and the grouped GEMM's M-tile schedule;
+//                     (offsets), and the grouped GEMMs' tile schedules;
 //   dispatch_scatter  per block, each warp owns a contiguous run of slots;
 //                     __match_any_sync gives each slot its rank among equal
 //                     experts in the warp; per-warp, per-expert running
@@ -25,7 +25,7 @@ namespace {
 constexpr int kCountThreads = 512;
 constexpr int kScatterWarps = 8;
 constexpr int kScanThreads = 1024;
-constexpr int kTileM = 128;   // rows per grouped-GEMM M tile
+constexpr int kTileM = 128;   // rows (tokens) per grouped-GEMM tile of the 1-SM tilings
 
 __global__ void __launch_bounds__(kCountThreads)
     dispatch_count_kernel(const int32_t* __restrict__ idx, int n, int E,
@@ -77,7 +77,9 @@ __device__ int block_inclusive_scan(int v, int* warp_sums) {
 
 // Grouped-GEMM schedules: sched[g] = sum over groups g' < g of ceil(rows_g' / 128),
 // routed groups first (rows = count), then S shared groups of T rows each; the
-// same for 256-row tiles (the 2-SM GEMM) at sched[G + 1 + g], G = E + S.
+// same for 256-row tiles (the 2-SM GEMMs) at sched[G + 1 + g], G = E + S.  The
+// row-tiled GEMMs read them as M tiles per group, the weight-major ones as
+// token tiles per group.
 __device__ void write_schedule(int count, int E, int S, int T, int32_t* sched, int* warp_sums) {
   const int e = threadIdx.x;
   const int G1 = E + S + 1;

@@ -29,10 +29,10 @@
 #include <string.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
+#include "tensor_map.cuh"
 
 namespace moe {
 namespace {
@@ -432,33 +432,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ---------------------------------------------------------------------------
 // Host side: tensor maps and launches.
 // ---------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-
-bool get_encoder() {
-  std::call_once(g_encode_once, [] {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  });
-  return g_encode != nullptr;
-}
-
-// 2-D bf16 tensor [rows][cols] (cols contiguous), box [box_rows][64], 128-byte
-// swizzle, out-of-bounds elements read as zero.
 bool encode_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, int box_rows) {
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {uint32_t(BK), uint32_t(box_rows)};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode_bf16_2d(map, base, rows, cols, box_rows);
 }
 
 template <bool kGateUp, bool kPair>
@@ -477,21 +452,28 @@ cudaError_t launch_gemm(const GemmParams& gp, int num_sms, cudaStream_t st) {
 
 }  // namespace
 
-// Tile choice.  A group of c rows costs ceil(c / M) tiles of M rows of tensor work;
-// with M = 256 (2-SM pairs) the padding averages ~128 rows per group against ~64
-// for M = 128, which outweighs the pair kernel's higher MMA rate until groups
-// average about 1024 rows.  MOE_GEMM_TILES=single|pair overrides the choice
-// (both compute the same result; for tuning and tests).
-bool use_pair_tiles(const Ctx& c, int T) {
+// Tile choice.  The row-tiled kernels here pay ceil(c / M) M-tiles for a group
+// of c rows (M = 128, or 256 for 2-SM pairs).  The weight-major kernels
+// (expert_gemm_swap.cu) put the weights on the MMA's M side and pad each token
+// tile only to a multiple of 16; measured on B200 at d = 6144, d_ff = 2048,
+// 256 experts top-8, they are faster at every batch: the 1-SM form while
+// groups average fewer than 96 rows, the 2-SM form (half the shared-memory
+// traffic per MMA cycle, token tiles up to 256) from there on.
+// MOE_GEMM_TILES=single|pair|swap|swap_pair overrides the choice (all compute
+// the same result; for tuning and tests).
+GemmTiling gemm_tiling(const Ctx& c, int T) {
   const char* v = getenv("MOE_GEMM_TILES");
-  if (v && strcmp(v, "pair") == 0) return true;
-  if (v && strcmp(v, "single") == 0) return false;
-  return int64_t(T) * c.k >= int64_t(1024) * c.E;
+  if (v && strcmp(v, "pair") == 0) return GemmTiling::kPair;
+  if (v && strcmp(v, "single") == 0) return GemmTiling::kSingle;
+  if (v && strcmp(v, "swap") == 0) return GemmTiling::kSwap;
+  if (v && strcmp(v, "swap_pair") == 0) return GemmTiling::kSwapPair;
+  return int64_t(T) * c.k >= int64_t(kSwapPairMinRowsPerExpert) * c.E ? GemmTiling::kSwapPair
+                                                                        : GemmTiling::kSwap;
 }
 
 moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                              cudaStream_t st) {
-  if (!get_encoder()) return MOE_ERR_CUDA;
+  if (!tensor_map_encoder()) return MOE_ERR_CUDA;
   static thread_local int attrs_device = -1;
   if (attrs_device != dev.device) {
     if (set_attrs<true, false>() != cudaSuccess || set_attrs<false, false>() != cudaSuccess ||
@@ -500,7 +482,10 @@ moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& d
     attrs_device = dev.device;
   }
   const int T = a.T;
-  const bool pair = use_pair_tiles(c, T);
+  const GemmTiling tiling = gemm_tiling(c, T);
+  if (tiling == GemmTiling::kSwap || tiling == GemmTiling::kSwapPair)
+    return launch_expert_ffn_swap(c, a, dev, tiling == GemmTiling::kSwapPair, st);
+  const bool pair = tiling == GemmTiling::kPair;
   const int b_box = pair ? 128 : 256;   // B rows one CTA loads per stage (down GEMM)
   const uint64_t nslots = uint64_t(T) * c.k;
   const uint64_t rows = nslots + uint64_t(c.S) * T;

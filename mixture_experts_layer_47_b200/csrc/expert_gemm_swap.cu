@@ -1,0 +1,605 @@
+// expert_gemm_swap.cu -- grouped expert GEMMs with the weights as the MMA's M side.
+//
+// Same contractions as expert_gemm.cu (m.xxqk.cn Hy4-preview MoE explainer,
+// section 2.1: each expert is an FFN sub-network; ZAKER Hy4 Preview release
+// news: 256 routed experts plus one shared expert):
+//   gate/up:  H_g = silu(X_g W_gate_g^T) * (X_g W_up_g^T)   -> bf16
+//   down:     Y_g = H_g W_down_g^T                           -> fp32 or bf16
+// but each tcgen05.mma computes D^T = W X^T: the A operand is 128 weight rows
+// (output features) and the B operand is a tile of the group's tokens.  The
+// M side of a tile is then always full, and a group of n tokens is cut into
+// ceil(n/128) token tiles of near-equal width rounded up to 16 (the MMA's N
+// step), so a group pays for at most 15 padding tokens per tile instead of up
+// to 127 padding rows of a 128-row M tile.  At prefill sizes (a few hundred
+// tokens per expert) that recovers most of the tensor work the row-tiled
+// kernel spends on padding.
+//
+// Two tilings share the kernel template:
+//   1-SM (kPair = false): two M=128 MMAs per K step share one token tile of
+//     N <= 128 --
+//       gate/up  A0 = 128 gate rows, A1 = the matching 128 up rows, so the two
+//                fp32 accumulators hold gate and up of the same features in the
+//                same TMEM lanes and the epilogue forms SwiGLU lane-locally;
+//       down     A0, A1 = 256 consecutive W_down rows;
+//     two 256-column accumulators, double buffered.
+//   2-SM (kPair = true): a CTA pair runs tcgen05.mma.cta_group::2 with M = 256
+//     weight rows (128 per CTA) and a token tile of N <= 256 whose rows are
+//     split between the two CTAs' shared memory --
+//       gate/up  a gate MMA and an up MMA per K step, accumulators at TMEM
+//                columns [0, N) and [256, 256+N) (one 512-column buffer);
+//       down     one MMA per K step, two 256-column accumulators.
+//     Each CTA stages its 128 weight rows and half the tokens, so a CTA moves
+//     about half the shared-memory bytes per MMA cycle of the 1-SM tiling --
+//     on sm_100a the TMA writes and the tensor core's operand reads share the
+//     SM's shared-memory bandwidth, which is what limits the 1-SM tilings.
+// Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer (the pair's
+// leader CTA issues for both), warps 2-9 epilogue (two per TMEM lane quarter,
+// taking alternate 32-token chunks).  The accumulator is
+// feature-major (TMEM lane = feature, column = token), so the epilogue
+// transposes each 32x32 block through shared memory and stores whole output
+// rows.  Every wait is bounded; on expiry the kernel records the fault,
+// drains, frees TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include <stdlib.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tensor_map.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BK = 64;                     // K elements per stage
+constexpr int WM = 128;                    // weight rows per CTA per MMA
+constexpr int W_BYTES = WM * BK * 2;       // one A box
+constexpr int B_BOX = 128;                 // token rows per CTA per stage
+constexpr int B_BYTES = B_BOX * BK * 2;    // one B box
+constexpr int EPI_WARPS = 8;               // two per TMEM lane quarter
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
+constexpr int TMEM_COLS = 512;
+constexpr int MAX_GROUPS = 1024 + 8;
+constexpr int MAX_STAGES = 6;
+constexpr int STG_LD = 33;                 // transpose staging row stride (floats)
+
+template <bool kGateUp, bool kPair>
+struct SwapCfg {
+  static constexpr int TN = kPair ? 256 : 128;               // largest token tile (MMA N)
+  static constexpr int NUM_A = (kPair && !kGateUp) ? 1 : 2;  // A boxes per stage
+  static constexpr int STAGE_BYTES = NUM_A * W_BYTES + B_BYTES;
+  static constexpr int STAGES = (kPair && !kGateUp) ? 6 : 4;
+  static constexpr int NUM_ACC = (kPair && kGateUp) ? 1 : 2;
+  static constexpr int ACC_STRIDE = TMEM_COLS / NUM_ACC;
+  static constexpr int SECOND = kPair ? 256 : 128;           // TMEM column of the 2nd MMA's D
+  static constexpr int FEAT = (kGateUp && !kPair) ? 128 : 256;  // output features per tile
+  static constexpr int MMA_M = kPair ? 256 : 128;
+  static constexpr int EPI_THREADS = (kPair ? 2 : 1) * 32 * EPI_WARPS;  // arrivals freeing an acc
+};
+
+struct __align__(64) SwapParams {
+  CUtensorMap tok_routed;  // gate/up: X_perm [T*k][d]; down: H [T*k+S*T][F]   (box 128 rows)
+  CUtensorMap tok_shared;  // gate/up: x [T][d];        down: same as tok_routed
+  CUtensorMap w0;          // gate/up: W_gate [E*F][d]; down: W_down [E*d][F]  (box 128 rows)
+  CUtensorMap w1;          // gate/up: W_up   [E*F][d]; down: unused
+  CUtensorMap s0;          // shared-expert counterparts of w0 / w1
+  CUtensorMap s1;
+  const int32_t* offsets;  // [E+1]
+  const int32_t* sched;    // [E+S+1] prefix sums of ceil(rows / TN) per group
+  void* out;               // gate/up: H bf16; down: Y fp32, or bf16 when out_bf16
+  int* status;
+  int out_bf16;
+  int T, E, S, k;
+  int K;                   // reduction length (d or F)
+  int n_out;               // output features per group (F or d)
+  int w_rows;              // weight rows per expert in the w maps (F or d)
+  int out_rows;            // rows of the output buffer (T*k + S*T)
+};
+
+struct SharedStorage {
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+  int sched[MAX_GROUPS + 1];
+  int offsets[MAX_GROUPS + 1];
+  float stage_t[EPI_WARPS][16 * STG_LD];   // per epilogue warp: one 16-token x 32 block
+};
+
+template <bool kGateUp, bool kPair>
+constexpr size_t swap_smem_bytes() {
+  return 1024 + size_t(SwapCfg<kGateUp, kPair>::STAGES) * SwapCfg<kGateUp, kPair>::STAGE_BYTES +
+         sizeof(SharedStorage);
+}
+static_assert(swap_smem_bytes<true, false>() <= 227 * 1024, "shared memory budget");
+static_assert(swap_smem_bytes<true, true>() <= 227 * 1024, "shared memory budget");
+static_assert(swap_smem_bytes<false, true>() <= 227 * 1024, "shared memory budget");
+
+struct SwapTile {
+  int w_row;     // first weight row of the tile in the w / s maps (of the pair)
+  int f0;        // first output feature of the tile (of the pair)
+  int tok_row;   // first B row (token) in the tok map
+  int out_row;   // output row of the tile's first token
+  int cnt;       // valid tokens in the tile (1..TN)
+  int n;         // MMA N: cnt rounded up to 16
+  bool shared;
+};
+
+// Tiles are numbered group by group; inside a group weight-tile-major with the
+// group's token tiles innermost, so the CTAs that share a weight tile run at
+// the same time and read it through L2.  A group of r tokens has
+// mt = ceil(r / TN) token tiles of ceil(r / mt) tokens rounded up to 16
+// (at most TN, since mt * TN >= r), the last one holding the remainder.
+template <bool kGateUp, bool kPair>
+__device__ __forceinline__ SwapTile decode_swap_tile(int t, int n_wt, int G,
+                                                     const SharedStorage& ss,
+                                                     const SwapParams& p) {
+  using C = SwapCfg<kGateUp, kPair>;
+  const int q = t / n_wt;
+  int lo = 0, hi = G;  // largest g in [0, G) with sched[g] <= q
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (ss.sched[mid] <= q) lo = mid; else hi = mid;
+  }
+  const int mt = ss.sched[lo + 1] - ss.sched[lo];
+  const int local = t - ss.sched[lo] * n_wt;
+  const int w_idx = local / mt;
+  const int j = local - w_idx * mt;
+  const bool shared = lo >= p.E;
+  int rows = shared ? p.T : ss.offsets[lo + 1] - ss.offsets[lo];
+  rows = max(0, min(rows, mt * C::TN));
+  const int per = (((rows + mt - 1) / mt) + 15) & ~15;
+  SwapTile tl;
+  tl.shared = shared;
+  const int first = j * per;
+  tl.cnt = max(0, min(per, rows - first));
+  tl.n = (tl.cnt + 15) & ~15;
+  if (tl.n < 16) tl.n = 16;
+  tl.f0 = w_idx * C::FEAT;
+  const int nslots = p.T * p.k;
+  if (!shared) {
+    tl.w_row = lo * p.w_rows + tl.f0;
+    tl.tok_row = ss.offsets[lo] + first;
+    tl.out_row = tl.tok_row;
+  } else {
+    const int s = lo - p.E;
+    tl.w_row = s * p.w_rows + tl.f0;
+    tl.out_row = nslots + s * p.T + first;
+    tl.tok_row = kGateUp ? first : tl.out_row;
+  }
+  return tl;
+}
+
+// Store a 32-feature x 32-token block held feature-major (this lane = feature,
+// v[i] = token i) as 32 output rows: transpose 16 tokens at a time through the
+// warp's staging block, then each instruction writes whole 16-byte pieces of
+// consecutive rows.
+template <bool kBf16>
+__device__ __forceinline__ void store_block_transposed(float* stg, const float (&v)[32], int lane,
+                                                       void* out, int n_out, int row0, int ntok,
+                                                       int col0, int out_rows) {
+#pragma unroll
+  for (int hb = 0; hb < 2; ++hb) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) stg[i * STG_LD + lane] = v[16 * hb + i];
+    __syncwarp();
+    if (kBf16) {
+      // 4 lanes per token row (64 bytes), 8 rows per instruction
+      const int piece = lane & 3;
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const int tl = (lane >> 2) + 8 * s;
+        const float* src = stg + tl * STG_LD + 8 * piece;
+        const uint4 val = make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                                     pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+        const int tok = 16 * hb + tl;
+        const int row = row0 + tok;
+        if (tok < ntok && row >= 0 && row < out_rows)
+          *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + size_t(row) * n_out +
+                                    col0 + 8 * piece) = val;
+      }
+    } else {
+      // 8 lanes per token row (128 bytes), 4 rows per instruction
+      const int piece = lane & 7;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const int tl = (lane >> 3) + 4 * s;
+        const float* src = stg + tl * STG_LD + 4 * piece;
+        const float4 val = make_float4(src[0], src[1], src[2], src[3]);
+        const int tok = 16 * hb + tl;
+        const int row = row0 + tok;
+        if (tok < ntok && row >= 0 && row < out_rows)
+          *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + size_t(row) * n_out + col0 +
+                                     4 * piece) = val;
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// silu(g) * u.  The exponent is clamped so that 1 + e^-g stays below 2^126,
+// where the fast divide is accurate; below g = -80 silu(g) is -80 e^-80 or
+// smaller, which the clamp reproduces to far under the bf16 output's precision.
+__device__ __forceinline__ float swiglu(float g, float u) {
+  return __fdividef(g, 1.0f + __expf(fminf(-g, 80.0f))) * u;
+}
+
+template <bool kGateUp, bool kPair>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_swap_kernel(const __grid_constant__ SwapParams p) {
+  using C = SwapCfg<kGateUp, kPair>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  SharedStorage& ss = *reinterpret_cast<SharedStorage*>(smem + C::STAGES * C::STAGE_BYTES);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = p.E + p.S;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;   // CTA rank inside the pair
+  const bool leader = rank == 0;
+  const int unit = kPair ? int(blockIdx.x >> 1) : int(blockIdx.x);
+  const int n_units = kPair ? int(gridDim.x >> 1) : int(gridDim.x);
+
+  // Prologue that reads no global data (overlaps the previous kernel under PDL).
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&ss.full[s], 1);
+      mbar_init(&ss.empty[s], 1);
+    }
+    for (int a = 0; a < C::NUM_ACC; ++a) {
+      mbar_init(&ss.tmem_full[a], 1);
+      mbar_init(&ss.tmem_empty[a], C::EPI_THREADS);
+    }
+    mbar_init(&ss.mma_done, 1);
+    ss.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tok_routed);
+    tma_prefetch_desc(&p.tok_shared);
+    tma_prefetch_desc(&p.w0);
+    tma_prefetch_desc(&p.s0);
+    if (kGateUp) {
+      tma_prefetch_desc(&p.w1);
+      tma_prefetch_desc(&p.s1);
+    }
+  }
+  if (warp == 1) {
+    if (kPair) {
+      tmem_alloc_pair(&ss.tmem_base, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&ss.tmem_base, TMEM_COLS);
+      tmem_relinquish();
+    }
+  }
+  pdl_wait();   // the schedule, offsets and token operands come from earlier kernels
+  pdl_launch_dependents();
+  for (int i = threadIdx.x; i <= G; i += NUM_THREADS) ss.sched[i] = p.sched[i];
+  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) ss.offsets[i] = p.offsets[i];
+  tc_fence_before();
+  if (kPair) cluster_sync_all(); else __syncthreads();   // barriers of both CTAs initialised
+  tc_fence_after();
+  const uint32_t tmem_base = ss.tmem_base;
+
+  const int n_wt = (p.n_out + C::FEAT - 1) / C::FEAT;
+  const int total = ss.sched[G] * n_wt;
+  const int kblocks = p.K / BK;
+  volatile int* abort_flag = &ss.abort_flag;
+  bool aborted = false;
+
+  if (warp == 0) {
+    // ---------------- TMA producer (each CTA of a pair loads its own halves) ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      for (int t = unit; t < total && !aborted; t += n_units) {
+        if (*abort_flag) { aborted = true; break; }
+        const SwapTile tl = decode_swap_tile<kGateUp, kPair>(t, n_wt, G, ss, p);
+        const CUtensorMap* mT = tl.shared ? &p.tok_shared : &p.tok_routed;
+        const CUtensorMap* mW0 = tl.shared ? &p.s0 : &p.w0;
+        const CUtensorMap* mW1 = kGateUp ? (tl.shared ? &p.s1 : &p.w1) : mW0;
+        // this CTA's weight rows and token rows
+        const int w0_row = tl.w_row + (kPair ? int(rank) * WM : 0);
+        const int w1_row = kGateUp ? w0_row : w0_row + WM;   // 1-SM down: second 128 rows
+        const int t_row = tl.tok_row + (kPair ? int(rank) * (tl.n >> 1) : 0);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&ss.empty[stage], phase ^ 1)) {
+            report_error(p.status, kDevTimeout, kSiteProducer);
+            *abort_flag = 1;
+            aborted = true;
+            break;
+          }
+          uint8_t* dst = smem + stage * C::STAGE_BYTES;
+          const int kc = kb * BK;
+          if (kPair) {
+            // The leader's full barrier counts the bytes of both CTAs' loads.
+            const uint32_t bar = mapa_shared(smem_u32(&ss.full[stage]), 0);
+            if (leader) mbar_arrive_expect_tx(&ss.full[stage], 2 * C::STAGE_BYTES);
+            tma_load_2d_pair(dst, mW0, bar, kc, w0_row);
+            if (C::NUM_A == 2) tma_load_2d_pair(dst + W_BYTES, mW1, bar, kc, w1_row);
+            tma_load_2d_pair(dst + C::NUM_A * W_BYTES, mT, bar, kc, t_row);
+          } else {
+            mbar_arrive_expect_tx(&ss.full[stage], C::STAGE_BYTES);
+            tma_load_2d_nohint(dst, mW0, &ss.full[stage], kc, w0_row);
+            tma_load_2d_nohint(dst + W_BYTES, mW1, &ss.full[stage], kc, w1_row);
+            tma_load_2d_nohint(dst + 2 * W_BYTES, mT, &ss.full[stage], kc, t_row);
+          }
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Drain: loads counted on this CTA's own full barriers must land before it
+      // exits (in the normal path the MMA consumed them all).
+      if (!kPair || leader) {
+        for (int s = 0; s < C::STAGES; ++s)
+          if (issued_mask & (1u << s))
+            if (!mbar_wait(&ss.full[s], (issued_parity >> s) & 1u, kDrainTimeoutNs))
+              report_error(p.status, kDevTimeout, kSiteDrain);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (the pair's leader only) ----------------
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int t = unit; t < total && !aborted; t += n_units) {
+        if (*abort_flag) { aborted = true; break; }
+        const SwapTile tl = decode_swap_tile<kGateUp, kPair>(t, n_wt, G, ss, p);
+        const uint32_t idesc = umma_idesc_bf16_f32(C::MMA_M, tl.n);
+        if (!mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1)) {
+          report_error(p.status, kDevTimeout, kSiteMma);
+          *abort_flag = 1;
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + uint32_t(acc * C::ACC_STRIDE);
+        const uint32_t d1 = d0 + uint32_t(C::SECOND);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&ss.full[stage], phase)) {
+            report_error(p.status, kDevTimeout, kSiteMma);
+            *abort_flag = 1;
+            aborted = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t base = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint64_t a0 = umma_desc_sw128_kmajor(base);
+          const uint64_t a1 = umma_desc_sw128_kmajor(base + W_BYTES);
+          const uint64_t b = umma_desc_sw128_kmajor(base + C::NUM_A * W_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            if (kPair) {
+              umma_bf16_pair(d0, a0 + uint64_t(2 * kk), b + uint64_t(2 * kk), idesc, accum);
+              if (C::NUM_A == 2)
+                umma_bf16_pair(d1, a1 + uint64_t(2 * kk), b + uint64_t(2 * kk), idesc, accum);
+            } else {
+              umma_bf16(d0, a0 + uint64_t(2 * kk), b + uint64_t(2 * kk), idesc, accum);
+              umma_bf16(d1, a1 + uint64_t(2 * kk), b + uint64_t(2 * kk), idesc, accum);
+            }
+          }
+          if (kPair) umma_commit_pair(&ss.empty[stage], 0x3); else umma_commit(&ss.empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (aborted) break;
+        if (kPair) umma_commit_pair(&ss.tmem_full[acc], 0x3); else umma_commit(&ss.tmem_full[acc]);
+        if (++acc == C::NUM_ACC) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      // Drain: wait until every MMA issued here has completed.
+      if (kPair) umma_commit_pair(&ss.mma_done, 0x1); else umma_commit(&ss.mma_done);
+      if (!mbar_wait(&ss.mma_done, 0, kDrainTimeoutNs))
+        report_error(p.status, kDevTimeout, kSiteDrain);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..9; TMEM lane = output feature) ----------------
+    const int quarter = warp & 3;               // TMEM lanes [32*quarter, 32*quarter+32)
+    const int sub = (warp - 2) >> 2;            // which of the quarter's two warps
+    const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+    float* stg = ss.stage_t[warp - 2];
+    const int feat_cta = kPair ? int(rank) * WM : 0;   // this CTA's first feature in a tile
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = unit; t < total; t += n_units) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) { aborted = true; break; }  // warp-uniform
+      const SwapTile tl = decode_swap_tile<kGateUp, kPair>(t, n_wt, G, ss, p);
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&ss.tmem_full[acc], acc_phase));
+      if (!ok) {
+        if (lane == 0) report_error(p.status, kDevTimeout, kSiteEpilogue);
+        *abort_flag = 1;
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + lane_addr + uint32_t(acc * C::ACC_STRIDE);
+      // this warp's 32-token chunks: c = 32 * (2 i + sub)
+      if (kGateUp) {
+        const int col0 = tl.f0 + feat_cta + quarter * 32;   // this warp's 32 features
+        const bool cols_ok = col0 < p.n_out;                // n_out is a multiple of 64
+        int c = 32 * sub;
+        uint32_t g[32], u[32];
+        if (c < tl.n) {
+          tmem_ld_32cols(tbase + uint32_t(c), g);
+          tmem_ld_32cols(tbase + uint32_t(C::SECOND + c), u);
+        }
+#pragma unroll 1
+        for (; c < tl.n; c += 64) {
+          tmem_ld_wait();
+          float h[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) h[i] = swiglu(__uint_as_float(g[i]), __uint_as_float(u[i]));
+          if (c + 64 < tl.n) {   // next chunk's loads overlap this chunk's stores
+            tmem_ld_32cols(tbase + uint32_t(c + 64), g);
+            tmem_ld_32cols(tbase + uint32_t(C::SECOND + c + 64), u);
+          }
+          if (cols_ok)
+            store_block_transposed<true>(stg, h, lane, p.out, p.n_out, tl.out_row + c,
+                                         tl.cnt - c, col0, p.out_rows);
+        }
+      } else {
+        constexpr int kHalves = kPair ? 1 : 2;
+#pragma unroll 1
+        for (int half = 0; half < kHalves; ++half) {
+          const int col0 = tl.f0 + feat_cta + half * WM + quarter * 32;
+          const bool cols_ok = col0 < p.n_out;
+          const uint32_t hbase = tbase + uint32_t(half * C::SECOND);
+          int c = 32 * sub;
+          uint32_t r[32];
+          if (c < tl.n) tmem_ld_32cols(hbase + uint32_t(c), r);
+#pragma unroll 1
+          for (; c < tl.n; c += 64) {
+            tmem_ld_wait();
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+            if (c + 64 < tl.n) tmem_ld_32cols(hbase + uint32_t(c + 64), r);
+            if (cols_ok) {
+              if (p.out_bf16)
+                store_block_transposed<true>(stg, v, lane, p.out, p.n_out, tl.out_row + c,
+                                             tl.cnt - c, col0, p.out_rows);
+              else
+                store_block_transposed<false>(stg, v, lane, p.out, p.n_out, tl.out_row + c,
+                                              tl.cnt - c, col0, p.out_rows);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      if (kPair)
+        mbar_arrive_cluster(mapa_shared(smem_u32(&ss.tmem_empty[acc]), 0));
+      else
+        mbar_arrive(&ss.tmem_empty[acc]);
+      if (++acc == C::NUM_ACC) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  if (kPair && aborted) {
+    // A CTA of a pair cannot observe its own loads' completion (they are
+    // counted on the leader's barrier): give copies in flight time to land.
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 100000ull) {
+    }
+  }
+  tc_fence_before();
+  if (kPair) cluster_sync_all(); else __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    if (kPair) tmem_dealloc_pair(tmem_base, TMEM_COLS); else tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+template <bool kGateUp, bool kPair>
+cudaError_t launch_swap(const SwapParams& sp, int num_sms, cudaStream_t st) {
+  static thread_local int attrs_device = -1;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (attrs_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<kGateUp, kPair>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(swap_smem_bytes<kGateUp, kPair>()));
+    if (e != cudaSuccess) return e;
+    attrs_device = dev;
+  }
+  const unsigned grid = kPair ? unsigned(num_sms & ~1) : unsigned(num_sms);
+  return launch_pdl(grouped_gemm_swap_kernel<kGateUp, kPair>, dim3(grid), dim3(NUM_THREADS),
+                    swap_smem_bytes<kGateUp, kPair>(), st, kPair ? 2 : 1, sp);
+}
+
+}  // namespace
+
+moe_status launch_expert_ffn_swap(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
+                                  bool pair, cudaStream_t st) {
+  const int T = a.T;
+  const uint64_t nslots = uint64_t(T) * c.k;
+  const uint64_t rows = nslots + uint64_t(c.S) * T;
+  // schedules of 128-token tiles at sched[0..G], of 256-token tiles at sched[G+1..2G+1]
+  const int32_t* sched = a.sched + (pair ? (c.E + c.S + 1) : 0);
+
+  // ---- gate/up + SwiGLU ----
+  SwapParams gp;
+  memset(&gp, 0, sizeof gp);
+  bool ok = encode_bf16_2d(&gp.tok_routed, a.x_perm, nslots, c.d, B_BOX) &&
+            encode_bf16_2d(&gp.tok_shared, a.x, uint64_t(T), c.d, B_BOX) &&
+            encode_bf16_2d(&gp.w0, a.Wg, uint64_t(c.E) * c.F, c.d, WM) &&
+            encode_bf16_2d(&gp.w1, a.Wu, uint64_t(c.E) * c.F, c.d, WM);
+  if (c.S > 0)
+    ok = ok && encode_bf16_2d(&gp.s0, a.Sg, uint64_t(c.S) * c.F, c.d, WM) &&
+         encode_bf16_2d(&gp.s1, a.Su, uint64_t(c.S) * c.F, c.d, WM);
+  else {
+    gp.s0 = gp.w0;
+    gp.s1 = gp.w1;
+  }
+  if (!ok) return MOE_ERR_CUDA;
+  gp.offsets = a.offsets;
+  gp.sched = sched;
+  gp.out = a.h_act;
+  gp.status = a.status;
+  gp.T = T;
+  gp.E = c.E;
+  gp.S = c.S;
+  gp.k = c.k;
+  gp.K = c.d;
+  gp.n_out = c.F;
+  gp.w_rows = c.F;
+  gp.out_rows = int(rows);
+  cudaError_t err = pair ? launch_swap<true, true>(gp, dev.num_sms, st)
+                         : launch_swap<true, false>(gp, dev.num_sms, st);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  if (a.after_gate_up && cudaEventRecord(a.after_gate_up, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  // ---- down projection ----
+  SwapParams dp;
+  memset(&dp, 0, sizeof dp);
+  ok = encode_bf16_2d(&dp.tok_routed, a.h_act, rows, c.F, B_BOX) &&
+       encode_bf16_2d(&dp.w0, a.Wd, uint64_t(c.E) * c.d, c.F, WM);
+  if (c.S > 0)
+    ok = ok && encode_bf16_2d(&dp.s0, a.Sd, uint64_t(c.S) * c.d, c.F, WM);
+  else
+    dp.s0 = dp.w0;
+  if (!ok) return MOE_ERR_CUDA;
+  dp.tok_shared = dp.tok_routed;
+  dp.w1 = dp.w0;
+  dp.s1 = dp.s0;
+  dp.offsets = a.offsets;
+  dp.sched = sched;
+  dp.out = a.Y;
+  dp.out_bf16 = a.y_bf16 ? 1 : 0;
+  dp.status = a.status;
+  dp.T = T;
+  dp.E = c.E;
+  dp.S = c.S;
+  dp.k = c.k;
+  dp.K = c.F;
+  dp.n_out = c.d;
+  dp.w_rows = c.d;
+  dp.out_rows = int(rows);
+  err = pair ? launch_swap<false, true>(dp, dev.num_sms, st)
+             : launch_swap<false, false>(dp, dev.num_sms, st);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace moe

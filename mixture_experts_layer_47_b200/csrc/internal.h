@@ -84,7 +84,10 @@ int router_tc_ksplit(const Ctx& c, int T, int num_sms);
 cudaError_t launch_router_tc(const Ctx& c, int ksplit, const uint16_t* x, const float* Wr, int T,
                              uint16_t* wparts, float* part, int* status, int num_sms,
                              cudaStream_t st);
-bool use_pair_tiles(const Ctx& c, int T);
+enum class GemmTiling { kSingle, kPair, kSwap, kSwapPair };
+// Average routed rows per expert from which the 2-SM weight-major kernel is used.
+constexpr int kSwapPairMinRowsPerExpert = 96;
+GemmTiling gemm_tiling(const Ctx& c, int T);
 
 cudaError_t launch_dispatch(const Ctx& c, const int32_t* topk_idx, int T, int nblk,
                             int32_t* blk_hist, int32_t* counts, int32_t* offsets, int32_t* perm,
@@ -109,7 +112,7 @@ struct FfnArgs {
   const uint16_t* x;        // [T][d]
   const uint16_t* x_perm;   // [T*k][d]
   const int32_t* offsets;   // [E+1]
-  const int32_t* sched;     // [E+S+1]
+  const int32_t* sched;     // [2(E+S+1)]: 128-row then 256-row tile prefix sums
   const uint16_t *Wg, *Wu, *Wd, *Sg, *Su, *Sd;
   uint16_t* h_act;          // [T*k+S*T][F]
   void* Y;                  // [T*k+S*T][d], fp32 or (y_bf16) bf16
@@ -120,5 +123,7 @@ struct FfnArgs {
 };
 moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                              cudaStream_t st);
+moe_status launch_expert_ffn_swap(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
+                                  bool pair, cudaStream_t st);
 
 }  // namespace moe

@@ -1,8 +1,8 @@
 """GPU parity of every step of the CUDA path against the fp64 oracle, through the C ABI.
 
-Sizes span several tiles and ragged tails (rows not a multiple of the 128-row
-M tile, d_ff not a multiple of the 128-feature gate/up tile, d not a multiple
-of the 256-feature down tile, dispatch runs over more than one 4096-slot
+Sizes span several tiles and ragged tails (groups not a multiple of the GEMMs'
+128- or 256-row tiles or 16-token N step, d_ff not a multiple of the 128- or
+256-feature gate/up tile, d not a multiple of the 256-feature down tile, dispatch runs over more than one 4096-slot
 block) plus the degenerate cases (one token, one expert, k = E, no shared
 expert, every token on one expert, an empty expert).
 """
@@ -26,7 +26,7 @@ SHAPES = [  # T, d, E, k, F, S, bias_scale
     (130, 320, 5, 3, 384, 2, 0.0),
     (513, 512, 64, 8, 256, 1, 0.2),
     (40, 256, 8, 8, 128, 1, 0.0),      # k == E
-    # T*k >= 128*E: the 2-SM (cta_group::2, 256-row tile) GEMM path
+    # T*k >= 96*E: the default 2-SM (cta_group::2) weight-major GEMM path
     (600, 256, 4, 2, 128, 1, 0.0),     # ~300 rows per expert: two pair tiles, ragged tail
     (200, 320, 2, 2, 192, 2, 0.0),     # k == E, every group 200 rows; two shared experts
     (1000, 128, 8, 2, 64, 1, 0.3),     # d_ff = 64: half of each gate/up tile masked
@@ -87,12 +87,17 @@ def test_router_logit_accuracy(shape, path, monkeypatch):
                  w.cpu().numpy(), h.k)
 
 
-@pytest.mark.parametrize("tiles", ["single", "pair"])
+TILINGS = ["single", "pair", "swap", "swap_pair"]
+
+
+@pytest.mark.parametrize("tiles", TILINGS)
 @pytest.mark.parametrize("shape", [(64, 256, 16, 2, 128, 1, 0.0), (600, 256, 4, 2, 128, 1, 0.0),
                                    (130, 320, 5, 3, 384, 2, 0.0)],
                          ids=lambda s: "T{}_d{}_E{}_k{}_F{}_S{}".format(*s[:6]))
-def test_forward_both_gemm_tilings(shape, tiles, monkeypatch):
-    """The 1-SM (128-row) and 2-SM (256-row, cta_group::2) GEMM paths on the same inputs."""
+def test_forward_all_gemm_tilings(shape, tiles, monkeypatch):
+    """The row-tiled 1-SM (128-row) and 2-SM (256-row, cta_group::2) GEMMs and the
+    weight-major GEMMs (weights on the MMA's M side; 1-SM token tiles of N <= 128, 2-SM
+    token tiles of N <= 256) on the same inputs."""
     monkeypatch.setenv("MOE_GEMM_TILES", tiles)
     T, d, E, k, F, S, bs = shape
     inp = make_small(T, d, E, k, F, S, seed=500 + T, bias_scale=bs)
@@ -139,9 +144,12 @@ def test_dispatch_flags_out_of_range_index():
     np.testing.assert_array_equal(counts, np.bincount(valid, minlength=E))
 
 
+@pytest.mark.parametrize("tiles", TILINGS)
 @pytest.mark.parametrize("shape", SHAPES, ids=_ids(SHAPES))
-def test_expert_ffn_stage(shape):
-    """Y rows (and the bf16 SwiGLU activations) against the oracle, given the oracle's dispatch."""
+def test_expert_ffn_stage(shape, tiles, monkeypatch):
+    """Y rows (fp32) and the bf16 SwiGLU activations against the oracle, given the oracle's
+    dispatch, for each GEMM tiling."""
+    monkeypatch.setenv("MOE_GEMM_TILES", tiles)
     T, d, E, k, F, S, bs = shape
     inp = make_small(T, d, E, k, F, S, seed=200 + T, bias_scale=bs)
     dev = to_device(inp, "cuda")
@@ -213,9 +221,12 @@ def test_forward_tiny_workload():
     assert err < Y_REL_TOL, err
 
 
-def test_every_token_on_one_expert_and_empty_experts():
-    """Dominant biases send all 300 tokens to experts 3 and 7 (3 M tiles each); the other
-    14 experts stay empty."""
+@pytest.mark.parametrize("tiles", ["single", "swap", "swap_pair"])
+def test_every_token_on_one_expert_and_empty_experts(tiles, monkeypatch):
+    """Dominant biases send all 300 tokens to experts 3 and 7 (3 M tiles of 128 rows each,
+    3 token tiles of 112, 112 and 76 tokens, or 2 pair token tiles of 160 and 140); the
+    other 14 experts stay empty."""
+    monkeypatch.setenv("MOE_GEMM_TILES", tiles)
     T, d, E, k, F, S = 300, 128, 16, 2, 128, 1
     inp = make_small(T, d, E, k, F, S, seed=9)
     bias = torch.zeros(E)
@@ -231,9 +242,11 @@ def test_every_token_on_one_expert_and_empty_experts():
     assert rel_err(y.float().numpy(), ref["y"]) < Y_REL_TOL
 
 
-def test_pair_tiles_hot_experts_and_empty_experts():
-    """2-SM path: two experts take all 700 tokens (3 pair tiles of 256, 256, 188 rows) and
-    the other two stay empty."""
+@pytest.mark.parametrize("tiles", ["pair", "swap_pair"])
+def test_pair_tiles_hot_experts_and_empty_experts(tiles, monkeypatch):
+    """2-SM paths: two experts take all 700 tokens (3 row tiles of 256, 256, 188 rows, or 3
+    token tiles of 240, 240, 220) and the other two stay empty."""
+    monkeypatch.setenv("MOE_GEMM_TILES", tiles)
     T, d, E, k, F, S = 700, 256, 4, 2, 128, 1
     inp = make_small(T, d, E, k, F, S, seed=19)
     bias = torch.tensor([0.0, 50.0, 0.0, 40.0])
