@@ -433,7 +433,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + lane_addr + uint32_t(acc * C::ACC_STRIDE);
       // this warp's 32-token chunks: c = 32 * (2 i + sub)
-      if (kGateUp) {
+      bool released = false;
+      if (kGateUp && kPair) {
+        // The pair's gate/up accumulator fills all 512 columns, so the next tile's
+        // MMAs wait for it: read the whole tile into registers first (SwiGLU packed
+        // to bf16 pairs, <= 4 chunks per warp), hand TMEM back, then store.
+        const int col0 = tl.f0 + feat_cta + quarter * 32;
+        const bool cols_ok = col0 < p.n_out;
+        uint32_t hp[4][16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = 32 * (2 * j + sub);
+          if (c < tl.n) {
+            uint32_t g[32], u[32];
+            tmem_ld_32cols(tbase + uint32_t(c), g);
+            tmem_ld_32cols(tbase + uint32_t(C::SECOND + c), u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              hp[j][i] = pack_bf16x2(swiglu(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                     swiglu(__uint_as_float(g[2 * i + 1]),
+                                            __uint_as_float(u[2 * i + 1])));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive_cluster(mapa_shared(smem_u32(&ss.tmem_empty[acc]), 0));
+        released = true;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = 32 * (2 * j + sub);
+          if (c < tl.n && cols_ok) {
+            float h[32];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              h[2 * i] = bf16_bits_to_float(hp[j][i] & 0xFFFFu);
+              h[2 * i + 1] = bf16_bits_to_float(hp[j][i] >> 16);
+            }
+            store_block_transposed<true>(stg, h, lane, p.out, p.n_out, tl.out_row + c,
+                                         tl.cnt - c, col0, p.out_rows);
+          }
+        }
+      } else if (kGateUp) {
         const int col0 = tl.f0 + feat_cta + quarter * 32;   // this warp's 32 features
         const bool cols_ok = col0 < p.n_out;                // n_out is a multiple of 64
         int c = 32 * sub;
@@ -484,11 +524,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      tc_fence_before();
-      if (kPair)
-        mbar_arrive_cluster(mapa_shared(smem_u32(&ss.tmem_empty[acc]), 0));
-      else
-        mbar_arrive(&ss.tmem_empty[acc]);
+      if (!released) {
+        tc_fence_before();
+        if (kPair)
+          mbar_arrive_cluster(mapa_shared(smem_u32(&ss.tmem_empty[acc]), 0));
+        else
+          mbar_arrive(&ss.tmem_empty[acc]);
+      }
       if (++acc == C::NUM_ACC) {
         acc = 0;
         acc_phase ^= 1;
