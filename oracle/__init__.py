@@ -11,6 +11,14 @@ follows the pages' statement of the layer (m.xxqk.cn Hy4-preview MoE explainer
 section 2.1 "FFN split" and 2.2 "router mechanism"; ZAKER Hy4 Preview release
 news, MoE paragraph) with the readings written at the top of ``moe_oracle.c``.
 
+FP8 expert weights (the format the Hy4 pages' FP8 checkpoint implies but does
+not specify; the stated choice is described in ``workloads``): ``e4m3_value``
+decodes one code from the OCP FP8 E4M3 definition, ``dequant_fp8`` applies the
+per-32-element power-of-two scales, and ``fp8_as_bf16`` hands the decoded
+weights to the bf16 layer above as exact bf16 bit patterns (every decoded
+weight has at most 4 significant bits, so the conversion is exact; it is
+checked, not assumed).
+
 Pinning: every function here is checked in ``tests/test_oracle.py`` against
 values fixed independently of it (hand-derived closed forms in
 ``tests/golden/``, numpy/torch float64 library routines on special cases,
@@ -275,3 +283,83 @@ def renormalised_gates(logits: np.ndarray, idx: np.ndarray) -> np.ndarray:
         sel = p[idx[t]]
         w[t] = sel / sel.sum()
     return w
+
+
+# ----------------------------------------------------------------------------
+# FP8 (E4M3) expert weights with power-of-two block scales.
+# ----------------------------------------------------------------------------
+FP8_BLOCK = 32
+
+
+def e4m3_value(code: int) -> float:
+    """The number an FP8 E4M3 code stands for (OCP 8-bit floating point specification,
+    E4M3 row): bit 7 sign, bits 6-3 exponent with bias 7, bits 2-0 mantissa; exponent
+    field 0 is subnormal (m/8 * 2^-6); all-ones exponent and mantissa is NaN; there is no
+    infinity."""
+    code = int(code) & 0xFF
+    sign = -1.0 if code & 0x80 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 0xF and m == 0x7:
+        return float("nan")
+    if e == 0:
+        return sign * (m / 8.0) * 2.0 ** -6
+    return sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+E4M3_TABLE = np.array([e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
+def dequant_fp8(codes, scales) -> np.ndarray:
+    """fp64 weights from codes [n, rows, K] (uint8) and scales [n, K/32, rows] (uint8):
+    w[e, r, j] = e4m3(codes[e, r, j]) * 2^(scales[e, j // 32, r] - 127)."""
+    c = _np(codes, np.uint8)
+    sc = _np(scales, np.uint8)
+    n, rows, K = c.shape
+    assert K % FP8_BLOCK == 0 and sc.shape == (n, K // FP8_BLOCK, rows), (c.shape, sc.shape)
+    mult = np.exp2(sc.astype(np.float64) - 127.0)           # [n, K/32, rows]
+    mult = np.repeat(np.transpose(mult, (0, 2, 1)), FP8_BLOCK, axis=2)   # [n, rows, K]
+    return E4M3_TABLE[c] * mult
+
+
+def fp8_as_bf16(codes, scales) -> np.ndarray:
+    """The dequantised weights as bf16 bit patterns (uint16), for the bf16 layer routines.
+    Raises if any weight is not exactly a bf16 value."""
+    w = dequant_fp8(codes, scales)
+    if not np.all(np.isfinite(w)):
+        raise ValueError("NaN code in FP8 weights")
+    f32 = w.astype(np.float32)
+    if not np.array_equal(f32.astype(np.float64), w):
+        raise ValueError("FP8 weight not representable in fp32")
+    bits = f32.view(np.uint32)
+    if np.any(bits & 0xFFFF):
+        raise ValueError("FP8 weight not representable in bf16")
+    return (bits >> 16).astype(np.uint16)
+
+
+def fp8_inputs(inp, routed, shared, experts: Optional[Sequence[int]] = None):
+    """``inp`` with its expert weights replaced by the decoded FP8 sets (``workloads.Fp8Set``).
+
+    With ``experts`` given, only those routed experts are decoded and returned as a
+    mapping for ``forward(..., weights=...)``; otherwise a full copy of ``inp`` is
+    returned."""
+    def dec(c, s):
+        return fp8_as_bf16(c, s)
+    sh = {k: dec(getattr(shared, k), getattr(shared, k + "_scale"))
+          for k in ("gate", "up", "down")}
+    if experts is not None:
+        m = {"W_gate": {}, "W_up": {}, "W_down": {}}
+        for e in experts:
+            for k in ("gate", "up", "down"):
+                c = _np(getattr(routed, k)[e:e + 1], np.uint8)
+                s = _np(getattr(routed, k + "_scale")[e:e + 1], np.uint8)
+                m["W_" + k][int(e)] = dec(c, s)[0]
+        m.update(Ws_gate=sh["gate"], Ws_up=sh["up"], Ws_down=sh["down"])
+        return m
+    import copy
+    out = copy.copy(inp)
+    out.W_gate = dec(routed.gate, routed.gate_scale)
+    out.W_up = dec(routed.up, routed.up_scale)
+    out.W_down = dec(routed.down, routed.down_scale)
+    out.Ws_gate, out.Ws_up, out.Ws_down = sh["gate"], sh["up"], sh["down"]
+    return out

@@ -262,3 +262,88 @@ def test_bad_arguments_rejected():
         oracle.route(np.zeros((2, 3)), 4)          # k > E
     with pytest.raises(ValueError):
         oracle.dispatch(np.array([[0, 5]], np.int32), 4)   # expert id out of range
+
+
+# ----------------------------------------------------------------------------
+# FP8 expert weights: decode and block scales.
+# ----------------------------------------------------------------------------
+def test_e4m3_decode_matches_torch_float8_for_every_code():
+    """All 256 codes against torch's float8_e4m3fn -> float64 conversion (a library
+    implementation of the same OCP format, independent of the oracle's decoder)."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.E4M3_TABLE
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got)) and nan.sum() == 2   # 0x7F and 0xFF
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+    # signed zeros are kept
+    assert math.copysign(1.0, got[0x80]) == -1.0 and got[0x00] == 0.0
+
+
+@pytest.mark.parametrize("code,value", [
+    (0x00, 0.0), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9), (0x08, 2.0 ** -6),
+    (0x38, 1.0), (0x39, 1.125), (0x3F, 1.875), (0x40, 2.0), (0x7E, 448.0),
+    (0xB8, -1.0), (0xFE, -448.0), (0x77, 240.0), (0x30, 0.5)])
+def test_e4m3_values_from_the_format_definition(code, value):
+    """Hand-derived values: (-1)^s * (1 + m/8) * 2^(e-7), subnormals m/8 * 2^-6."""
+    assert oracle.e4m3_value(code) == value
+
+
+def test_dequant_block_scales_and_layout():
+    """Two experts, 3 rows, K = 64 (two 32-element blocks): scale byte of (expert e, block
+    b, row r) = 120 + 4e + 2b + r, every code 0x38 (1.0) except row 1 of expert 0, whose
+    codes are 0x40 (2.0); so w[e, r, j] = c * 2^(-7 + 4e + 2(j // 32) + r)."""
+    n, rows, K = 2, 3, 64
+    codes = np.full((n, rows, K), 0x38, np.uint8)
+    codes[0, 1, :] = 0x40
+    scales = np.zeros((n, K // 32, rows), np.uint8)
+    for e in range(n):
+        for b in range(K // 32):
+            for r in range(rows):
+                scales[e, b, r] = 120 + 4 * e + 2 * b + r
+    w = oracle.dequant_fp8(codes, scales)
+    for e in range(n):
+        for r in range(rows):
+            for j in (0, 31, 32, 63):
+                c = 2.0 if (e, r) == (0, 1) else 1.0
+                assert w[e, r, j] == c * 2.0 ** (-7 + 4 * e + 2 * (j // 32) + r), (e, r, j)
+
+
+def test_fp8_checkpoint_round_trip_and_exact_bf16():
+    """The workload's FP8 checkpoint decodes to within half an e4m3 step of the bf16 draws
+    (relative 2^-4 of each value for normal codes, 2^-10 of the block maximum below the
+    normal range), and the decoded weights are exact bf16 values."""
+    from workloads import make_fp8
+    inp = make_small(4, 128, 3, 2, 64, 1, seed=11)
+    routed, shared = make_fp8(inp)
+    for W, c, s in ((inp.W_gate, routed.gate, routed.gate_scale),
+                    (inp.W_down, routed.down, routed.down_scale),
+                    (inp.Ws_up, shared.up, shared.up_scale)):
+        w = W.to(torch.float64).numpy()
+        got = oracle.dequant_fp8(c, s)
+        blocks = np.abs(w).reshape(w.shape[0], w.shape[1], -1, 32).max(-1)
+        floor = np.repeat(blocks, 32, axis=2) * 2.0 ** -10
+        assert np.all(np.abs(got - w) <= np.maximum(np.abs(w) * 2.0 ** -4, floor))
+        bits = oracle.fp8_as_bf16(c, s)
+        back = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64)
+        np.testing.assert_array_equal(back.numpy(), got)
+
+
+def test_fp8_layer_is_the_bf16_layer_on_decoded_weights():
+    """The oracle's FP8 layer equals its bf16 layer run on weights that are already exactly
+    the decoded values (both from the same seeded draws, via independent routes: the
+    decoded bits versus torch's float8 -> bf16 cast of the same codes times the scales)."""
+    from workloads import make_fp8
+    inp = make_small(12, 128, 4, 2, 64, 1, seed=12)
+    routed, shared = make_fp8(inp)
+    via_oracle = oracle.forward(oracle.fp8_inputs(inp, routed, shared))["y"]
+
+    def torch_dec(c, s):
+        v = c.view(torch.float8_e4m3fn).to(torch.float32)
+        m = torch.exp2(s.to(torch.float32) - 127.0).transpose(1, 2)
+        return (v * m.repeat_interleave(32, dim=2)).to(torch.bfloat16)
+    alt = Inputs(inp.wl, inp.x, inp.W_router, inp.bias,
+                 torch_dec(routed.gate, routed.gate_scale), torch_dec(routed.up, routed.up_scale),
+                 torch_dec(routed.down, routed.down_scale), torch_dec(shared.gate, shared.gate_scale),
+                 torch_dec(shared.up, shared.up_scale), torch_dec(shared.down, shared.down_scale))
+    np.testing.assert_array_equal(via_oracle, oracle.forward(alt)["y"])

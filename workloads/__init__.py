@@ -48,6 +48,7 @@ class Workload:
     zipf_s: Optional[float] = None  # per-expert bias making expert popularity ~ Zipf(s)
     seed: int = 0
     description: str = ""
+    weights: str = "bf16"           # "bf16", or "fp8": the same draws stored as e4m3 + block scales
 
     @property
     def slots(self) -> int:
@@ -81,6 +82,15 @@ WORKLOADS = {
         zipf_s=1.2, seed=0,
         description="Skewed-load prefill: T=8192, router logits plus a per-expert bias "
                     "calibrated so expert popularity follows Zipf s=1.2"),
+    "decode_fp8": Workload(
+        "decode_fp8", T=16, d=6144, E=256, k=8, F=2048, S=1, router="normal", seed=0,
+        weights="fp8",
+        description="the decode workload with its expert weights stored as FP8 (e4m3 codes, one "
+                    "power-of-two scale per 32 K elements of a row)"),
+    "batched_decode_fp8": Workload(
+        "batched_decode_fp8", T=256, d=6144, E=256, k=8, F=2048, S=1, router="uniform", seed=0,
+        weights="fp8",
+        description="the batched decode workload with FP8 expert weights"),
 }
 
 # Reduced cases of the same kernels for profiler captures that must stay a few GB on the
@@ -250,3 +260,68 @@ def to_device(inp: Inputs, device) -> Inputs:
     return Inputs(inp.wl, mv(inp.x), mv(inp.W_router), mv(inp.bias), mv(inp.W_gate),
                   mv(inp.W_up), mv(inp.W_down), mv(inp.Ws_gate), mv(inp.Ws_up),
                   mv(inp.Ws_down), dict(inp.extra))
+
+
+# ----------------------------------------------------------------------------
+# FP8 expert weights (an input format, not part of the layer's arithmetic).
+#
+# The Hy4 pages mention an official FP8 checkpoint but print no scaling scheme;
+# this layer's stated choice is the OCP microscaling layout: every weight is an
+# FP8 E4M3 code (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no
+# infinities, S.1111.111 = NaN, largest finite 448), and each run of 32
+# consecutive K elements of a weight row shares one power-of-two scale stored
+# as a biased exponent byte (value 2^(byte - 127)).  Scales are stored
+# K-block-major, scale[n][K/32][rows], so the scales of 128 consecutive rows
+# for one K block are contiguous.  The FP8 checkpoint of a workload is made
+# from the same seeded bf16 draws: per block the smallest power of two 2^e with
+# max|w| / 2^e <= 448, codes = e4m3(w / 2^e) rounded to nearest even.
+# ----------------------------------------------------------------------------
+FP8_BLOCK = 32
+FP8_E4M3_MAX = 448.0
+
+
+@dataclass
+class Fp8Set:
+    """FP8 weights of one set of experts (routed or shared)."""
+    gate: torch.Tensor         # [n, F, d] uint8 e4m3 codes
+    gate_scale: torch.Tensor   # [n, d/32, F] uint8 biased exponents
+    up: torch.Tensor           # [n, F, d]
+    up_scale: torch.Tensor     # [n, d/32, F]
+    down: torch.Tensor         # [n, d, F]
+    down_scale: torch.Tensor   # [n, F/32, d]
+
+    def to(self, device) -> "Fp8Set":
+        return Fp8Set(*(t.to(device) for t in (self.gate, self.gate_scale, self.up,
+                                               self.up_scale, self.down, self.down_scale)))
+
+
+def quantize_fp8(W: torch.Tensor, chunk: int = 8) -> tuple:
+    """[n, rows, K] weights -> (codes [n, rows, K] uint8, scales [n, K/32, rows] uint8).
+
+    Works on W's device, ``chunk`` leading slices at a time."""
+    n, rows, K = W.shape
+    if K % FP8_BLOCK:
+        raise ValueError("K must be a multiple of 32")
+    codes = torch.empty((n, rows, K), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((n, K // FP8_BLOCK, rows), dtype=torch.uint8, device=W.device)
+    for i in range(0, n, chunk):
+        j = min(n, i + chunk)
+        w = W[i:j].to(torch.float32).reshape(j - i, rows, K // FP8_BLOCK, FP8_BLOCK)
+        amax = w.abs().amax(dim=-1)
+        e = torch.ceil(torch.log2(amax / FP8_E4M3_MAX))
+        e = torch.where(amax > 0, e, torch.full_like(e, -127.0)).clamp(-127.0, 127.0)
+        q = (w / torch.exp2(e).unsqueeze(-1)).to(torch.float8_e4m3fn)
+        codes[i:j] = q.view(torch.uint8).reshape(j - i, rows, K)
+        scales[i:j] = (e + 127.0).to(torch.uint8).transpose(1, 2)
+        del w, amax, e, q
+    return codes, scales
+
+
+def make_fp8(inp: Inputs) -> tuple:
+    """(routed, shared) FP8 sets made from the bf16 expert weights of ``inp``."""
+    def one(Wg, Wu, Wd):
+        g, gs = quantize_fp8(Wg)
+        u, us = quantize_fp8(Wu)
+        dn, ds = quantize_fp8(Wd)
+        return Fp8Set(g, gs, u, us, dn, ds)
+    return one(inp.W_gate, inp.W_up, inp.W_down), one(inp.Ws_gate, inp.Ws_up, inp.Ws_down)
