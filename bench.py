@@ -32,7 +32,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import ALL_WORKLOADS, Workload, make_inputs  # noqa: E402
+from workloads import ALL_WORKLOADS, Workload, make_fp8, make_inputs  # noqa: E402
 
 DEFAULT_WORKLOAD = "decode"
 
@@ -162,13 +162,19 @@ def sum_over_ranks(value: float, world: int, device) -> float:
 # ----------------------------------------------------------------------------
 # algorithmic work of one forward (counts only touched expert weights, W_r, x, y)
 # ----------------------------------------------------------------------------
+def weight_bytes_per_element(wl: Workload) -> float:
+    """bf16: 2 bytes; FP8: 1 byte of code plus 1/32 byte of block scale."""
+    return 1.0 + 1.0 / 32 if wl.weights == "fp8" else 2.0
+
+
 def algorithmic_work(wl: Workload, counts: np.ndarray) -> dict:
     touched = int((counts > 0).sum())
-    per_expert_w = 3 * wl.F * wl.d * 2
+    bpe = weight_bytes_per_element(wl)
+    per_expert_w = int(3 * wl.F * wl.d * bpe)
     w_bytes = (touched + wl.S) * per_expert_w
     rows = wl.T * wl.k + wl.S * wl.T
-    gate_up_bytes = (touched + wl.S) * 2 * wl.F * wl.d * 2
-    down_bytes = (touched + wl.S) * wl.F * wl.d * 2
+    gate_up_bytes = int((touched + wl.S) * 2 * wl.F * wl.d * bpe)
+    down_bytes = int((touched + wl.S) * wl.F * wl.d * bpe)
     return {
         "touched_experts": touched,
         "layer_bytes": w_bytes + wl.E * wl.d * 4 + 2 * wl.T * wl.d * 2,
@@ -181,7 +187,7 @@ def algorithmic_work(wl: Workload, counts: np.ndarray) -> dict:
     }
 
 
-def measured_traffic(kernel: str, bound: str, units: int):
+def measured_traffic(kernel: str, bound: str, units: int, weights: str = "bf16"):
     """DRAM bytes per launch of ``kernel`` scaled from the committed ncu capture
     (profiles/traffic.json), or None when there is none or the kernel source has
     changed since the counters were taken."""
@@ -189,8 +195,9 @@ def measured_traffic(kernel: str, bound: str, units: int):
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
+    key = f"{kernel}/{bound}" + ("/fp8" if weights == "fp8" else "")
     with open(path) as f:
-        entry = json.load(f).get(f"{kernel}/{bound}")
+        entry = json.load(f).get(key)
     if not entry or entry.get("bound") != bound:
         return None
     src = os.path.join(ROOT, "mixture_experts_layer_47_b200", "csrc",
@@ -228,10 +235,24 @@ def run_ours(args, rank, local, world):
     # step behind it, so no launch latency falls inside the timed interval
     flush = torch.empty(1 << 30, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
+    fp8 = None
+    if wl.weights == "fp8":
+        fp8 = make_fp8(inp)   # the FP8 checkpoint of the same draws
+        inp.W_gate = inp.W_up = inp.W_down = None   # the bf16 copies are not used
+        inp.Ws_gate = inp.Ws_up = inp.Ws_down = None
+        torch.cuda.empty_cache()
     weights = (inp.W_gate, inp.W_up, inp.W_down, inp.Ws_gate, inp.Ws_up, inp.Ws_down)
 
+    def forward(x_arg, y_arg, host=False):
+        if fp8 is not None:
+            f = moe.moe_forward_fp8_host if host else moe.moe_forward_fp8
+            f(h, x_arg, inp.W_router, inp.bias, fp8[0], fp8[1], y_arg, ws, stream)
+        else:
+            f = moe.moe_forward_host if host else moe.moe_forward
+            f(h, x_arg, inp.W_router, inp.bias, *weights, y_arg, ws, stream)
+
     def step():
-        moe.moe_forward(h, inp.x, inp.W_router, inp.bias, *weights, y, ws, stream)
+        forward(inp.x, y)
 
     for _ in range(args.warmup):
         flush.fill_(1)
@@ -286,7 +307,7 @@ def run_ours(args, rank, local, world):
     x_host = inp.x.cpu().pin_memory()
     y_host = torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory()
     for _ in range(max(1, args.warmup)):
-        moe.moe_forward_host(h, x_host, inp.W_router, inp.bias, *weights, y_host, ws, stream)
+        forward(x_host, y_host, host=True)
     torch.cuda.synchronize(device)
     barrier(world)
     e2e_ms = []
@@ -294,7 +315,7 @@ def run_ours(args, rank, local, world):
         flush.fill_(i & 0xFF)
         torch.cuda.synchronize(device)
         t0 = time.perf_counter()
-        moe.moe_forward_host(h, x_host, inp.W_router, inp.bias, *weights, y_host, ws, stream)
+        forward(x_host, y_host, host=True)
         stream.synchronize()
         e2e_ms.append((time.perf_counter() - t0) * 1e3)
     barrier(world)
@@ -318,7 +339,8 @@ def run_ours(args, rank, local, world):
         peak = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4)}
-    traffic = measured_traffic(dominant, roof["bound"], work["touched_experts"] + wl.S)
+    traffic = measured_traffic(dominant, roof["bound"], work["touched_experts"] + wl.S,
+                               wl.weights)
     roof.update({"kernel": dominant, "traffic": traffic, "peak_source": peaks["source"],
                  "algorithmic_per_launch": work[key + ("_bytes" if roof["bound"] == "hbm"
                                                        else "_flops")],
@@ -342,7 +364,7 @@ def run_ours(args, rank, local, world):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, random-init weights)",
         "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d, "n_experts": wl.E,
                    "top_k": wl.k, "d_ff": wl.F, "n_shared": wl.S, "router": wl.router,
-                   "zipf_s": wl.zipf_s, "global_batch": wl.T * world,
+                   "zipf_s": wl.zipf_s, "weights": wl.weights, "global_batch": wl.T * world,
                    "parallelism": f"replicas{world}",
                    "l2": "flushed before every step (1 GB write, outside the timed interval)"},
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
@@ -353,8 +375,11 @@ def run_ours(args, rank, local, world):
         "layer": layer,
         "clocks": clocks.summary(),
     }
+    if fp8 is not None:
+        out["weights"] = ("fp8: E4M3 codes, one power-of-two scale per 32 K elements of a row, "
+                          "decoded to bf16 in shared memory; bf16 tensor-core MMAs")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(inp, args.cpu_seconds)
+        out["cpu_baseline"] = cpu_baseline(inp, args.cpu_seconds, fp8)
     if rank == 0:
         print(json.dumps(out), flush=True)
 
@@ -362,8 +387,9 @@ def run_ours(args, rank, local, world):
 # ----------------------------------------------------------------------------
 # the fp64 oracle on the host cores (CPU baseline and reference arm)
 # ----------------------------------------------------------------------------
-def _oracle_sample(inp, tokens: np.ndarray):
-    """Host copies the oracle needs for these tokens: x, router, bias, used experts."""
+def _oracle_sample(inp, tokens: np.ndarray, fp8=None):
+    """Host copies the oracle needs for these tokens: x, router, bias, used experts (for an
+    FP8 checkpoint, those experts decoded by the oracle once, like loading a checkpoint)."""
     import oracle
     x = inp.x.cpu()
     Wr = inp.W_router.cpu()
@@ -371,6 +397,8 @@ def _oracle_sample(inp, tokens: np.ndarray):
     logits = oracle.router_logits(x[tokens], Wr, b)
     idx, _, _ = oracle.route(logits, inp.wl.k)
     used = sorted(set(idx.reshape(-1).tolist()))
+    if fp8 is not None:
+        return x[tokens].contiguous(), Wr, b, oracle.fp8_inputs(inp, fp8[0], fp8[1], used)
     W = {"W_gate": {e: inp.W_gate[e].cpu() for e in used},
          "W_up": {e: inp.W_up[e].cpu() for e in used},
          "W_down": {e: inp.W_down[e].cpu() for e in used},
@@ -393,11 +421,11 @@ def _sample_tokens(wl: Workload) -> np.ndarray:
     return np.unique(np.linspace(0, wl.T - 1, n).round().astype(np.int64))
 
 
-def cpu_baseline(inp, seconds: float) -> dict:
+def cpu_baseline(inp, seconds: float, fp8=None) -> dict:
     import oracle
     wl = inp.wl
     tokens = _sample_tokens(wl)
-    x, Wr, b, W = _oracle_sample(inp, tokens)
+    x, Wr, b, W = _oracle_sample(inp, tokens, fp8)
     passes, t0 = 0, time.perf_counter()
     while True:
         _oracle_pass(x, Wr, b, W, wl)
@@ -418,8 +446,9 @@ def run_reference(args, rank, local, world):
     wl = ALL_WORKLOADS[args.workload]
     device = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     inp = make_inputs(wl, device=device)
+    fp8 = make_fp8(inp) if wl.weights == "fp8" else None
     tokens = _sample_tokens(wl)
-    x, Wr, b, W = _oracle_sample(inp, tokens)
+    x, Wr, b, W = _oracle_sample(inp, tokens, fp8)
     for _ in range(args.warmup):
         _oracle_pass(x, Wr, b, W, wl)
     t0 = time.perf_counter()

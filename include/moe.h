@@ -194,6 +194,63 @@ moe_status moe_forward_host(moe_handle h, const uint16_t *x_host, const float *W
                             uint16_t *y_host, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * FP8 expert weights.  The Hy4 pages mention an FP8 checkpoint of the model
+ * (ZAKER Hy4 Preview release news; gpuvram.cloud "Tencent Hy4 preview" model
+ * card) but print no scaling scheme; this library takes the OCP microscaling
+ * layout.  Every expert weight is an FP8 E4M3 code (1 sign bit, 4 exponent
+ * bits with bias 7, 3 mantissa bits, no infinities, S.1111.111 = NaN, largest
+ * finite value 448), and each run of 32 consecutive K elements of a weight
+ * row shares one power-of-two scale stored as a biased exponent byte e
+ * (scale 2^(e - 127)).  Scales are stored K-block-major: scale[n][K/32][rows],
+ * so the scales of consecutive rows for one 32-element K block are adjacent.
+ * Each set holds n = E (routed) or n = S (shared) experts:
+ */
+typedef struct moe_fp8_expert_weights {
+  const uint8_t *gate;        /* [n][F][d]    E4M3 codes          */
+  const uint8_t *gate_scale;  /* [n][d/32][F] biased exponents    */
+  const uint8_t *up;          /* [n][F][d]                        */
+  const uint8_t *up_scale;    /* [n][d/32][F]                     */
+  const uint8_t *down;        /* [n][d][F]                        */
+  const uint8_t *down_scale;  /* [n][F/32][d]                     */
+} moe_fp8_expert_weights;
+
+/*
+ * moe_expert_ffn with FP8 expert weights.  The GEMMs decode codes and scales
+ * to bf16 in shared memory and run the same bf16 tensor-core contractions
+ * (fp32 accumulation, activation rounded to bf16, Y in fp32), so Y equals
+ * moe_expert_ffn's Y given the decoded weights.  The decoding is exact for
+ * every finite code whose scaled value is zero or at least 2^-133 in
+ * magnitude (bf16's smallest subnormal), which holds for scale bytes >= 7,
+ * and for scale bytes up to 134 (scales up to 2^7, weights up to 57344 in
+ * magnitude).  The E4M3 NaN codes (0x7F, 0xFF) and scale bytes above 134 are
+ * outside the accepted input: they decode to unspecified values.
+ * routed: the E routed experts' set (all six pointers required);
+ * shared: the S shared experts' set (NULL when S == 0).  Every pointer must be
+ * 16-byte aligned.  Other arguments as in moe_expert_ffn.
+ */
+moe_status moe_expert_ffn_fp8(moe_handle h, const uint16_t *x, const int32_t *perm,
+                              const int32_t *offsets, int T, const moe_fp8_expert_weights *routed,
+                              const moe_fp8_expert_weights *shared, float *Y, void *workspace,
+                              size_t ws_bytes, void *stream);
+
+/*
+ * moe_forward with FP8 expert weights (as in moe_expert_ffn_fp8); the router,
+ * dispatch and combine are those of moe_forward.
+ */
+moe_status moe_forward_fp8(moe_handle h, const uint16_t *x, const float *W_router,
+                           const float *bias, const moe_fp8_expert_weights *routed,
+                           const moe_fp8_expert_weights *shared, int T, uint16_t *y,
+                           void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * moe_forward_fp8 with the activations in host memory, as moe_forward_host.
+ */
+moe_status moe_forward_fp8_host(moe_handle h, const uint16_t *x_host, const float *W_router,
+                                const float *bias, const moe_fp8_expert_weights *routed,
+                                const moe_fp8_expert_weights *shared, int T, uint16_t *y_host,
+                                void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Synchronise the stream and read the workspace's device status word, which
  * the last call on this workspace wrote: MOE_OK, MOE_ERR_TIMEOUT or
  * MOE_ERR_BAD_INDEX.  *device_detail receives the raw word (0 if none).

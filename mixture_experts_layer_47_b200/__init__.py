@@ -37,7 +37,7 @@ EXPORTS = ("moe_create", "moe_destroy", "moe_workspace_size", "moe_get_workspace
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_host", "moe_device_status", "moe_set_stage_events",
            "moe_dispatch_noalloc", "moe_selftest_wait_timeout", "moe_forward_kernel_count",
-           "moe_status_string")
+           "moe_status_string", "moe_expert_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_host")
 MOE_STAGE_EVENTS = 7
 STAGE_NAMES = ("router", "dispatch", "gather", "gate_up_gemm", "down_gemm", "combine")
 
@@ -52,6 +52,12 @@ class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("status", "topk_idx", "topk_w", "counts", "offsets", "perm", "pos", "h_act",
                  "y_rows", "total", "router_partials", "router_ksplit")]
+
+
+class Fp8ExpertWeights(ctypes.Structure):
+    """struct moe_fp8_expert_weights: E4M3 codes and K-block-major scale bytes of one set."""
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("gate", "gate_scale", "up", "up_scale", "down", "down_scale")]
 
 
 _lib = None
@@ -85,6 +91,12 @@ def load_library() -> ctypes.CDLL:
         "moe_selftest_wait_timeout": ([P, Z, ctypes.c_ulonglong, P], I),
         "moe_forward_kernel_count": ([P, I], I),
         "moe_status_string": ([I], ctypes.c_char_p),
+        "moe_expert_ffn_fp8": ([P, P, P, P, I, ctypes.POINTER(Fp8ExpertWeights),
+                                ctypes.POINTER(Fp8ExpertWeights), P, P, Z, P], I),
+        "moe_forward_fp8": ([P, P, P, P, ctypes.POINTER(Fp8ExpertWeights),
+                             ctypes.POINTER(Fp8ExpertWeights), I, P, P, Z, P], I),
+        "moe_forward_fp8_host": ([P, P, P, P, ctypes.POINTER(Fp8ExpertWeights),
+                                  ctypes.POINTER(Fp8ExpertWeights), I, P, P, Z, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -236,6 +248,65 @@ def moe_expert_ffn(h: Handle, x, perm, offsets, W_gate, W_up, W_down, Ws_gate, W
         _ptr(offsets, torch.int32, "offsets", (h.E + 1,)), T,
         *_weights(h, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down),
         _ptr(Y, torch.float32, "Y", (rows, h.d)), wp, wn, _stream(stream)), "moe_expert_ffn")
+
+
+def _fp8_set(h: Handle, fs, n: int, name: str):
+    """A Fp8ExpertWeights for an object with uint8 tensors gate, gate_scale, up, up_scale,
+    down, down_scale (e.g. ``workloads.Fp8Set``); None when n == 0."""
+    if n == 0:
+        return None
+    if fs is None:
+        raise ValueError(f"{name}: FP8 weights required")
+    d, F = h.d, h.F
+    shapes = dict(gate=(n, F, d), gate_scale=(n, d // 32, F), up=(n, F, d),
+                  up_scale=(n, d // 32, F), down=(n, d, F), down_scale=(n, F // 32, d))
+    return Fp8ExpertWeights(**{k: _ptr(getattr(fs, k), torch.uint8, f"{name}.{k}", shp)
+                               for k, shp in shapes.items()})
+
+
+def _byref(s):
+    return None if s is None else ctypes.byref(s)
+
+
+def moe_expert_ffn_fp8(h: Handle, x, perm, offsets, routed, shared, Y, workspace,
+                       stream=None) -> None:
+    """moe_expert_ffn with FP8 expert weights (``routed``/``shared``: see ``_fp8_set``)."""
+    T = x.shape[0]
+    rows = T * h.k + h.S * T
+    wp, wn = _ws(workspace)
+    r, sh = _fp8_set(h, routed, h.E, "routed"), _fp8_set(h, shared, h.S, "shared")
+    _check(load_library().moe_expert_ffn_fp8(
+        h.value, _ptr(x, torch.bfloat16, "x", (T, h.d)),
+        _ptr(perm, torch.int32, "perm", (T * h.k,)),
+        _ptr(offsets, torch.int32, "offsets", (h.E + 1,)), T, _byref(r), _byref(sh),
+        _ptr(Y, torch.float32, "Y", (rows, h.d)), wp, wn, _stream(stream)),
+        "moe_expert_ffn_fp8")
+
+
+def moe_forward_fp8(h: Handle, x, W_router, bias, routed, shared, y, workspace,
+                    stream=None) -> None:
+    T = x.shape[0]
+    wp, wn = _ws(workspace)
+    r, sh = _fp8_set(h, routed, h.E, "routed"), _fp8_set(h, shared, h.S, "shared")
+    _check(load_library().moe_forward_fp8(
+        h.value, _ptr(x, torch.bfloat16, "x", (T, h.d)),
+        _ptr(W_router, torch.float32, "W_router", (h.E, h.d)),
+        _ptr(bias, torch.float32, "bias", (h.E,)), _byref(r), _byref(sh), T,
+        _ptr(y, torch.bfloat16, "y", (T, h.d)), wp, wn, _stream(stream)), "moe_forward_fp8")
+
+
+def moe_forward_fp8_host(h: Handle, x_host, W_router, bias, routed, shared, y_host, workspace,
+                         stream=None) -> None:
+    """x_host / y_host: CPU bf16 tensors (pinned for asynchronous copies)."""
+    T = x_host.shape[0]
+    wp, wn = _ws(workspace)
+    r, sh = _fp8_set(h, routed, h.E, "routed"), _fp8_set(h, shared, h.S, "shared")
+    _check(load_library().moe_forward_fp8_host(
+        h.value, _ptr(x_host, torch.bfloat16, "x_host", (T, h.d), "cpu"),
+        _ptr(W_router, torch.float32, "W_router", (h.E, h.d)),
+        _ptr(bias, torch.float32, "bias", (h.E,)), _byref(r), _byref(sh), T,
+        _ptr(y_host, torch.bfloat16, "y_host", (T, h.d), "cpu"), wp, wn, _stream(stream)),
+        "moe_forward_fp8_host")
 
 
 def moe_combine(h: Handle, Y, topk_w, pos, y, stream=None) -> None:

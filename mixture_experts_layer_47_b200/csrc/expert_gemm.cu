@@ -481,6 +481,7 @@ moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& d
       return MOE_ERR_CUDA;
     attrs_device = dev.device;
   }
+  if (a.fp8_routed) return launch_expert_ffn_fp8(c, a, dev, st);
   const int T = a.T;
   const GemmTiling tiling = gemm_tiling(c, T);
   if (tiling == GemmTiling::kSwap || tiling == GemmTiling::kSwapPair)

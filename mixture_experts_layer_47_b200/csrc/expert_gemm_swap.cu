@@ -47,6 +47,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "tensor_map.cuh"
+#include "weight_major.cuh"
 
 namespace moe {
 namespace {
@@ -61,7 +62,6 @@ constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_GROUPS = 1024 + 8;
 constexpr int MAX_STAGES = 6;
-constexpr int STG_LD = 33;                 // transpose staging row stride (floats)
 
 template <bool kGateUp, bool kPair>
 struct SwapCfg {
@@ -106,7 +106,7 @@ struct SharedStorage {
   int abort_flag;
   int sched[MAX_GROUPS + 1];
   int offsets[MAX_GROUPS + 1];
-  float stage_t[EPI_WARPS][16 * STG_LD];   // per epilogue warp: one 16-token x 32 block
+  float stage_t[EPI_WARPS][16 * wm::STG_LD];   // per epilogue warp: one 16-token x 32 block
 };
 
 template <bool kGateUp, bool kPair>
@@ -117,115 +117,6 @@ constexpr size_t swap_smem_bytes() {
 static_assert(swap_smem_bytes<true, false>() <= 227 * 1024, "shared memory budget");
 static_assert(swap_smem_bytes<true, true>() <= 227 * 1024, "shared memory budget");
 static_assert(swap_smem_bytes<false, true>() <= 227 * 1024, "shared memory budget");
-
-struct SwapTile {
-  int w_row;     // first weight row of the tile in the w / s maps (of the pair)
-  int f0;        // first output feature of the tile (of the pair)
-  int tok_row;   // first B row (token) in the tok map
-  int out_row;   // output row of the tile's first token
-  int cnt;       // valid tokens in the tile (1..TN)
-  int n;         // MMA N: cnt rounded up to 16
-  bool shared;
-};
-
-// Tiles are numbered group by group; inside a group weight-tile-major with the
-// group's token tiles innermost, so the CTAs that share a weight tile run at
-// the same time and read it through L2.  A group of r tokens has
-// mt = ceil(r / TN) token tiles of ceil(r / mt) tokens rounded up to 16
-// (at most TN, since mt * TN >= r), the last one holding the remainder.
-template <bool kGateUp, bool kPair>
-__device__ __forceinline__ SwapTile decode_swap_tile(int t, int n_wt, int G,
-                                                     const SharedStorage& ss,
-                                                     const SwapParams& p) {
-  using C = SwapCfg<kGateUp, kPair>;
-  const int q = t / n_wt;
-  int lo = 0, hi = G;  // largest g in [0, G) with sched[g] <= q
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (ss.sched[mid] <= q) lo = mid; else hi = mid;
-  }
-  const int mt = ss.sched[lo + 1] - ss.sched[lo];
-  const int local = t - ss.sched[lo] * n_wt;
-  const int w_idx = local / mt;
-  const int j = local - w_idx * mt;
-  const bool shared = lo >= p.E;
-  int rows = shared ? p.T : ss.offsets[lo + 1] - ss.offsets[lo];
-  rows = max(0, min(rows, mt * C::TN));
-  const int per = (((rows + mt - 1) / mt) + 15) & ~15;
-  SwapTile tl;
-  tl.shared = shared;
-  const int first = j * per;
-  tl.cnt = max(0, min(per, rows - first));
-  tl.n = (tl.cnt + 15) & ~15;
-  if (tl.n < 16) tl.n = 16;
-  tl.f0 = w_idx * C::FEAT;
-  const int nslots = p.T * p.k;
-  if (!shared) {
-    tl.w_row = lo * p.w_rows + tl.f0;
-    tl.tok_row = ss.offsets[lo] + first;
-    tl.out_row = tl.tok_row;
-  } else {
-    const int s = lo - p.E;
-    tl.w_row = s * p.w_rows + tl.f0;
-    tl.out_row = nslots + s * p.T + first;
-    tl.tok_row = kGateUp ? first : tl.out_row;
-  }
-  return tl;
-}
-
-// Store a 32-feature x 32-token block held feature-major (this lane = feature,
-// v[i] = token i) as 32 output rows: transpose 16 tokens at a time through the
-// warp's staging block, then each instruction writes whole 16-byte pieces of
-// consecutive rows.
-template <bool kBf16>
-__device__ __forceinline__ void store_block_transposed(float* stg, const float (&v)[32], int lane,
-                                                       void* out, int n_out, int row0, int ntok,
-                                                       int col0, int out_rows) {
-#pragma unroll
-  for (int hb = 0; hb < 2; ++hb) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) stg[i * STG_LD + lane] = v[16 * hb + i];
-    __syncwarp();
-    if (kBf16) {
-      // 4 lanes per token row (64 bytes), 8 rows per instruction
-      const int piece = lane & 3;
-#pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        const int tl = (lane >> 2) + 8 * s;
-        const float* src = stg + tl * STG_LD + 8 * piece;
-        const uint4 val = make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
-                                     pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
-        const int tok = 16 * hb + tl;
-        const int row = row0 + tok;
-        if (tok < ntok && row >= 0 && row < out_rows)
-          *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + size_t(row) * n_out +
-                                    col0 + 8 * piece) = val;
-      }
-    } else {
-      // 8 lanes per token row (128 bytes), 4 rows per instruction
-      const int piece = lane & 7;
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        const int tl = (lane >> 3) + 4 * s;
-        const float* src = stg + tl * STG_LD + 4 * piece;
-        const float4 val = make_float4(src[0], src[1], src[2], src[3]);
-        const int tok = 16 * hb + tl;
-        const int row = row0 + tok;
-        if (tok < ntok && row >= 0 && row < out_rows)
-          *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + size_t(row) * n_out + col0 +
-                                     4 * piece) = val;
-      }
-    }
-    __syncwarp();
-  }
-}
-
-// silu(g) * u.  The exponent is clamped so that 1 + e^-g stays below 2^126,
-// where the fast divide is accurate; below g = -80 silu(g) is -80 e^-80 or
-// smaller, which the clamp reproduces to far under the bf16 output's precision.
-__device__ __forceinline__ float swiglu(float g, float u) {
-  return __fdividef(g, 1.0f + __expf(fminf(-g, 80.0f))) * u;
-}
 
 template <bool kGateUp, bool kPair>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -300,7 +191,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t issued_mask = 0, issued_parity = 0;
       for (int t = unit; t < total && !aborted; t += n_units) {
         if (*abort_flag) { aborted = true; break; }
-        const SwapTile tl = decode_swap_tile<kGateUp, kPair>(t, n_wt, G, ss, p);
+        const wm::Tile tl = wm::decode_tile<C::TN, C::FEAT, kGateUp>(
+            t, n_wt, G, ss.sched, ss.offsets, p.E, p.T, p.k, p.w_rows);
         const CUtensorMap* mT = tl.shared ? &p.tok_shared : &p.tok_routed;
         const CUtensorMap* mW0 = tl.shared ? &p.s0 : &p.w0;
         const CUtensorMap* mW1 = kGateUp ? (tl.shared ? &p.s1 : &p.w1) : mW0;
@@ -357,7 +249,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t acc_phase = 0;
       for (int t = unit; t < total && !aborted; t += n_units) {
         if (*abort_flag) { aborted = true; break; }
-        const SwapTile tl = decode_swap_tile<kGateUp, kPair>(t, n_wt, G, ss, p);
+        const wm::Tile tl = wm::decode_tile<C::TN, C::FEAT, kGateUp>(
+            t, n_wt, G, ss.sched, ss.offsets, p.E, p.T, p.k, p.w_rows);
         const uint32_t idesc = umma_idesc_bf16_f32(C::MMA_M, tl.n);
         if (!mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1)) {
           report_error(p.status, kDevTimeout, kSiteMma);
@@ -422,7 +315,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t acc_phase = 0;
     for (int t = unit; t < total; t += n_units) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) { aborted = true; break; }  // warp-uniform
-      const SwapTile tl = decode_swap_tile<kGateUp, kPair>(t, n_wt, G, ss, p);
+      const wm::Tile tl = wm::decode_tile<C::TN, C::FEAT, kGateUp>(
+            t, n_wt, G, ss.sched, ss.offsets, p.E, p.T, p.k, p.w_rows);
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&ss.tmem_full[acc], acc_phase));
       if (!ok) {
         if (lane == 0) report_error(p.status, kDevTimeout, kSiteEpilogue);
@@ -451,9 +345,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              hp[j][i] = pack_bf16x2(swiglu(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
-                                     swiglu(__uint_as_float(g[2 * i + 1]),
-                                            __uint_as_float(u[2 * i + 1])));
+              hp[j][i] = pack_bf16x2(
+                  wm::swiglu(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                  wm::swiglu(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
           }
         }
         tc_fence_before();
@@ -469,7 +363,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               h[2 * i] = bf16_bits_to_float(hp[j][i] & 0xFFFFu);
               h[2 * i + 1] = bf16_bits_to_float(hp[j][i] >> 16);
             }
-            store_block_transposed<true>(stg, h, lane, p.out, p.n_out, tl.out_row + c,
+            wm::store_block_transposed<true>(stg, h, lane, p.out, p.n_out, tl.out_row + c,
                                          tl.cnt - c, col0, p.out_rows);
           }
         }
@@ -487,13 +381,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_ld_wait();
           float h[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) h[i] = swiglu(__uint_as_float(g[i]), __uint_as_float(u[i]));
+          for (int i = 0; i < 32; ++i)
+            h[i] = wm::swiglu(__uint_as_float(g[i]), __uint_as_float(u[i]));
           if (c + 64 < tl.n) {   // next chunk's loads overlap this chunk's stores
             tmem_ld_32cols(tbase + uint32_t(c + 64), g);
             tmem_ld_32cols(tbase + uint32_t(C::SECOND + c + 64), u);
           }
           if (cols_ok)
-            store_block_transposed<true>(stg, h, lane, p.out, p.n_out, tl.out_row + c,
+            wm::store_block_transposed<true>(stg, h, lane, p.out, p.n_out, tl.out_row + c,
                                          tl.cnt - c, col0, p.out_rows);
         }
       } else {
@@ -515,10 +410,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (c + 64 < tl.n) tmem_ld_32cols(hbase + uint32_t(c + 64), r);
             if (cols_ok) {
               if (p.out_bf16)
-                store_block_transposed<true>(stg, v, lane, p.out, p.n_out, tl.out_row + c,
+                wm::store_block_transposed<true>(stg, v, lane, p.out, p.n_out, tl.out_row + c,
                                              tl.cnt - c, col0, p.out_rows);
               else
-                store_block_transposed<false>(stg, v, lane, p.out, p.n_out, tl.out_row + c,
+                wm::store_block_transposed<false>(stg, v, lane, p.out, p.n_out, tl.out_row + c,
                                               tl.cnt - c, col0, p.out_rows);
             }
           }

@@ -120,10 +120,16 @@ struct FfnArgs {
   int* status;
   int T;
   cudaEvent_t after_gate_up;  // recorded between the two GEMMs when non-null
+  // FP8 weights (then Wg..Sd are unused): the routed set and the shared set
+  // (nullptr when S == 0); both nullptr for bf16 weights.
+  const moe_fp8_expert_weights* fp8_routed = nullptr;
+  const moe_fp8_expert_weights* fp8_shared = nullptr;
 };
 moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                              cudaStream_t st);
 moe_status launch_expert_ffn_swap(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                                   bool pair, cudaStream_t st);
+moe_status launch_expert_ffn_fp8(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
+                                 cudaStream_t st);
 
 }  // namespace moe

@@ -230,28 +230,78 @@ moe_status moe_dispatch(moe_handle h, const int32_t* topk_idx, int T, int32_t* c
                                      st));
 }
 
-static moe_status check_weights(const Ctx& c, const uint16_t* Wg, const uint16_t* Wu,
-                                const uint16_t* Wd, const uint16_t* Sg, const uint16_t* Su,
-                                const uint16_t* Sd) {
-  if (!Wg || !Wu || !Wd) return MOE_ERR_INVALID_ARG;
-  if (c.S > 0 && (!Sg || !Su || !Sd)) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(Wg) || !aligned16(Wu) || !aligned16(Wd)) return MOE_ERR_ALIGNMENT;
-  if (c.S > 0 && (!aligned16(Sg) || !aligned16(Su) || !aligned16(Sd))) return MOE_ERR_ALIGNMENT;
+// Expert weights of one call: bf16 (Wg..Sd) or FP8 (r8 / s8, the others null).
+struct Weights {
+  const uint16_t *Wg = nullptr, *Wu = nullptr, *Wd = nullptr;
+  const uint16_t *Sg = nullptr, *Su = nullptr, *Sd = nullptr;
+  const moe_fp8_expert_weights* r8 = nullptr;
+  const moe_fp8_expert_weights* s8 = nullptr;
+};
+
+static Weights bf16_weights(const uint16_t* Wg, const uint16_t* Wu, const uint16_t* Wd,
+                            const uint16_t* Sg, const uint16_t* Su, const uint16_t* Sd) {
+  Weights w;
+  w.Wg = Wg;
+  w.Wu = Wu;
+  w.Wd = Wd;
+  w.Sg = Sg;
+  w.Su = Su;
+  w.Sd = Sd;
+  return w;
+}
+
+static Weights fp8_weights(const moe_fp8_expert_weights* r8, const moe_fp8_expert_weights* s8) {
+  Weights w;
+  w.r8 = r8;
+  w.s8 = s8;
+  return w;
+}
+
+static moe_status check_fp8_set(const moe_fp8_expert_weights* w) {
+  if (!w) return MOE_ERR_INVALID_ARG;
+  const uint8_t* ptrs[6] = {w->gate, w->gate_scale, w->up, w->up_scale, w->down, w->down_scale};
+  for (const uint8_t* q : ptrs)
+    if (!q) return MOE_ERR_INVALID_ARG;
+  for (const uint8_t* q : ptrs)
+    if (!aligned16(q)) return MOE_ERR_ALIGNMENT;
   return MOE_OK;
 }
 
-moe_status moe_expert_ffn(moe_handle h, const uint16_t* x, const int32_t* perm,
-                          const int32_t* offsets, int T, const uint16_t* W_gate,
-                          const uint16_t* W_up, const uint16_t* W_down, const uint16_t* Ws_gate,
-                          const uint16_t* Ws_up, const uint16_t* Ws_down, float* Y,
-                          void* workspace, size_t ws_bytes, void* stream) {
+static moe_status check_weights(const Ctx& c, const Weights& w) {
+  if (w.r8 || w.s8) {
+    moe_status s = check_fp8_set(w.r8);
+    if (s) return s;
+    return c.S > 0 ? check_fp8_set(w.s8) : MOE_OK;
+  }
+  if (!w.Wg || !w.Wu || !w.Wd) return MOE_ERR_INVALID_ARG;
+  if (c.S > 0 && (!w.Sg || !w.Su || !w.Sd)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w.Wg) || !aligned16(w.Wu) || !aligned16(w.Wd)) return MOE_ERR_ALIGNMENT;
+  if (c.S > 0 && (!aligned16(w.Sg) || !aligned16(w.Su) || !aligned16(w.Sd)))
+    return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+static void set_weights(FfnArgs& a, const Weights& w) {
+  a.Wg = w.Wg;
+  a.Wu = w.Wu;
+  a.Wd = w.Wd;
+  a.Sg = w.Sg;
+  a.Su = w.Su;
+  a.Sd = w.Sd;
+  a.fp8_routed = w.r8;
+  a.fp8_shared = w.s8;
+}
+
+static moe_status expert_ffn_impl(moe_handle h, const uint16_t* x, const int32_t* perm,
+                                  const int32_t* offsets, int T, const Weights& w, float* Y,
+                                  void* workspace, size_t ws_bytes, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   const Ctx& c = h->c;
   moe_status s = check_T(c, T);
   if (s) return s;
   if (T == 0) return MOE_OK;
   if (!x || !perm || !offsets || !Y) return MOE_ERR_INVALID_ARG;
-  if ((s = check_weights(c, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down))) return s;
+  if ((s = check_weights(c, w))) return s;
   if (!aligned16(x) || !aligned16(Y)) return MOE_ERR_ALIGNMENT;
   if ((s = check_ws(h, T, workspace, ws_bytes))) return s;
   DeviceInfo* dev;
@@ -270,12 +320,7 @@ moe_status moe_expert_ffn(moe_handle h, const uint16_t* x, const int32_t* perm,
   a.x_perm = x_perm;
   a.offsets = offsets;
   a.sched = sched;
-  a.Wg = W_gate;
-  a.Wu = W_up;
-  a.Wd = W_down;
-  a.Sg = Ws_gate;
-  a.Su = Ws_up;
-  a.Sd = Ws_down;
+  set_weights(a, w);
   a.h_act = reinterpret_cast<uint16_t*>(ws + L.h_act);
   a.Y = Y;
   a.y_bf16 = false;
@@ -283,6 +328,25 @@ moe_status moe_expert_ffn(moe_handle h, const uint16_t* x, const int32_t* perm,
   a.T = T;
   a.after_gate_up = nullptr;
   return launch_expert_ffn(c, a, *dev, st);
+}
+
+moe_status moe_expert_ffn(moe_handle h, const uint16_t* x, const int32_t* perm,
+                          const int32_t* offsets, int T, const uint16_t* W_gate,
+                          const uint16_t* W_up, const uint16_t* W_down, const uint16_t* Ws_gate,
+                          const uint16_t* Ws_up, const uint16_t* Ws_down, float* Y,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  return expert_ffn_impl(h, x, perm, offsets, T,
+                         bf16_weights(W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down), Y,
+                         workspace, ws_bytes, stream);
+}
+
+moe_status moe_expert_ffn_fp8(moe_handle h, const uint16_t* x, const int32_t* perm,
+                              const int32_t* offsets, int T, const moe_fp8_expert_weights* routed,
+                              const moe_fp8_expert_weights* shared, float* Y, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  if (!routed) return MOE_ERR_INVALID_ARG;
+  return expert_ffn_impl(h, x, perm, offsets, T, fp8_weights(routed, shared), Y, workspace,
+                         ws_bytes, stream);
 }
 
 moe_status moe_combine(moe_handle h, const float* Y, const float* topk_w, const int32_t* pos,
@@ -300,11 +364,8 @@ moe_status moe_combine(moe_handle h, const float* Y, const float* topk_w, const 
 }
 
 static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W_router,
-                                 const float* bias, const uint16_t* W_gate, const uint16_t* W_up,
-                                 const uint16_t* W_down, const uint16_t* Ws_gate,
-                                 const uint16_t* Ws_up, const uint16_t* Ws_down, int T,
-                                 uint16_t* y, uint8_t* ws, const Layout& L, DeviceInfo* dev,
-                                 cudaStream_t st) {
+                                 const float* bias, const Weights& w, int T, uint16_t* y,
+                                 uint8_t* ws, const Layout& L, DeviceInfo* dev, cudaStream_t st) {
   const Ctx& c = h->c;
   moe_status s;
   int* status = reinterpret_cast<int*>(ws + L.status);
@@ -341,12 +402,7 @@ static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W
   a.x_perm = x_perm;
   a.offsets = offsets;
   a.sched = sched;
-  a.Wg = W_gate;
-  a.Wu = W_up;
-  a.Wd = W_down;
-  a.Sg = Ws_gate;
-  a.Su = Ws_up;
-  a.Sd = Ws_down;
+  set_weights(a, w);
   a.h_act = reinterpret_cast<uint16_t*>(ws + L.h_act);
   a.Y = Y;
   a.status = status;
@@ -360,49 +416,39 @@ static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W
 }
 
 static moe_status check_forward_args(moe_handle h, const uint16_t* x, const float* W_router,
-                                     const uint16_t* W_gate, const uint16_t* W_up,
-                                     const uint16_t* W_down, const uint16_t* Ws_gate,
-                                     const uint16_t* Ws_up, const uint16_t* Ws_down, int T,
-                                     const uint16_t* y, bool host_io, const void* workspace,
-                                     size_t ws_bytes) {
+                                     const Weights& w, int T, const uint16_t* y, bool host_io,
+                                     const void* workspace, size_t ws_bytes) {
   if (!x || !W_router || !y) return MOE_ERR_INVALID_ARG;
   moe_status s;
-  if ((s = check_weights(h->c, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down))) return s;
+  if ((s = check_weights(h->c, w))) return s;
   if (!aligned16(W_router)) return MOE_ERR_ALIGNMENT;
   if (!host_io && (!aligned16(x) || !aligned16(y))) return MOE_ERR_ALIGNMENT;
   return check_ws(h, T, workspace, ws_bytes);
 }
 
-moe_status moe_forward(moe_handle h, const uint16_t* x, const float* W_router, const float* bias,
-                       const uint16_t* W_gate, const uint16_t* W_up, const uint16_t* W_down,
-                       const uint16_t* Ws_gate, const uint16_t* Ws_up, const uint16_t* Ws_down,
-                       int T, uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
+static moe_status forward_impl(moe_handle h, const uint16_t* x, const float* W_router,
+                               const float* bias, const Weights& w, int T, uint16_t* y,
+                               void* workspace, size_t ws_bytes, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   moe_status s = check_T(h->c, T);
   if (s) return s;
   if (T == 0) return MOE_OK;
-  if ((s = check_forward_args(h, x, W_router, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, T,
-                              y, false, workspace, ws_bytes)))
-    return s;
+  if ((s = check_forward_args(h, x, W_router, w, T, y, false, workspace, ws_bytes))) return s;
   DeviceInfo* dev;
   if ((s = ensure_device(&dev))) return s;
   const Layout L = make_layout(h->c, T, kPlanSms);
-  return forward_device(h, x, W_router, bias, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, T,
-                        y, aligned_base(workspace), L, dev,
+  return forward_device(h, x, W_router, bias, w, T, y, aligned_base(workspace), L, dev,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
-moe_status moe_forward_host(moe_handle h, const uint16_t* x_host, const float* W_router,
-                            const float* bias, const uint16_t* W_gate, const uint16_t* W_up,
-                            const uint16_t* W_down, const uint16_t* Ws_gate,
-                            const uint16_t* Ws_up, const uint16_t* Ws_down, int T,
-                            uint16_t* y_host, void* workspace, size_t ws_bytes, void* stream) {
+static moe_status forward_host_impl(moe_handle h, const uint16_t* x_host, const float* W_router,
+                                    const float* bias, const Weights& w, int T, uint16_t* y_host,
+                                    void* workspace, size_t ws_bytes, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   moe_status s = check_T(h->c, T);
   if (s) return s;
   if (T == 0) return MOE_OK;
-  if ((s = check_forward_args(h, x_host, W_router, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down,
-                              T, y_host, true, workspace, ws_bytes)))
+  if ((s = check_forward_args(h, x_host, W_router, w, T, y_host, true, workspace, ws_bytes)))
     return s;
   DeviceInfo* dev;
   if ((s = ensure_device(&dev))) return s;
@@ -414,10 +460,45 @@ moe_status moe_forward_host(moe_handle h, const uint16_t* x_host, const float* W
   uint16_t* y_dev = reinterpret_cast<uint16_t*>(ws + L.y_stage);
   if ((s = cuda_status(cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st))))
     return s;
-  if ((s = forward_device(h, x_dev, W_router, bias, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down,
-                          T, y_dev, ws, L, dev, st)))
-    return s;
+  if ((s = forward_device(h, x_dev, W_router, bias, w, T, y_dev, ws, L, dev, st))) return s;
   return cuda_status(cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st));
+}
+
+moe_status moe_forward(moe_handle h, const uint16_t* x, const float* W_router, const float* bias,
+                       const uint16_t* W_gate, const uint16_t* W_up, const uint16_t* W_down,
+                       const uint16_t* Ws_gate, const uint16_t* Ws_up, const uint16_t* Ws_down,
+                       int T, uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
+  return forward_impl(h, x, W_router, bias,
+                      bf16_weights(W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down), T, y,
+                      workspace, ws_bytes, stream);
+}
+
+moe_status moe_forward_host(moe_handle h, const uint16_t* x_host, const float* W_router,
+                            const float* bias, const uint16_t* W_gate, const uint16_t* W_up,
+                            const uint16_t* W_down, const uint16_t* Ws_gate,
+                            const uint16_t* Ws_up, const uint16_t* Ws_down, int T,
+                            uint16_t* y_host, void* workspace, size_t ws_bytes, void* stream) {
+  return forward_host_impl(h, x_host, W_router, bias,
+                           bf16_weights(W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down), T,
+                           y_host, workspace, ws_bytes, stream);
+}
+
+moe_status moe_forward_fp8(moe_handle h, const uint16_t* x, const float* W_router,
+                           const float* bias, const moe_fp8_expert_weights* routed,
+                           const moe_fp8_expert_weights* shared, int T, uint16_t* y,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  if (!routed) return MOE_ERR_INVALID_ARG;
+  return forward_impl(h, x, W_router, bias, fp8_weights(routed, shared), T, y, workspace,
+                      ws_bytes, stream);
+}
+
+moe_status moe_forward_fp8_host(moe_handle h, const uint16_t* x_host, const float* W_router,
+                                const float* bias, const moe_fp8_expert_weights* routed,
+                                const moe_fp8_expert_weights* shared, int T, uint16_t* y_host,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  if (!routed) return MOE_ERR_INVALID_ARG;
+  return forward_host_impl(h, x_host, W_router, bias, fp8_weights(routed, shared), T, y_host,
+                           workspace, ws_bytes, stream);
 }
 
 moe_status moe_device_status(moe_handle h, int T, const void* workspace, void* stream,

@@ -39,4 +39,21 @@ inline bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, ui
   return r == CUDA_SUCCESS;
 }
 
+// 2-D byte tensor [rows][cols] (cols contiguous), box [box_rows][box_cols],
+// out-of-bounds elements read as zero; no swizzle unless given.
+inline bool encode_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                         int box_rows, int box_cols,
+                         CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {uint32_t(box_cols), uint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace moe

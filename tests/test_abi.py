@@ -142,6 +142,43 @@ def test_host_side_argument_errors_need_no_device(lib):
         moe.MOE_ERR_UNSUPPORTED
 
 
+def test_fp8_entry_points_validate_on_the_host(lib):
+    """The FP8 calls: a missing or incomplete weight set, a missing shared set when S = 1,
+    a misaligned code or scale pointer, and T = 0, all decided before any CUDA call."""
+    h = moe.moe_create(256, 16, 2, 128, 1)
+    hv = h.value
+    T = 64
+    ws_size = moe.moe_workspace_size(h, T)
+    A = 1 << 20
+    L = moe.load_library()
+    full = moe.Fp8ExpertWeights(A, A, A, A, A, A)
+    holed = moe.Fp8ExpertWeights(A, A, A, None, A, A)
+    skew = moe.Fp8ExpertWeights(A, A, A, A, A, A + 8)
+    ref = ctypes.byref
+    assert L.moe_forward_fp8(hv, A, A, None, None, ref(full), T, A, A, ws_size, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert L.moe_forward_fp8(hv, A, A, None, ref(holed), ref(full), T, A, A, ws_size, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert L.moe_forward_fp8(hv, A, A, None, ref(full), None, T, A, A, ws_size, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert L.moe_forward_fp8(hv, A, A, None, ref(skew), ref(full), T, A, A, ws_size, None) == \
+        moe.MOE_ERR_ALIGNMENT
+    assert L.moe_forward_fp8(hv, A, A, None, ref(full), ref(full), T, A, A, ws_size - 1,
+                             None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_forward_fp8_host(hv, A, None, None, ref(full), ref(full), T, A, A, ws_size,
+                                  None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_ffn_fp8(hv, A, A, A, T, ref(full), ref(skew), A, A, ws_size, None) == \
+        moe.MOE_ERR_ALIGNMENT
+    assert L.moe_expert_ffn_fp8(hv, A, None, A, T, ref(full), ref(full), A, A, ws_size,
+                                None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_forward_fp8(hv, None, None, None, ref(full), None, 0, None, None, 0, None) == \
+        moe.MOE_OK
+    # no shared experts: the shared set may be NULL
+    h0 = moe.moe_create(256, 16, 2, 128, 0)
+    assert L.moe_forward_fp8(h0.value, A, A, None, ref(full), None, T, A, A, 10, None) == \
+        moe.MOE_ERR_WORKSPACE
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
 def test_valid_call_without_device_reports_cuda_error(lib):
     """With valid arguments but no GPU, a launch returns MOE_ERR_CUDA instead of crashing."""
