@@ -103,6 +103,10 @@ PROFILE_WORKLOADS = {
         "profile_prefill_e32", T=1024, d=6144, E=32, k=8, F=2048, S=1, router="uniform", seed=0,
         description="prefill-shaped profiling case: T=1024 (256 rows per expert), d=6144, "
                     "32 experts top-8 + 1 shared"),
+    "profile_decode_fp8_e32": Workload(
+        "profile_decode_fp8_e32", T=16, d=6144, E=32, k=8, F=2048, S=1, router="normal", seed=0,
+        weights="fp8",
+        description="decode-shaped profiling case with FP8 expert weights (1.2 GB of codes)"),
 }
 ALL_WORKLOADS = {**WORKLOADS, **PROFILE_WORKLOADS}
 
