@@ -51,38 +51,44 @@ __global__ void __launch_bounds__(kGatherThreads)
   }
 }
 
-// Token-major gather: one warp reads a token's row of x once (in chunks held in
-// registers) and writes it to the token's k positions pos[t*k + i].  x is read
-// once instead of k times, so the X_perm write stream cannot push it out of L2.
+// Token-major gather: a warp reads a segment of a token's row of x once (held
+// in registers) and writes it to the token's k positions pos[t*k + i].  x is
+// read once instead of k times, so the X_perm write stream cannot push it out of
+// L2.  Work items are (token, segment) pairs; segments are seg_vecs 16-byte
+// vectors (a multiple of 32, at most 256), chosen short when there are few
+// tokens so that enough warps are in flight.
 __global__ void __launch_bounds__(kGatherThreads)
     gather_tokens_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ pos, int T,
-                         int k, int d, uint16_t* __restrict__ x_perm) {
+                         int k, int d, int seg_vecs, uint16_t* __restrict__ x_perm) {
   pdl_wait();
   pdl_launch_dependents();
   const int nslots = T * k;
   const int warps_total = gridDim.x * (kGatherThreads / 32);
   const int lane = threadIdx.x & 31;
   const int vec = d / 8;  // 16-byte vectors per row
-  constexpr int kChunk = 8;  // vectors per lane held at once
-  for (int t = blockIdx.x * (kGatherThreads / 32) + (threadIdx.x >> 5); t < T;
-       t += warps_total) {
+  const int nseg = (vec + seg_vecs - 1) / seg_vecs;
+  const int per_lane = seg_vecs / 32;
+  constexpr int kChunk = 8;  // vectors per lane held at once (seg_vecs <= 256)
+  const int64_t items = int64_t(T) * nseg;
+  for (int64_t item = blockIdx.x * (kGatherThreads / 32) + (threadIdx.x >> 5); item < items;
+       item += warps_total) {
+    const int t = int(item / nseg);
+    const int base = int(item - int64_t(t) * nseg) * seg_vecs;
     const uint4* __restrict__ src = reinterpret_cast<const uint4*>(x + size_t(t) * d);
-    for (int base = 0; base < vec; base += 32 * kChunk) {
-      uint4 v[kChunk];
+    uint4 v[kChunk];
+#pragma unroll
+    for (int j = 0; j < kChunk; ++j) {
+      const int i = base + lane + 32 * j;
+      if (j < per_lane && i < vec) v[j] = src[i];
+    }
+    for (int c = 0; c < k; ++c) {
+      const int p = pos[size_t(t) * k + c];
+      if (p < 0 || p >= nslots) continue;
+      uint4* __restrict__ dst = reinterpret_cast<uint4*>(x_perm + size_t(p) * d);
 #pragma unroll
       for (int j = 0; j < kChunk; ++j) {
         const int i = base + lane + 32 * j;
-        if (i < vec) v[j] = src[i];
-      }
-      for (int c = 0; c < k; ++c) {
-        const int p = pos[size_t(t) * k + c];
-        if (p < 0 || p >= nslots) continue;
-        uint4* __restrict__ dst = reinterpret_cast<uint4*>(x_perm + size_t(p) * d);
-#pragma unroll
-        for (int j = 0; j < kChunk; ++j) {
-          const int i = base + lane + 32 * j;
-          if (i < vec) dst[i] = v[j];
-        }
+        if (j < per_lane && i < vec) dst[i] = v[j];
       }
     }
   }
@@ -160,11 +166,16 @@ cudaError_t launch_gather(const Ctx& c, const uint16_t* x, const int32_t* perm,
 cudaError_t launch_gather_tokens(const Ctx& c, const uint16_t* x, const int32_t* pos, int T,
                                  uint16_t* x_perm, int num_sms, cudaStream_t st) {
   const int warps_per_block = kGatherThreads / 32;
-  int blocks = (T + warps_per_block - 1) / warps_per_block;
-  blocks = blocks < num_sms * 8 ? blocks : num_sms * 8;
+  const int vec = c.d / 8;
+  // 4 KB segments, or 1 KB ones when 4 KB segments would leave most SMs idle
+  int seg_vecs = 256;
+  if (int64_t(T) * ((vec + 255) / 256) < int64_t(4) * num_sms) seg_vecs = 64;
+  const int64_t items = int64_t(T) * ((vec + seg_vecs - 1) / seg_vecs);
+  int64_t blocks = (items + warps_per_block - 1) / warps_per_block;
+  if (blocks > int64_t(num_sms) * 8) blocks = int64_t(num_sms) * 8;
   if (blocks < 1) blocks = 1;
-  return launch_pdl(gather_tokens_kernel, dim3(blocks), dim3(kGatherThreads), 0, st, 1, x, pos,
-                    T, c.k, c.d, x_perm);
+  return launch_pdl(gather_tokens_kernel, dim3(unsigned(blocks)), dim3(kGatherThreads), 0, st, 1,
+                    x, pos, T, c.k, c.d, seg_vecs, x_perm);
 }
 
 cudaError_t launch_combine(const Ctx& c, const float* Y, const float* topk_w, const int32_t* pos,

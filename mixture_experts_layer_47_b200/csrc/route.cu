@@ -176,9 +176,9 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
 template <int TPC>
 __global__ void __launch_bounds__(1024)
     router_topk_kernel(const float* __restrict__ part, const float* __restrict__ bias, int T, int E,
-                       int k, int ksplit, int32_t* __restrict__ topk_idx,
+                       int k, int ksplit, int nsub, int32_t* __restrict__ topk_idx,
                        float* __restrict__ topk_w) {
-  extern __shared__ float logit_all[];  // [TPC][E]
+  extern __shared__ float logit_all[];  // [TPC][E], then (TPC == 1) [nsub][E] partial sums
   pdl_wait();
   pdl_launch_dependents();
   const int per_tok = blockDim.x / TPC;                 // threads per token
@@ -186,21 +186,41 @@ __global__ void __launch_bounds__(1024)
   const int t = blockIdx.x * TPC + grp;
   if (t >= T) return;   // whole token groups (warps) leave together
   float* logit = logit_all + grp * E;
-  for (int e = tid; e < E; e += per_tok) {
+  // With one CTA per token and threads to spare, nsub threads share an expert: each adds a
+  // contiguous run of the split-K partials in order, and the runs are added in order after
+  // (nsub is 1 for TPC > 1; the launch sizes shared memory for [1 + nsub][E] floats).
+  const int run = (ksplit + nsub - 1) / nsub;
+  float* sub = logit_all + TPC * E;
+  for (int idx = tid; idx < E * nsub; idx += per_tok) {
+    const int e = idx % E, q = idx / E;
     float s = 0.f;
     const float* p = part + size_t(t) * E + e;
     const size_t stride = size_t(T) * E;
-    int ks = 0;
-    for (; ks + 8 <= ksplit; ks += 8) {   // eight independent loads in flight, added in order
+    const int k1 = min(ksplit, (q + 1) * run);
+    int ks = q * run;
+    for (; ks + 8 <= k1; ks += 8) {   // eight independent loads in flight, added in order
       float v[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = p[(ks + q) * stride];
+      for (int j = 0; j < 8; ++j) v[j] = p[(ks + j) * stride];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) s += v[q];
+      for (int j = 0; j < 8; ++j) s += v[j];
     }
-    for (; ks < ksplit; ++ks) s += p[ks * stride];
-    if (bias) s += bias[e];
-    logit[e] = (s == s) ? s : -INFINITY;  // a NaN score is never preferred
+    for (; ks < k1; ++ks) s += p[ks * stride];
+    if (nsub == 1) {
+      if (bias) s += bias[e];
+      logit[e] = (s == s) ? s : -INFINITY;  // a NaN score is never preferred
+    } else {
+      sub[q * E + e] = s;
+    }
+  }
+  if (nsub > 1) {
+    __syncthreads();
+    for (int e = tid; e < E; e += per_tok) {
+      float s = sub[e];
+      for (int q = 1; q < nsub; ++q) s += sub[q * E + e];
+      if (bias) s += bias[e];
+      logit[e] = (s == s) ? s : -INFINITY;
+    }
   }
   if (TPC == 1) __syncthreads(); else __syncwarp();
   if (tid >= 32) return;
@@ -314,11 +334,14 @@ cudaError_t launch_router(const Ctx& c, const RouterPlan& rp, const uint16_t* x,
   if (err != cudaSuccess) return err;
   if (rp.ksplit <= 4)   // a warp per token, 8 tokens per CTA
     return launch_pdl(router_topk_kernel<8>, dim3((T + 7) / 8), dim3(256), 8 * c.E * sizeof(float),
-                      st, 1, static_cast<const float*>(part), bias, T, c.E, c.k, rp.ksplit,
+                      st, 1, static_cast<const float*>(part), bias, T, c.E, c.k, rp.ksplit, 1,
                       topk_idx, topk_w);
-  const int threads = std::min(1024, std::max(32, (c.E + 31) / 32 * 32));
-  return launch_pdl(router_topk_kernel<1>, dim3(T), dim3(threads), c.E * sizeof(float), st, 1,
-                    static_cast<const float*>(part), bias, T, c.E, c.k, rp.ksplit, topk_idx,
+  // a CTA per token; up to four threads per expert share its partial sums
+  const int nsub = std::max(1, std::min(4, std::min(rp.ksplit / 8, 1024 / std::max(1, c.E))));
+  const int threads = std::min(1024, std::max(32, (nsub * c.E + 31) / 32 * 32));
+  const size_t smem = size_t(1 + nsub) * c.E * sizeof(float);
+  return launch_pdl(router_topk_kernel<1>, dim3(T), dim3(threads), smem, st, 1,
+                    static_cast<const float*>(part), bias, T, c.E, c.k, rp.ksplit, nsub, topk_idx,
                     topk_w);
 }
 
