@@ -23,7 +23,8 @@ def lib():
 
 
 def declared_symbols():
-    text = open(HEADER).read()
+    with open(HEADER) as f:
+        text = f.read()
     return sorted(set(re.findall(r"^\s*(?:moe_status|size_t|int|const char \*)\s*(moe_\w+)\s*\(",
                                  text, re.M)))
 

@@ -82,7 +82,8 @@ def test_measured_traffic_lookup_and_invalidation(tmp_path, monkeypatch):
 
 def test_committed_traffic_table_names_existing_sources():
     path = os.path.join(os.path.dirname(os.path.dirname(__file__)), "profiles", "traffic.json")
-    table = json.load(open(path))
+    with open(path) as f:
+        table = json.load(f)
     assert table, "profiles/traffic.json is empty"
     for key, entry in table.items():
         kernel, bound = key.split("/")[:2]
