@@ -80,7 +80,8 @@ __global__ void __launch_bounds__(kRouterThreads)
       wr[l][0] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (i < W_LOADS) {
         const int r = i / (kBK / 4), c4 = (i % (kBK / 4)) * 4;
-        if (e0 + r < E) wr[l][0] = *reinterpret_cast<const float4*>(Wr + size_t(e0 + r) * d + k0 + c4);
+        if (e0 + r < E)
+          wr[l][0] = *reinterpret_cast<const float4*>(Wr + size_t(e0 + r) * d + k0 + c4);
       }
     }
   };
@@ -277,9 +278,9 @@ cudaError_t launch_partial(const Ctx& c, const RouterPlan& rp, const uint16_t* x
 
 // Path and tile shape by batch size.  The score GEMM runs on the tensor cores
 // (router_tc.cu) for more than 32 tokens and on fp32 FFMA tiles otherwise;
-// MOE_ROUTER=tc|ffma forces one.  Both compute fp32-accurate logits.  The FFMA K split is chosen so the grid
-// fills the GPU (about two CTAs per SM, counted for a 148-SM part so that the
-// plan, and with it the summation order, is the same on every device).
+// MOE_ROUTER=tc|ffma forces one.  Both compute fp32-accurate logits.  The FFMA K split is chosen
+// so the grid fills the GPU (about two CTAs per SM, counted for a 148-SM part so that the plan,
+// and with it the summation order, is the same on every device).
 RouterPlan router_plan(const Ctx& c, int T, int num_sms) {
   RouterPlan rp;
   const char* env = getenv("MOE_ROUTER");

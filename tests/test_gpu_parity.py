@@ -2,9 +2,9 @@
 
 Sizes span several tiles and ragged tails (groups not a multiple of the GEMMs'
 128- or 256-row tiles or 16-token N step, d_ff not a multiple of the 128- or
-256-feature gate/up tile, d not a multiple of the 256-feature down tile, dispatch runs over more than one 4096-slot
-block) plus the degenerate cases (one token, one expert, k = E, no shared
-expert, every token on one expert, an empty expert).
+256-feature gate/up tile, d not a multiple of the 256-feature down tile, dispatch
+runs over more than one 4096-slot block) plus the degenerate cases (one token,
+one expert, k = E, no shared expert, every token on one expert, an empty expert).
 """
 import numpy as np
 import pytest
