@@ -87,7 +87,7 @@ Layout make_layout(const Ctx& c, int T, int num_sms) {
   L.sched = take(2 * size_t(c.E + c.S + 1) * sizeof(int32_t));  // 128- and 256-row tiles
   L.x_perm = take(nslots * c.d * sizeof(uint16_t));
   L.h_act = take(rows * c.F * sizeof(uint16_t));
-  L.y_rows = take(rows * c.d * sizeof(float));  // fp32 for moe_expert_ffn, bf16 in moe_forward
+  L.y_rows = take(rows * c.d * sizeof(uint16_t));  // bf16 rows of moe_forward
   L.x_stage = take(size_t(T) * c.d * sizeof(uint16_t));
   L.y_stage = take(size_t(T) * c.d * sizeof(uint16_t));
   L.end = off;
