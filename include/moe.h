@@ -68,6 +68,10 @@ typedef int moe_status;
  * 1 <= E <= 1024; 1 <= k <= min(E, 32); 0 <= S <= 8.  Shapes outside it give
  * MOE_ERR_UNSUPPORTED, impossible ones MOE_ERR_INVALID_ARG.  No CUDA call is
  * made here; the device is checked (sm_100 required) at the first launch.
+ * Two tuning overrides are read from the environment here, once, and fixed for
+ * the context's lifetime: MOE_ROUTER=tc|ffma (router path) and
+ * MOE_GEMM_TILES=single|pair|swap|swap_pair (expert GEMM tiling); all choices
+ * compute the same result.
  */
 moe_status moe_create(int d_model, int n_experts, int top_k, int d_ff, int n_shared,
                       moe_handle *out);
@@ -79,7 +83,8 @@ moe_status moe_destroy(moe_handle h);
  * Bytes of device workspace that any call below needs for T tokens
  * (0 when h is NULL or T < 0).  One workspace of this size serves every
  * call; it holds intermediates only and may be reused across calls that the
- * stream orders.  At the Hy4 shape and T = 8192 it is about 3 GB.
+ * stream orders.  At the Hy4 shape it is about 2.2 GB at T = 8192 and about
+ * 5 MB at T = 16.
  */
 size_t moe_workspace_size(moe_handle h, int T);
 
@@ -109,10 +114,11 @@ moe_status moe_get_workspace_layout(moe_handle h, int T, uintptr_t workspace_add
  * Router: score, top-k select and gate (explainer section 2.2).
  *   logits[t][e] = sum_j x[t][j] * W_router[e][j] + bias[e]     (fp32-accurate:
  *                  on the tensor cores with W_router split exactly into three
- *                  bf16 parts and every 64-wide K chunk accumulated separately
+ *                  bf16 parts and every 128-wide K chunk accumulated separately
  *                  and added in fp32 (T > 32), or with fp32 FMA on the CUDA
- *                  cores (T <= 32); MOE_ROUTER=tc|ffma in the environment forces
- *                  one; split-K partial sums added in a fixed order)
+ *                  cores (T <= 32); MOE_ROUTER=tc|ffma in the environment when
+ *                  the context is created forces one for that context; split-K
+ *                  partial sums added in a fixed order)
  *   topk_idx[t][i] = the i-th largest logit's expert (ties: lower index)
  *   topk_w[t][i]   = exp(l_i - l_0) / sum_{j<k} exp(l_j - l_0)
  * x: bf16 [T][d]; W_router: fp32 [E][d]; bias: fp32 [E] or NULL;
@@ -130,7 +136,10 @@ moe_status moe_route(moe_handle h, const uint16_t *x, const float *W_router, con
  *   perm[p]    = slot at position p; ascending slots within each expert
  *   pos[s]     = position of slot s (perm[pos[s]] == s)      int32 [T*k] each
  * Indices outside [0, E) are skipped and flagged MOE_ERR_BAD_INDEX in the
- * workspace status word.
+ * workspace status word: such a slot gets pos[s] = -1 and belongs to no
+ * segment, offsets[E] is then the number of valid slots (less than T*k), and
+ * perm[p] for p >= offsets[E] is left unwritten.  moe_combine and
+ * moe_forward leave slots with pos = -1 out of the sum.
  */
 moe_status moe_dispatch(moe_handle h, const int32_t *topk_idx, int T, int32_t *counts,
                         int32_t *offsets, int32_t *perm, int32_t *pos, void *workspace,
@@ -280,18 +289,24 @@ moe_status moe_set_stage_events(moe_handle h, void *const *events, int n_events)
  * Same arguments and results as moe_dispatch, minus the workspace: the
  * scratch it needs (per-block histograms, the GEMM tile schedule, a status
  * word) lives in a fixed array of about 74 KB compiled into the library,
- * which every GPU that loads the library keeps until the process exits.
+ * which every CUDA context that loads the library's kernels keeps until the
+ * context ends (for a device's primary context: process exit or
+ * cudaDeviceReset).
  * Limits: T * k <= 65536 slots and E <= 1024; larger calls return
  * MOE_ERR_WORKSPACE and enqueue nothing.  It allocates nothing: no
  * cudaMalloc / cudaFree or allocating library routine.
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) and caches it; make that first call before any
- * stream capture.  All calls share the one array and it keeps the last
+ * Every call looks up the array's device address in the calling thread's
+ * current CUDA context (cudaGetSymbolAddress, a lookup that allocates
+ * nothing), so the array used is the one of the context current at the call,
+ * also under a context the host application created itself and after a
+ * cudaDeviceReset.  The first call in a context also loads the library's
+ * kernels into it; make that first call before any stream capture.  All
+ * calls in one context share the one array and it keeps the last
  * call's contents (each call clears what must start at zero), so calls that
  * overlap on the GPU -- on different streams without ordering between them
  * -- race and corrupt each other's results.  Out-of-range expert indices are
- * skipped as in moe_dispatch, but the status word is not readable through
- * this entry point.
+ * skipped as in moe_dispatch (pos = -1, offsets[E] = the number of valid
+ * slots), but the status word is not readable through this entry point.
  */
 moe_status moe_dispatch_noalloc(moe_handle h, const int32_t *topk_idx, int T, int32_t *counts,
                                 int32_t *offsets, int32_t *perm, int32_t *pos, void *stream);

@@ -185,6 +185,8 @@ __global__ void __launch_bounds__(kScatterWarps * 32)
       perm[p] = s;
       pos[s] = p;
       if (lane == __ffs(m) - 1) my[e] = base + __popc(m);
+    } else if (s < end) {
+      pos[s] = -1;   // a skipped (out-of-range) slot: no position, left out of the combine
     }
     __syncwarp();
   }
@@ -259,6 +261,8 @@ __global__ void __launch_bounds__(kScanThreads)
       perm[p] = s;
       pos[s] = p;
       if (lane == __ffs(m) - 1) my[e2] = base + __popc(m);
+    } else if (s < end) {
+      pos[s] = -1;   // a skipped (out-of-range) slot: no position, left out of the combine
     }
     __syncwarp();
   }

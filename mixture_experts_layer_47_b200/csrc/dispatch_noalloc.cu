@@ -10,14 +10,15 @@
 // with the same kernels, using a fixed scratch array compiled into this
 // library instead of a workspace.
 //
-// The scratch is a file-scope __device__ array: every GPU on which the
-// library's kernels are loaded holds its own copy (about 74 KB) until the
-// process exits.  Host code cannot use the array's name as a device pointer;
-// the device address is obtained once per device with cudaGetSymbolAddress
-// (on the first call made with that device current) and cached.
+// The scratch is a file-scope __device__ array: every CUDA context in which
+// the library's kernels are loaded holds its own copy (about 74 KB) until the
+// context or the process ends.  Host code cannot use the array's name as a
+// device pointer; every call asks for the array's address in the calling
+// thread's current context with cudaGetSymbolAddress (a lookup, not an
+// allocation).  The address is not cached: a cached one would belong to a
+// context that cudaDeviceReset has destroyed, or to the primary context when
+// a host application runs this code under a context of its own.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -37,23 +38,15 @@ constexpr int kScratchInts = kStatusInts + kHistInts + kSchedInts;
 
 static __device__ __align__(256) int32_t g_dispatch_scratch[kScratchInts];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-int32_t* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_dispatch_scratch on the current device (looked up once per device).
-moe_status scratch_address(int device, int32_t** out) {
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[device]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
-    if (e != cudaSuccess || p == nullptr) {
-      cudaGetLastError();
-      return MOE_ERR_CUDA;
-    }
-    g_scratch_addr[device] = static_cast<int32_t*>(p);
+// Device address of g_dispatch_scratch in the current context.
+moe_status scratch_address(int32_t** out) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
+  if (e != cudaSuccess || p == nullptr) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
   }
-  *out = g_scratch_addr[device];
+  *out = static_cast<int32_t*>(p);
   return MOE_OK;
 }
 
@@ -77,7 +70,7 @@ extern "C" moe_status moe_dispatch_noalloc(moe_handle h, const int32_t* topk_idx
   moe_status s = ensure_device(&dev);
   if (s) return s;
   int32_t* scratch = nullptr;
-  if ((s = scratch_address(dev->device, &scratch))) return s;
+  if ((s = scratch_address(&scratch))) return s;
   int* status = reinterpret_cast<int*>(scratch);
   int32_t* blk_hist = scratch + kStatusInts;
   int32_t* sched = blk_hist + kHistInts;

@@ -459,14 +459,17 @@ cudaError_t launch_gemm(const GemmParams& gp, int num_sms, cudaStream_t st) {
 // 256 experts top-8, they are faster at every batch: the 1-SM form while
 // groups average fewer than 96 rows, the 2-SM form (half the shared-memory
 // traffic per MMA cycle, token tiles up to 256) from there on.
-// MOE_GEMM_TILES=single|pair|swap|swap_pair overrides the choice (all compute
-// the same result; for tuning and tests).
+// The context's tiling mode (MOE_GEMM_TILES=single|pair|swap|swap_pair at
+// moe_create) overrides the choice (all compute the same result; for tuning
+// and tests).
 GemmTiling gemm_tiling(const Ctx& c, int T) {
-  const char* v = getenv("MOE_GEMM_TILES");
-  if (v && strcmp(v, "pair") == 0) return GemmTiling::kPair;
-  if (v && strcmp(v, "single") == 0) return GemmTiling::kSingle;
-  if (v && strcmp(v, "swap") == 0) return GemmTiling::kSwap;
-  if (v && strcmp(v, "swap_pair") == 0) return GemmTiling::kSwapPair;
+  switch (c.tiles) {
+    case TilesMode::kPair: return GemmTiling::kPair;
+    case TilesMode::kSingle: return GemmTiling::kSingle;
+    case TilesMode::kSwap: return GemmTiling::kSwap;
+    case TilesMode::kSwapPair: return GemmTiling::kSwapPair;
+    case TilesMode::kAuto: break;
+  }
   return int64_t(T) * c.k >= int64_t(kSwapPairMinRowsPerExpert) * c.E ? GemmTiling::kSwapPair
                                                                         : GemmTiling::kSwap;
 }

@@ -40,8 +40,17 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Forced choices of the router path and the GEMM tiling (tuning and tests).  They are
+// read from the environment once, when the context is created (MOE_ROUTER,
+// MOE_GEMM_TILES), so the workspace size and every later call of one context
+// agree on the plan whatever the environment does afterwards.
+enum class RouterMode { kAuto, kTensorCore, kFfma };
+enum class TilesMode { kAuto, kSingle, kPair, kSwap, kSwapPair };
+
 struct Ctx {
   int d, E, k, F, S;
+  RouterMode router = RouterMode::kAuto;
+  TilesMode tiles = TilesMode::kAuto;
 };
 
 // Geometry of the router's split-K partial sums for T tokens.

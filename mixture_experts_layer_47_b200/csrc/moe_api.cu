@@ -7,6 +7,7 @@
 // workspace size and every result are the same on any sm_100 GPU.
 #include <cuda_runtime.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -147,6 +148,17 @@ moe_status moe_create(int d_model, int n_experts, int top_k, int d_ff, int n_sha
   moe_ctx* h = new (std::nothrow) moe_ctx;
   if (!h) return MOE_ERR_INVALID_ARG;
   h->c = Ctx{d_model, n_experts, top_k, d_ff, n_shared};
+  // Tuning overrides, fixed for the context's lifetime (unknown values are ignored).
+  if (const char* v = getenv("MOE_ROUTER")) {
+    if (strcmp(v, "tc") == 0) h->c.router = RouterMode::kTensorCore;
+    if (strcmp(v, "ffma") == 0) h->c.router = RouterMode::kFfma;
+  }
+  if (const char* v = getenv("MOE_GEMM_TILES")) {
+    if (strcmp(v, "single") == 0) h->c.tiles = TilesMode::kSingle;
+    if (strcmp(v, "pair") == 0) h->c.tiles = TilesMode::kPair;
+    if (strcmp(v, "swap") == 0) h->c.tiles = TilesMode::kSwap;
+    if (strcmp(v, "swap_pair") == 0) h->c.tiles = TilesMode::kSwapPair;
+  }
   h->n_stage_events = 0;
   *out = h;
   return MOE_OK;

@@ -278,15 +278,14 @@ cudaError_t launch_partial(const Ctx& c, const RouterPlan& rp, const uint16_t* x
 
 // Path and tile shape by batch size.  The score GEMM runs on the tensor cores
 // (router_tc.cu) for more than 32 tokens and on fp32 FFMA tiles otherwise;
-// MOE_ROUTER=tc|ffma forces one.  Both compute fp32-accurate logits.  The FFMA K split is chosen
+// the context's router mode (MOE_ROUTER=tc|ffma at moe_create) forces one.  Both compute fp32-accurate logits.  The FFMA K split is chosen
 // so the grid fills the GPU (about two CTAs per SM, counted for a 148-SM part so that the plan,
 // and with it the summation order, is the same on every device).
 RouterPlan router_plan(const Ctx& c, int T, int num_sms) {
   RouterPlan rp;
-  const char* env = getenv("MOE_ROUTER");
-  if (env && strcmp(env, "ffma") == 0)
+  if (c.router == RouterMode::kFfma)
     rp.tc = false;
-  else if (env && strcmp(env, "tc") == 0)
+  else if (c.router == RouterMode::kTensorCore)
     rp.tc = true;
   else
     rp.tc = T > 32;   // below that the FFMA tiles finish first (measured on B200)

@@ -87,3 +87,32 @@ def oracle_rows(inp, idx, perm, tokens_rows=None):
         h, y = oracle.expert_one(x[t], Wg.cpu(), Wu.cpu(), Wd.cpu())
         H[r], Y[r] = h, y
     return H, Y
+
+
+def bad_index_routing(T, E, k, seed):
+    """Random distinct experts per token with a few slots set out of range (E, E + 5, -1)."""
+    g = torch.Generator().manual_seed(seed)
+    idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
+    flat = idx.view(-1)
+    bad = torch.randperm(T * k, generator=g)[:max(2, T * k // 50)]
+    for j, s in enumerate(bad.tolist()):
+        flat[s] = (E, E + 5, -1)[j % 3]
+    return idx
+
+
+def check_skipped_slots(idx, E, counts, offsets, perm, pos):
+    """Dispatch of routing with out-of-range slots: those slots are skipped (pos = -1), the
+    valid ones are grouped exactly as a stable sort of the valid slots by expert."""
+    flat = np.asarray(idx).reshape(-1)
+    valid = (flat >= 0) & (flat < E)
+    slots = np.nonzero(valid)[0]
+    order = slots[np.argsort(flat[slots], kind="stable")]
+    n = len(order)
+    c = np.bincount(flat[valid], minlength=E)
+    np.testing.assert_array_equal(np.asarray(counts), c)
+    np.testing.assert_array_equal(np.asarray(offsets), np.concatenate([[0], np.cumsum(c)]))
+    assert int(offsets[-1]) == n < flat.size
+    np.testing.assert_array_equal(np.asarray(perm)[:n], order)
+    exp_pos = np.full(flat.size, -1, np.int64)
+    exp_pos[order] = np.arange(n)
+    np.testing.assert_array_equal(np.asarray(pos), exp_pos)

@@ -198,3 +198,25 @@ def test_python_binding_validates_tensors(lib):
     with pytest.raises(TypeError):
         moe.moe_route(h, x, torch.zeros(16, 256), None, torch.zeros(4, 2, dtype=torch.int32),
                       torch.zeros(4, 2), ws)
+
+
+def test_tuning_overrides_are_fixed_when_the_context_is_created(lib, monkeypatch):
+    """MOE_ROUTER / MOE_GEMM_TILES are read once by moe_create: changing the environment
+    afterwards changes neither the workspace size nor the plan of an existing context.
+    The two router paths carve the workspace differently (the tensor-core path keeps a
+    split copy of W_router, the FFMA path more split-K partials), so the size shows which
+    path a context took."""
+    T = 64
+    monkeypatch.setenv("MOE_ROUTER", "ffma")
+    monkeypatch.setenv("MOE_GEMM_TILES", "single")
+    h_ffma = moe.moe_create(6144, 256, 8, 2048, 1)
+    size_ffma = moe.moe_workspace_size(h_ffma, T)
+    monkeypatch.setenv("MOE_ROUTER", "tc")
+    monkeypatch.setenv("MOE_GEMM_TILES", "swap_pair")
+    assert moe.moe_workspace_size(h_ffma, T) == size_ffma
+    h_tc = moe.moe_create(6144, 256, 8, 2048, 1)
+    size_tc = moe.moe_workspace_size(h_tc, T)
+    assert size_tc != size_ffma
+    monkeypatch.delenv("MOE_ROUTER")
+    assert moe.moe_workspace_size(h_tc, T) == size_tc
+    assert moe.moe_workspace_size(h_ffma, T) == size_ffma

@@ -12,8 +12,8 @@ import torch
 
 import mixture_experts_layer_47_b200 as moe
 import oracle
-from gpu_helpers import (Y_REL_TOL, dispatch_parity, gpu_forward, oracle_rows, rel_err,
-                         route_parity)
+from gpu_helpers import (Y_REL_TOL, bad_index_routing, check_skipped_slots, dispatch_parity,
+                         gpu_forward, oracle_rows, rel_err, route_parity)
 from workloads import WORKLOADS, Inputs, make_inputs, make_small, to_device
 
 pytestmark = pytest.mark.gpu
@@ -126,11 +126,11 @@ def test_dispatch_stage(T, E, k):
     dispatch_parity(idx.numpy(), E, counts.cpu(), offsets.cpu(), perm.cpu(), pos.cpu())
 
 
-def test_dispatch_flags_out_of_range_index():
-    T, E, k = 10, 8, 2
-    idx = torch.tensor([[e % E, (e + 1) % E] for e in range(T)], dtype=torch.int32)
-    idx[3, 1] = E          # out of range
-    idx[7, 0] = -1         # out of range
+@pytest.mark.parametrize("T,E,k", [(10, 8, 2), (900, 64, 8), (64, 512, 8)])
+def test_dispatch_flags_and_skips_out_of_range_index(T, E, k):
+    """Out-of-range expert indices (one CTA path, three-kernel path, E > 256) are flagged
+    MOE_ERR_BAD_INDEX, get pos = -1 and are left out of every segment."""
+    idx = bad_index_routing(T, E, k, seed=T + E)
     h = moe.moe_create(64, E, k, 64, 1)
     ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
     out = [torch.full((n,), -7, dtype=torch.int32, device="cuda")
@@ -138,10 +138,34 @@ def test_dispatch_flags_out_of_range_index():
     moe.moe_dispatch(h, idx.cuda(), *out, ws)
     st, detail = moe.moe_device_status(h, T, ws)
     assert st == moe.MOE_ERR_BAD_INDEX and (detail >> 16) == 2
-    counts = out[0].cpu().numpy()
-    valid = idx.numpy().reshape(-1)
-    valid = valid[(valid >= 0) & (valid < E)]
-    np.testing.assert_array_equal(counts, np.bincount(valid, minlength=E))
+    check_skipped_slots(idx.numpy(), E, *[o.cpu().numpy() for o in out])
+
+
+def test_combine_leaves_out_skipped_slots():
+    """A slot with pos = -1 (an out-of-range index that dispatch skipped) adds nothing: the
+    combine equals the oracle's with that slot's gate set to zero."""
+    T, E, k, S, d = 40, 8, 2, 1, 256
+    idx = bad_index_routing(T, E, k, seed=77)
+    h = moe.moe_create(d, E, k, 64, S)
+    ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
+    out = [torch.empty(n, dtype=torch.int32, device="cuda") for n in (E, E + 1, T * k, T * k)]
+    moe.moe_dispatch(h, idx.cuda(), *out, ws)
+    pos = out[3]
+    g = torch.Generator().manual_seed(5)
+    Y = torch.randn(T * k + S * T, d, generator=g)
+    w = torch.rand(T, k, generator=g)
+    y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(h, Y.cuda(), w.cuda(), pos, y)
+    torch.cuda.synchronize()
+    pos_c = pos.cpu().numpy()
+    skipped = pos_c < 0
+    assert skipped.any()
+    w_ref = w.double().numpy().reshape(-1).copy()
+    w_ref[skipped] = 0.0
+    pos_ref = np.where(skipped, 0, pos_c).astype(np.int32)
+    ref = oracle.combine(Y.double().numpy(), w_ref.reshape(T, k), pos_ref, T, k, S)
+    got = y.float().cpu().numpy()
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6)
 
 
 @pytest.mark.parametrize("tiles", TILINGS)

@@ -14,6 +14,7 @@ import pytest
 import torch
 
 import mixture_experts_layer_47_b200 as moe
+from gpu_helpers import bad_index_routing, check_skipped_slots
 
 pytestmark = pytest.mark.gpu
 
@@ -27,7 +28,10 @@ def _outputs(E, n):
     return [torch.full((m,), -1, dtype=torch.int32, device="cuda") for m in (E, E + 1, n, n)]
 
 
-@pytest.mark.parametrize("T,E,k", [(16, 256, 8), (8192, 256, 8), (777, 64, 4)])
+# E = 512 and E = 1024 take the three-kernel dispatch at few slots, and 1024 is the number
+# of experts the fixed scratch is sized for.
+@pytest.mark.parametrize("T,E,k", [(16, 256, 8), (8192, 256, 8), (777, 64, 4), (64, 1024, 8),
+                                   (512, 512, 8), (2000, 1024, 32)])
 def test_noalloc_dispatch_matches_workspace_dispatch(T, E, k):
     h = moe.moe_create(64, E, k, 64, 1)
     ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
@@ -52,3 +56,15 @@ def test_noalloc_dispatch_rejects_sizes_beyond_its_scratch():
         moe.moe_dispatch_noalloc(h, idx, *out)
     assert e.value.status == moe.MOE_ERR_WORKSPACE
     assert torch.all(out[0] == -1)                   # nothing was enqueued
+
+
+def test_noalloc_dispatch_skips_out_of_range_index():
+    """Out-of-range expert indices: the same skipped slots (pos = -1) and segments as
+    moe_dispatch, although the status word is not readable through this entry point."""
+    T, E, k = 900, 64, 8
+    idx = bad_index_routing(T, E, k, seed=3).cuda()
+    h = moe.moe_create(64, E, k, 64, 1)
+    got = _outputs(E, T * k)
+    moe.moe_dispatch_noalloc(h, idx, *got)
+    torch.cuda.synchronize()
+    check_skipped_slots(idx.cpu().numpy(), E, *[o.cpu().numpy() for o in got])
