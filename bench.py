@@ -1,13 +1,19 @@
 """Benchmark of the B200 MoE FFN layer forward (tokens/s), one JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+                    [--workloads all|none|name,name]
     python bench.py --impl reference ...      # the fp64 CPU oracle arm
 
 A step is one moe_forward over one batch of T tokens: router, dispatch,
-gather, gate/up GEMM + SwiGLU, down GEMM, combine.  With N GPUs (torchrun, one
-process per GPU) every rank runs its own replica of the layer on its own batch
-(the layer has no exchange between token batches): "scaling": "weak", value =
-tokens of all ranks / the slowest rank's time.
+gather, gate/up GEMM + SwiGLU, down GEMM, combine.  The headline is the
+decode workload (T = 16); every other configuration of the layer (batched
+decode, prefill, skewed prefill, and the two FP8-weight decodes) is timed in
+the same run the same way and reported under "workloads" in the same line.
+With N GPUs (one process per GPU; `--gpus N` starts them through torchrun
+when the script is not already running under it) every rank runs its own
+replica of the layer on its own batch (the layer has no exchange between
+token batches): "scaling": "weak", value = tokens of all ranks / the slowest
+rank's time.
 
 Timing: W untimed warm-up steps, then exactly K steps.  Before each step a
 1 GB buffer (eight times L2) is written on the same stream, outside the timed
@@ -219,12 +225,23 @@ def hbm_bound(wl: Workload, work: dict, peaks: dict) -> bool:
 # ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
-def run_ours(args, rank, local, world):
+# Every workload of the layer's configurations is timed in one run: the headline
+# (--workload, decode by default) and, in "workloads", the others.  Each is created,
+# timed and freed before the next (19.4 GB of weights each).
+EXTRA_WORKLOADS = ("batched_decode", "prefill", "skewed_prefill", "decode_fp8",
+                   "batched_decode_fp8")
+
+
+def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds: float,
+                  cpu_tokens: int) -> dict:
+    """This rank's raw timings of one workload on its GPU (nothing reduced over ranks yet).
+
+    Keys: step_ms (K device-timed steps), stage_ms (mean per stage of K evented steps),
+    e2e_ms (K host-timed steps through moe_forward_host), counts (realised expert loads),
+    clocks, kernels_per_step, h2d/d2h bytes per step, fp8, and on rank 0 of a one-GPU run
+    cpu_baseline."""
     import mixture_experts_layer_47_b200 as moe
 
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    wl = ALL_WORKLOADS[args.workload]
     inp = make_inputs(wl, device=device)
     if rank > 0:
         inp.x = rank_batch(wl, rank).to(device)
@@ -260,7 +277,7 @@ def run_ours(args, rank, local, world):
     torch.cuda.synchronize(device)
     st, detail = moe.moe_device_status(h, wl.T, ws, stream)
     if st != moe.MOE_OK:
-        raise RuntimeError(f"device status {st} ({detail:#x}) after warm-up")
+        raise RuntimeError(f"{wl.name}: device status {st} ({detail:#x}) after warm-up")
     counts = moe.workspace_views(h, wl.T, ws)["counts"].cpu().numpy()
 
     # ---- the timed steps (headline): events around each whole forward only ----
@@ -278,13 +295,9 @@ def run_ours(args, rank, local, world):
         torch.cuda.synchronize(device)
     barrier(world)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = max_over_ranks(sum(step_ms), world, device)
-    ms_per_step = total_ms / args.steps
-    tokens_all = wl.T * world * args.steps
-    value = tokens_all / (total_ms / 1e3)
     st, detail = moe.moe_device_status(h, wl.T, ws, stream)
     if st != moe.MOE_OK:
-        raise RuntimeError(f"device status {st} ({detail:#x}) after the timed loop")
+        raise RuntimeError(f"{wl.name}: device status {st} ({detail:#x}) after the timed loop")
 
     # ---- stage times for the roofline: the same steps again with an event at every
     # stage boundary (the events serialise the kernels, so this loop is not the headline) ----
@@ -300,8 +313,6 @@ def run_ours(args, rank, local, world):
         for j in range(moe.MOE_STAGE_EVENTS - 1):
             stage_ms[i, j] = stage_ev[j].elapsed_time(stage_ev[j + 1])
     moe.moe_set_stage_events(h, None)
-    stage_ms_max = np.array([max_over_ranks(float(v), world, device)
-                             for v in stage_ms.mean(0)])
 
     # ---- end to end: pinned host x in, host y out, through moe_forward_host ----
     x_host = inp.x.cpu().pin_memory()
@@ -319,14 +330,25 @@ def run_ours(args, rank, local, world):
         stream.synchronize()
         e2e_ms.append((time.perf_counter() - t0) * 1e3)
     barrier(world)
-    e2e_total = max_over_ranks(sum(e2e_ms), world, device)
-    e2e_value = tokens_all / (e2e_total / 1e3)
 
-    # ---- roofline of the dominant kernel, from the live stage events ----
-    peaks = load_peaks()
-    work = algorithmic_work(wl, counts)
-    names = moe.STAGE_NAMES
-    stage_mean = {n: float(stage_ms_max[j]) for j, n in enumerate(names)}
+    raw = {"step_ms": step_ms, "stage_ms": stage_ms.mean(0).tolist(), "e2e_ms": e2e_ms,
+           "counts": counts, "clocks": clocks.summary(),
+           "kernels_per_step": moe.moe_forward_kernel_count(h, wl.T),
+           "h2d_bytes": int(x_host.numel() * x_host.element_size()),
+           "d2h_bytes": int(y_host.numel() * y_host.element_size()), "fp8": fp8 is not None}
+    if rank == 0 and world == 1 and cpu_seconds > 0:
+        raw["cpu_baseline"] = cpu_baseline(inp, cpu_seconds, fp8, cpu_tokens)
+    del inp, fp8, weights, ws, y, flush, x_host, y_host
+    moe.moe_destroy(h)
+    torch.cuda.synchronize(device)
+    torch.cuda.empty_cache()
+    return raw
+
+
+def roofline(wl: Workload, work: dict, stage_mean: dict, peaks: dict) -> dict:
+    """Roofline of the dominant kernel (the slower of the two expert GEMMs) from its live
+    stage time: algorithmic bytes against the HBM peak below the machine balance,
+    algorithmic FLOPs against the bf16 peak (burst and sustained) above it."""
     dominant = max(("gate_up_gemm", "down_gemm"), key=lambda n: stage_mean[n])
     dom_ms = stage_mean[dominant]
     key = "gate_up" if dominant == "gate_up_gemm" else "down"
@@ -338,13 +360,39 @@ def run_ours(args, rank, local, world):
         achieved = work[key + "_flops"] / (dom_ms / 1e3) / 1e12
         peak = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 4)}
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_sustained": peaks["bf16_tflops_sustained"],
+                "frac_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4)}
     traffic = measured_traffic(dominant, roof["bound"], work["touched_experts"] + wl.S,
                                wl.weights)
     roof.update({"kernel": dominant, "traffic": traffic, "peak_source": peaks["source"],
                  "algorithmic_per_launch": work[key + ("_bytes" if roof["bound"] == "hbm"
                                                        else "_flops")],
                  "launch_ms": round(dom_ms, 4)})
+    return roof
+
+
+def workload_config(wl: Workload, world: int) -> dict:
+    """The "config" of a bench line (the same for both arms)."""
+    return {"workload": wl.name, "T": wl.T, "d_model": wl.d, "n_experts": wl.E,
+            "top_k": wl.k, "d_ff": wl.F, "n_shared": wl.S, "router": wl.router,
+            "zipf_s": wl.zipf_s, "weights": wl.weights, "global_batch": wl.T * world,
+            "parallelism": f"replicas{world}",
+            "l2": "flushed before every step (1 GB write, outside the timed interval)"}
+
+
+def report_workload(wl: Workload, raw: dict, args, world: int, device, stage_names) -> dict:
+    """Reduce one workload's raw timings over ranks (the slowest rank sets every time) and
+    derive tokens/s, the end-to-end number, the roofline and the layer's rates."""
+    total_ms = max_over_ranks(sum(raw["step_ms"]), world, device)
+    ms_per_step = total_ms / args.steps
+    tokens_all = wl.T * world * args.steps
+    stage_mean = {n: max_over_ranks(float(v), world, device)
+                  for n, v in zip(stage_names, raw["stage_ms"])}
+    e2e_total = max_over_ranks(sum(raw["e2e_ms"]), world, device)
+    peaks = load_peaks()
+    counts = raw["counts"]
+    work = algorithmic_work(wl, counts)
     layer = {
         "tflops": round((work["expert_flops"] + work["router_flops"]) / (ms_per_step / 1e3)
                         / 1e12, 2),
@@ -356,32 +404,63 @@ def run_ours(args, rank, local, world):
         "stage_ms": {n: round(v, 4) for n, v in stage_mean.items()},
         "max_expert_rows": int(counts.max()), "min_expert_rows": int(counts.min()),
     }
-
-    out = {
-        "metric": "MoE-layer tokens/s", "value": round(value, 1), "unit": "tokens/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, random-init weights)",
-        "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d, "n_experts": wl.E,
-                   "top_k": wl.k, "d_ff": wl.F, "n_shared": wl.S, "router": wl.router,
-                   "zipf_s": wl.zipf_s, "weights": wl.weights, "global_batch": wl.T * world,
-                   "parallelism": f"replicas{world}",
-                   "l2": "flushed before every step (1 GB write, outside the timed interval)"},
-        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
-                "h2d_bytes_per_step": wl.T * wl.d * 2, "d2h_bytes_per_step": wl.T * wl.d * 2,
-                "api": "moe_forward_host (pinned host x in, host y out)"},
-        "gpu_launches": moe.moe_forward_kernel_count(h, wl.T) * args.steps,
-        "roofline": roof,
+    entry = {
+        "value": round(tokens_all / (total_ms / 1e3), 1), "unit": "tokens/s",
+        "ms_per_step": round(ms_per_step, 4),
+        "config": workload_config(wl, world),
+        "e2e": {"value": round(tokens_all / (e2e_total / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": raw["h2d_bytes"], "d2h_bytes_per_step": raw["d2h_bytes"],
+                "api": ("moe_forward_fp8_host" if raw["fp8"] else "moe_forward_host")
+                       + " (pinned host x in, host y out)"},
+        "gpu_launches": raw["kernels_per_step"] * args.steps,
+        "roofline": roofline(wl, work, stage_mean, peaks),
         "layer": layer,
-        "clocks": clocks.summary(),
+        "clocks": raw["clocks"],
     }
-    if fp8 is not None:
-        out["weights"] = ("fp8: E4M3 codes, one power-of-two scale per 32 K elements of a row, "
-                          "decoded to bf16 in shared memory; bf16 tensor-core MMAs")
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(inp, args.cpu_seconds, fp8)
+    if raw["fp8"]:
+        entry["weights"] = ("fp8: E4M3 codes, one power-of-two scale per 32 K elements of a "
+                            "row, decoded to bf16 on the SMs; bf16 tensor-core MMAs")
+    if "cpu_baseline" in raw:
+        entry["cpu_baseline"] = raw["cpu_baseline"]
+    return entry
+
+
+def run_ours(args, rank, local, world, device=None, timer=time_workload, stage_names=None):
+    """Time the headline workload and the extra ones on every rank; rank 0 prints the line.
+    ``timer`` produces one rank's raw timings of one workload (the GPU work)."""
+    if device is None:
+        device = torch.device("cuda", local)
+        torch.cuda.set_device(device)
+    if stage_names is None:
+        import mixture_experts_layer_47_b200 as moe
+        stage_names = moe.STAGE_NAMES
+    head_wl = ALL_WORKLOADS[args.workload]
+    raw = timer(head_wl, args, rank, world, device, args.cpu_seconds, 16)
+    head = report_workload(head_wl, raw, args, world, device, stage_names)
+    extras = {}
+    names = [] if args.workloads == "none" else \
+        [n for n in (EXTRA_WORKLOADS if args.workloads == "all" else args.workloads.split(","))
+         if n != args.workload]
+    for name in names:
+        wl = ALL_WORKLOADS[name]
+        raw = timer(wl, args, rank, world, device, args.extra_cpu_seconds, 4)
+        extras[name] = report_workload(wl, raw, args, world, device, stage_names)
+    out = {
+        "metric": "MoE-layer tokens/s", "value": head["value"], "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, random-init weights)",
+        "config": head["config"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+        "roofline": head["roofline"], "layer": head["layer"], "clocks": head["clocks"],
+    }
+    for key in ("weights", "cpu_baseline"):
+        if key in head:
+            out[key] = head[key]
+    if extras:
+        out["workloads"] = extras
     if rank == 0:
         print(json.dumps(out), flush=True)
+    return out
 
 
 # ----------------------------------------------------------------------------
@@ -416,15 +495,15 @@ def _oracle_pass(x, Wr, b, W, wl) -> None:
                           W["Ws_up"], W["Ws_down"], None, E=wl.E, F=wl.F, S=wl.S)
 
 
-def _sample_tokens(wl: Workload) -> np.ndarray:
-    n = min(wl.T, 16)
+def _sample_tokens(wl: Workload, n: int = 16) -> np.ndarray:
+    n = min(wl.T, n)
     return np.unique(np.linspace(0, wl.T - 1, n).round().astype(np.int64))
 
 
-def cpu_baseline(inp, seconds: float, fp8=None) -> dict:
+def cpu_baseline(inp, seconds: float, fp8=None, n_tokens: int = 16) -> dict:
     import oracle
     wl = inp.wl
-    tokens = _sample_tokens(wl)
+    tokens = _sample_tokens(wl, n_tokens)
     x, Wr, b, W = _oracle_sample(inp, tokens, fp8)
     passes, t0 = 0, time.perf_counter()
     while True:
@@ -464,9 +543,7 @@ def run_reference(args, rank, local, world):
         "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, random-init weights)",
-        "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d, "n_experts": wl.E,
-                   "top_k": wl.k, "d_ff": wl.F, "n_shared": wl.S, "global_batch": wl.T,
-                   "parallelism": "cpu oracle"},
+        "config": workload_config(wl, world),
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s",
                          "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -475,19 +552,65 @@ def run_reference(args, rank, local, world):
     print(json.dumps(out), flush=True)
 
 
-def main():
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_command(n: int, argv, port: int) -> list:
+    """The torchrun command that starts n ranks of this script with the same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__), *argv]
+
+
+def spawn_ranks(n: int, argv, visible: int) -> int:
+    """--gpus N without a torchrun environment: start N ranks, one per visible GPU.
+    Fails before starting anything when fewer than N GPUs are visible."""
+    if visible < n:
+        raise SystemExit(f"bench.py: --gpus {n} asked for, but {visible} CUDA device(s) are "
+                         "visible")
+    import subprocess
+    # bounded: each rank's process group times out after 120 s; this is the last bound above
+    cmd = ["timeout", "-k", "60", "3600", *launch_command(n, argv, _free_port())]
+    return subprocess.run(cmd).returncode
+
+
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(ALL_WORKLOADS))
+    ap.add_argument("--workloads", default="all",
+                    help="extra workloads timed in the same run: 'all' (every configuration "
+                         "of the layer), 'none', or a comma-separated list")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    args = ap.parse_args()
+    ap.add_argument("--extra-cpu-seconds", type=float, default=3.0)
+    args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("at least 3 warm-up steps are required")
+    if args.workloads not in ("all", "none"):
+        for n in args.workloads.split(","):
+            if n not in ALL_WORKLOADS:
+                ap.error(f"unknown workload {n}")
+    if args.no_cpu_baseline:
+        args.cpu_seconds = args.extra_cpu_seconds = 0.0
+    return args
+
+
+def main():
+    args = parse_args()
     rank, local, world = dist_env()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        visible = torch.cuda.device_count() if torch.cuda.is_available() else 0
+        sys.exit(spawn_ranks(args.gpus, sys.argv[1:], visible))
+    if world > 1 and args.gpus not in (1, world):
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}")
     if args.impl == "reference":
         run_reference(args, rank, local, world)   # rank 0 only; no process group needed
         return

@@ -116,3 +116,23 @@ def check_skipped_slots(idx, E, counts, offsets, perm, pos):
     exp_pos = np.full(flat.size, -1, np.int64)
     exp_pos[order] = np.arange(n)
     np.testing.assert_array_equal(np.asarray(pos), exp_pos)
+
+
+def coverage_tokens(idx, T, n_even):
+    """Tokens for a sampled full-size output check that reach every part of the grouped GEMMs:
+    for every routed expert the last token routed to it (so each group's last, ragged token
+    tile is checked), the first token of the most loaded expert, and n_even evenly spaced
+    tokens.  The shared expert runs on all of them."""
+    idx = np.asarray(idx)
+    chosen = set(np.linspace(0, T - 1, min(n_even, T)).round().astype(np.int64).tolist())
+    flat = idx.reshape(-1)
+    k = idx.shape[1]
+    last = {}
+    for s in range(flat.size - 1, -1, -1):       # last slot per expert, scanning backwards
+        e = int(flat[s])
+        if e not in last:
+            last[e] = s // k
+    chosen.update(last.values())
+    hottest = np.bincount(flat).argmax()
+    chosen.add(int(np.nonzero((idx == hottest).any(axis=1))[0][0]))
+    return np.array(sorted(chosen), dtype=np.int32)

@@ -43,3 +43,71 @@ def test_two_gloo_ranks():
     wl = WORKLOADS["tiny"]
     x0 = make_inputs(wl).x
     assert not torch.equal(bench.rank_batch(wl, 1), x0)   # replicas see different tokens
+
+
+def _fake_timer(wl, args, rank, world, device, cpu_seconds, cpu_tokens):
+    """One rank's raw timings without a GPU: rank r's steps take (r + 1) ms, so the
+    reduction over ranks must report the slower rank."""
+    import bench
+    import numpy as np
+    bench.barrier(world)
+    counts = np.bincount(np.arange(wl.T * wl.k) % wl.E, minlength=wl.E)   # balanced load
+    return {"step_ms": [1.0 + rank] * args.steps, "stage_ms": [0.1 * (rank + 1)] * 6,
+            "e2e_ms": [2.0 + rank] * args.steps, "counts": counts,
+            "clocks": {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0},
+            "kernels_per_step": 8, "h2d_bytes": wl.T * wl.d * 2, "d2h_bytes": wl.T * wl.d * 2,
+            "fp8": wl.weights == "fp8"}
+
+
+def _bench_worker(rank: int, world: int, port: int, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import bench
+    args = bench.parse_args(["--gpus", str(world), "--steps", "4", "--warmup", "3",
+                             "--workloads", "prefill,decode_fp8"])
+    r, local, w = bench.dist_env()
+    bench.init_dist(w, "gloo")
+    line = bench.run_ours(args, r, local, w, device="cpu", timer=_fake_timer,
+                          stage_names=("router", "dispatch", "gather", "gate_up_gemm",
+                                       "down_gemm", "combine"))
+    out[rank] = line
+    torch.distributed.destroy_process_group()
+
+
+def test_bench_line_of_two_gloo_ranks():
+    """bench.py's rank-level path on two CPU ranks (the GPU timing replaced by a fixed one):
+    every rank reduces the same numbers, n_gpus is 2, the step time is the slower rank's,
+    tokens count both ranks, and every extra workload gets its own entry."""
+    world, port = 2, _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.spawn(_bench_worker, args=(world, port, out), nprocs=world, join=True)
+    line = out[0]
+    assert out[1]["value"] == line["value"]
+    assert line["n_gpus"] == 2 and line["scaling"] == "weak"
+    assert line["ms_per_step"] == 2.0                     # rank 1's (slower) steps
+    assert line["value"] == 16 * 2 / 2.0e-3               # decode tokens of both ranks / time
+    assert line["e2e"]["value"] == round(16 * 2 / 3.0e-3, 1)
+    assert line["config"]["parallelism"] == "replicas2"
+    assert sorted(line["workloads"]) == ["decode_fp8", "prefill"]
+    pre = line["workloads"]["prefill"]
+    assert pre["ms_per_step"] == 2.0 and pre["value"] == 8192 * 2 / 2.0e-3
+    assert pre["roofline"]["bound"] == "tensor" and "frac_sustained" in pre["roofline"]
+    assert line["workloads"]["decode_fp8"]["roofline"]["bound"] == "hbm"
+    assert "cpu_baseline" not in line                     # only on a one-GPU run
+
+
+def test_gpus_n_starts_n_ranks_through_torchrun_or_fails_loudly():
+    import subprocess
+    import sys
+    import bench
+    cmd = bench.launch_command(4, ["--gpus", "4", "--steps", "5"], 29511)
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert "--nproc-per-node=4" in cmd and "--master-addr=127.0.0.1" in cmd
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "5"] and cmd[-5].endswith("bench.py")
+    # without enough visible GPUs the script stops before starting anything
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    env.pop("WORLD_SIZE", None)
+    r = subprocess.run([sys.executable, bench.__file__, "--gpus", "2"], capture_output=True,
+                       text=True, env=env, timeout=300)
+    assert r.returncode != 0 and "--gpus 2 asked for" in r.stderr
