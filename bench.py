@@ -552,6 +552,137 @@ def run_reference(args, rank, local, world):
     print(json.dumps(out), flush=True)
 
 
+# ----------------------------------------------------------------------------
+# sharded arm (--parallel tp|ep): one layer over N GPUs, the parts added by collective
+# ----------------------------------------------------------------------------
+def shard_plan(parallel: str, rank: int, world: int, E: int, F: int) -> dict:
+    """What rank holds of the layer.  tp: rows [f0, f1) of every routed and shared expert's
+    W_gate / W_up and the matching columns of W_down (F / world each); ep: routed experts
+    [e0, e0 + n) (E / world each, full d_ff) and, on rank 0 only, the shared experts."""
+    if parallel == "tp":
+        if F % world or (F // world) % 64:
+            raise ValueError(f"d_ff {F} does not split into {world} slices of a multiple of 64")
+        w = F // world
+        return {"e0": 0, "n": E, "f0": rank * w, "f1": (rank + 1) * w, "shared": True}
+    if parallel == "ep":
+        if E % world:
+            raise ValueError(f"{E} experts do not split over {world} ranks")
+        n = E // world
+        return {"e0": rank * n, "n": n, "f0": 0, "f1": F, "shared": rank == 0}
+    raise ValueError(parallel)
+
+
+def shard_weights(inp, plan: dict) -> tuple:
+    """This rank's contiguous copies (or views) of its expert weights."""
+    e0, e1, f0, f1 = plan["e0"], plan["e0"] + plan["n"], plan["f0"], plan["f1"]
+
+    def rows(W, a, b):
+        return W[a:b, f0:f1, :].contiguous()
+
+    def cols(W, a, b):
+        return W[a:b, :, f0:f1].contiguous()
+    routed = (rows(inp.W_gate, e0, e1), rows(inp.W_up, e0, e1), cols(inp.W_down, e0, e1))
+    S = inp.Ws_gate.shape[0]
+    shared = ((rows(inp.Ws_gate, 0, S), rows(inp.Ws_up, 0, S), cols(inp.Ws_down, 0, S))
+              if plan["shared"] else (None, None, None))
+    return routed, shared
+
+
+def gather_parts(part: torch.Tensor, world: int) -> list:
+    """Every rank's fp32 part, in rank order (one all-gather; none at world 1)."""
+    if world == 1:
+        return [part]
+    n = part.shape[0]
+    buf = torch.empty((world * n,) + tuple(part.shape[1:]), dtype=part.dtype, device=part.device)
+    torch.distributed.all_gather_into_tensor(buf, part)
+    return [buf[r * n:(r + 1) * n] for r in range(world)]
+
+
+def run_sharded(args, rank, local, world):
+    """One layer over the ranks: every rank routes all T tokens (x is the same on every
+    rank), computes its shard's fp32 part (moe_forward_partial), the parts are all-gathered
+    (NCCL) and every rank adds them in rank order (moe_reduce_partials): "scaling": "strong"
+    (the same T tokens whatever the number of GPUs)."""
+    import mixture_experts_layer_47_b200 as moe
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = ALL_WORKLOADS[args.workload]
+    if wl.weights != "bf16":
+        raise SystemExit("--parallel tp|ep takes a bf16-weight workload")
+    plan = shard_plan(args.parallel, rank, world, wl.E, wl.F)
+    inp = make_inputs(wl, device=device)      # same seed, so the same x and router everywhere
+    (Wg, Wu, Wd), (Sg, Su, Sd) = shard_weights(inp, plan)
+    inp.W_gate = inp.W_up = inp.W_down = inp.Ws_gate = inp.Ws_up = inp.Ws_down = None
+    torch.cuda.empty_cache()
+    F_local = plan["f1"] - plan["f0"]
+    h = moe.moe_create(wl.d, wl.E, wl.k, F_local, wl.S)
+    ws = torch.empty(moe.moe_workspace_size(h, wl.T), dtype=torch.uint8, device=device)
+    part = torch.empty(wl.T, wl.d, dtype=torch.float32, device=device)
+    y = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=device)
+    flush = torch.empty(1 << 30, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(x_in):
+        moe.moe_forward_partial(h, x_in, inp.W_router, inp.bias, plan["e0"], Wg, Wu, Wd, Sg, Su,
+                                Sd, part, ws, stream)
+        moe.moe_reduce_partials(h, gather_parts(part, world), y, stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step(inp.x)
+    torch.cuda.synchronize(device)
+    st, detail = moe.moe_device_status(h, wl.T, ws, stream)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status {st} ({detail:#x}) after warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(device)
+    with ClockSampler(device) as clocks:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            step(inp.x)
+            ends[i].record(stream)
+            ends[i].synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), world,
+                              device)
+    # end to end: pinned host x in, y out, every step
+    x_host = inp.x.cpu().pin_memory()
+    y_host = torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(inp.x)
+    barrier(world)
+    e2e_ms = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        torch.cuda.synchronize(device)
+        t0 = time.perf_counter()
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        y_host.copy_(y, non_blocking=True)
+        stream.synchronize()
+        e2e_ms.append((time.perf_counter() - t0) * 1e3)
+    barrier(world)
+    e2e_total = max_over_ranks(sum(e2e_ms), world, device)
+    ms = total_ms / args.steps
+    out = {
+        "metric": "MoE-layer tokens/s", "value": round(wl.T * args.steps / (total_ms / 1e3), 1),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, random-init weights)",
+        "config": dict(workload_config(wl, 1), parallelism=f"{args.parallel}{world}"),
+        "e2e": {"value": round(wl.T * args.steps / (e2e_total / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": wl.T * wl.d * 2, "d2h_bytes_per_step": wl.T * wl.d * 2,
+                "api": "moe_forward_partial + all-gather + moe_reduce_partials"},
+        "gpu_launches": (moe.moe_forward_kernel_count(h, wl.T) + 1) * args.steps,
+        "shard": plan, "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return out
+
+
 def _free_port() -> int:
     import socket
     with socket.socket() as s:
@@ -591,6 +722,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--extra-cpu-seconds", type=float, default=3.0)
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "tp", "ep"],
+                    help="replicas: every GPU runs the whole layer on its own tokens (weak "
+                         "scaling); tp / ep: one layer over the GPUs, d_ff slices or expert "
+                         "ranges per GPU, parts added after an all-gather (strong scaling)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("at least 3 warm-up steps are required")
@@ -616,7 +751,10 @@ def main():
         return
     init_dist(world, "nccl")
     try:
-        run_ours(args, rank, local, world)
+        if args.parallel == "replicas":
+            run_ours(args, rank, local, world)
+        else:
+            run_sharded(args, rank, local, world)
     finally:
         if world > 1 and torch.distributed.is_initialized():
             torch.distributed.destroy_process_group()

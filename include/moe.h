@@ -260,6 +260,60 @@ moe_status moe_forward_fp8_host(moe_handle h, const uint16_t *x_host, const floa
                                 void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Sharded layer, for tensor parallelism over d_ff and expert parallelism.
+ * The pages deploy the model on eight GPUs with vLLM's tensor-parallel
+ * recipe (gpuvram.cloud "Tencent Hy4 preview" model card, hardware row: vLLM
+ * TP8 on 8 x H200-class GPUs) and name vLLM's expert parallelism for MoE
+ * (pgsm.cn Hy4 preview hands-on, vLLM deployment section).  Both shard the
+ * expert FFNs so that each GPU computes part of every token's output y, and
+ * y is the sum of the parts:
+ *  - over d_ff: SwiGLU acts on each feature alone, so a GPU holding rows
+ *    [f0, f1) of every W_gate and W_up and the matching columns of every
+ *    W_down computes W_down[:, f0:f1] h[f0:f1] of every expert, and the sum
+ *    over the slices is the layer;
+ *  - over experts: a GPU holding experts [e0, e0 + n) computes the terms of
+ *    the slots routed to them, and the sum over GPUs is the layer.
+ *
+ * moe_forward_partial runs the whole router (every routed expert scores, so
+ * W_router is the full [E][d]) and computes one shard's part of y:
+ *   y_partial[t] = sum_s FFN_s(x_t) + sum_{i : e0 <= idx[t][i] < e0 + n}
+ *                  topk_w[t][i] * FFN_{idx[t][i]}(x_t)
+ * with FFN restricted to this GPU's slice of d_ff, in fp32 and unrounded.
+ * The context gives the slice: create it with d_ff = the slice's width (a
+ * multiple of 64) and E, k, S of the whole layer.
+ * expert_begin, n_local_experts: the routed experts this GPU holds,
+ *   0 <= expert_begin, 1 <= n_local_experts, expert_begin + n_local_experts <= E;
+ * W_gate, W_up: bf16 [n_local_experts][F][d] and W_down: bf16
+ *   [n_local_experts][d][F] for those experts' slices (F = the context's d_ff);
+ * Ws_gate, Ws_up, Ws_down: the shared experts' slices as in moe_forward, or
+ *   all three NULL when this GPU computes no shared-expert term (expert
+ *   parallelism: one GPU adds them; tensor parallelism: every GPU adds its
+ *   slice);
+ * y_partial: fp32 [T][d] (output).
+ * Slots routed to experts outside the local range are skipped like an
+ * out-of-range index in moe_dispatch but are not flagged.  Workspace: as
+ * moe_forward with the same context.  Other arguments as in moe_forward.
+ */
+moe_status moe_forward_partial(moe_handle h, const uint16_t *x, const float *W_router,
+                               const float *bias, int expert_begin, int n_local_experts,
+                               const uint16_t *W_gate, const uint16_t *W_up,
+                               const uint16_t *W_down, const uint16_t *Ws_gate,
+                               const uint16_t *Ws_up, const uint16_t *Ws_down, int T,
+                               float *y_partial, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * The layer output from the shards' parts:
+ *   y[t][j] = bf16( sum_{r < n_partials} partials[r][t][j] )
+ * added in fp32 in the order r = 0, 1, ..., then rounded once.
+ * partials: a HOST array of n_partials (1..16) device pointers, each fp32
+ * [T][d] and 16-byte aligned; they may point to another GPU's memory where
+ * peer access is enabled, and the caller orders their writers before this
+ * call.  y: bf16 [T][d] (output); d is the context's d_model.
+ */
+moe_status moe_reduce_partials(moe_handle h, const float *const *partials, int n_partials, int T,
+                               uint16_t *y, void *stream);
+
+/*
  * Synchronise the stream and read the workspace's device status word, which
  * the last call on this workspace wrote: MOE_OK, MOE_ERR_TIMEOUT or
  * MOE_ERR_BAD_INDEX.  *device_detail receives the raw word (0 if none).

@@ -37,7 +37,8 @@ EXPORTS = ("moe_create", "moe_destroy", "moe_workspace_size", "moe_get_workspace
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_forward",
            "moe_forward_host", "moe_device_status", "moe_set_stage_events",
            "moe_dispatch_noalloc", "moe_selftest_wait_timeout", "moe_forward_kernel_count",
-           "moe_status_string", "moe_expert_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_host")
+           "moe_status_string", "moe_expert_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_host",
+           "moe_forward_partial", "moe_reduce_partials")
 MOE_STAGE_EVENTS = 7
 STAGE_NAMES = ("router", "dispatch", "gather", "gate_up_gemm", "down_gemm", "combine")
 
@@ -97,6 +98,8 @@ def load_library() -> ctypes.CDLL:
                              ctypes.POINTER(Fp8ExpertWeights), I, P, P, Z, P], I),
         "moe_forward_fp8_host": ([P, P, P, P, ctypes.POINTER(Fp8ExpertWeights),
                                   ctypes.POINTER(Fp8ExpertWeights), I, P, P, Z, P], I),
+        "moe_forward_partial": ([P, P, P, P, I, I, P, P, P, P, P, P, I, P, P, Z, P], I),
+        "moe_reduce_partials": ([P, ctypes.POINTER(P), I, I, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -343,6 +346,39 @@ def moe_forward_host(h: Handle, x_host, W_router, bias, W_gate, W_up, W_down, Ws
         *_weights(h, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down), T,
         _ptr(y_host, torch.bfloat16, "y_host", (T, h.d), "cpu"), wp, wn, _stream(stream)),
         "moe_forward_host")
+
+
+def moe_forward_partial(h: Handle, x, W_router, bias, expert_begin: int, W_gate, W_up, W_down,
+                        Ws_gate, Ws_up, Ws_down, y_partial, workspace, stream=None) -> None:
+    """One shard's fp32 part of the layer output (tensor parallelism over d_ff: the handle's
+    d_ff is the slice width; expert parallelism: W_* hold experts expert_begin ... of the
+    layer).  Ws_* are all None when this shard adds no shared-expert term."""
+    T = x.shape[0]
+    n_local = W_gate.shape[0]
+    wp, wn = _ws(workspace)
+    shared = Ws_gate is not None and h.S > 0
+    _check(load_library().moe_forward_partial(
+        h.value, _ptr(x, torch.bfloat16, "x", (T, h.d)),
+        _ptr(W_router, torch.float32, "W_router", (h.E, h.d)),
+        _ptr(bias, torch.float32, "bias", (h.E,)), int(expert_begin), int(n_local),
+        _ptr(W_gate, torch.bfloat16, "W_gate", (n_local, h.F, h.d)),
+        _ptr(W_up, torch.bfloat16, "W_up", (n_local, h.F, h.d)),
+        _ptr(W_down, torch.bfloat16, "W_down", (n_local, h.d, h.F)),
+        _ptr(Ws_gate, torch.bfloat16, "Ws_gate", (h.S, h.F, h.d)) if shared else None,
+        _ptr(Ws_up, torch.bfloat16, "Ws_up", (h.S, h.F, h.d)) if shared else None,
+        _ptr(Ws_down, torch.bfloat16, "Ws_down", (h.S, h.d, h.F)) if shared else None, T,
+        _ptr(y_partial, torch.float32, "y_partial", (T, h.d)), wp, wn, _stream(stream)),
+        "moe_forward_partial")
+
+
+def moe_reduce_partials(h: Handle, partials, y, stream=None) -> None:
+    """y = bf16(sum of the fp32 partial outputs, added in list order)."""
+    T = y.shape[0]
+    arr = (ctypes.c_void_p * len(partials))(
+        *[_ptr(p, torch.float32, f"partials[{i}]", (T, h.d)) for i, p in enumerate(partials)])
+    _check(load_library().moe_reduce_partials(
+        h.value, arr, len(partials), T, _ptr(y, torch.bfloat16, "y", (T, h.d)),
+        _stream(stream)), "moe_reduce_partials")
 
 
 def moe_device_status(h: Handle, T: int, workspace, stream=None) -> tuple:

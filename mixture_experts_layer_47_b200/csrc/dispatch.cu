@@ -16,6 +16,12 @@
 //                     counts make the order ascending in slot index.
 // Up to 4096 slots and 256 experts the three steps run in one CTA
 // (dispatch_single).
+//
+// The experts grouped are the E experts e_base .. e_base + E - 1 of a layer of
+// e_all routed experts (e_base = 0, e_all = E for the whole layer; a range of
+// them when the experts are sharded over GPUs).  A slot routed to an expert
+// outside the range is skipped (pos = -1); an index outside [0, e_all) is
+// skipped too and flagged in the status word.
 #include "common.cuh"
 #include "internal.h"
 
@@ -27,8 +33,15 @@ constexpr int kScatterWarps = 8;
 constexpr int kScanThreads = 1024;
 constexpr int kTileM = 128;   // rows (tokens) per grouped-GEMM tile of the 1-SM tilings
 
+// The local group of a routed expert index g, or -1 when g is outside the
+// local range [e_base, e_base + E).
+__device__ __forceinline__ int local_group(int g, int e_base, int E) {
+  const int e = g - e_base;
+  return (e >= 0 && e < E) ? e : -1;
+}
+
 __global__ void __launch_bounds__(kCountThreads)
-    dispatch_count_kernel(const int32_t* __restrict__ idx, int n, int E,
+    dispatch_count_kernel(const int32_t* __restrict__ idx, int n, int E, int e_base, int e_all,
                           int32_t* __restrict__ blk_hist, int* status) {
   extern __shared__ int32_t hist[];
   pdl_wait();
@@ -39,11 +52,10 @@ __global__ void __launch_bounds__(kCountThreads)
   const int end = min(n, beg + kDispatchChunk);
   bool bad = false;
   for (int s = beg + threadIdx.x; s < end; s += blockDim.x) {
-    const int e = idx[s];
-    if (e >= 0 && e < E)
-      atomicAdd(&hist[e], 1);
-    else
-      bad = true;
+    const int g = idx[s];
+    const int e = local_group(g, e_base, E);
+    if (e >= 0) atomicAdd(&hist[e], 1);
+    if (g < 0 || g >= e_all) bad = true;
   }
   if (bad) report_error(status, kDevBadIndex, kSiteDispatch);
   __syncthreads();
@@ -140,7 +152,7 @@ __global__ void __launch_bounds__(kScanThreads)
 }
 
 __global__ void __launch_bounds__(kScatterWarps * 32)
-    dispatch_scatter_kernel(const int32_t* __restrict__ idx, int n, int E,
+    dispatch_scatter_kernel(const int32_t* __restrict__ idx, int n, int E, int e_base,
                             const int32_t* __restrict__ blk_base, int32_t* __restrict__ perm,
                             int32_t* __restrict__ pos) {
   extern __shared__ int32_t cnt[];  // [kScatterWarps][E]
@@ -156,8 +168,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32)
 
   for (int s0 = beg; s0 < end; s0 += 32) {
     const int s = s0 + lane;
-    int e = (s < end) ? idx[s] : -1;
-    if (e < 0 || e >= E) e = -1;
+    const int e = (s < end) ? local_group(idx[s], e_base, E) : -1;
     const unsigned m = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && lane == __ffs(m) - 1) my[e] += __popc(m);
     __syncwarp();
@@ -174,8 +185,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32)
   __syncthreads();
   for (int s0 = beg; s0 < end; s0 += 32) {
     const int s = s0 + lane;
-    int e = (s < end) ? idx[s] : -1;
-    if (e < 0 || e >= E) e = -1;
+    const int e = (s < end) ? local_group(idx[s], e_base, E) : -1;
     const unsigned m = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(m & ((1u << lane) - 1u));
     const int base = (e >= 0) ? my[e] : 0;
@@ -186,7 +196,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32)
       pos[s] = p;
       if (lane == __ffs(m) - 1) my[e] = base + __popc(m);
     } else if (s < end) {
-      pos[s] = -1;   // a skipped (out-of-range) slot: no position, left out of the combine
+      pos[s] = -1;   // a skipped slot: no position, left out of the combine
     }
     __syncwarp();
   }
@@ -200,8 +210,9 @@ constexpr int kSingleWarps = kScanThreads / 32;
 constexpr int kSingleMaxExperts = 256;
 
 __global__ void __launch_bounds__(kScanThreads)
-    dispatch_single_kernel(const int32_t* __restrict__ idx, int n, int E, int S, int T,
-                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    dispatch_single_kernel(const int32_t* __restrict__ idx, int n, int E, int e_base, int e_all,
+                           int S, int T, int32_t* __restrict__ counts,
+                           int32_t* __restrict__ offsets,
                            int32_t* __restrict__ perm, int32_t* __restrict__ pos,
                            int32_t* __restrict__ sched, int* status) {
   extern __shared__ int32_t cnt[];  // [kSingleWarps][E]
@@ -218,9 +229,9 @@ __global__ void __launch_bounds__(kScanThreads)
   bool bad = false;
   for (int s0 = beg; s0 < end; s0 += 32) {
     const int s = s0 + lane;
-    int e = (s < end) ? idx[s] : -1;
-    if (s < end && (e < 0 || e >= E)) bad = true;
-    if (e < 0 || e >= E) e = -1;
+    const int g = (s < end) ? idx[s] : 0;
+    if (g < 0 || g >= e_all) bad = true;
+    const int e = (s < end) ? local_group(g, e_base, E) : -1;
     const unsigned m = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && lane == __ffs(m) - 1) my[e] += __popc(m);
     __syncwarp();
@@ -250,8 +261,7 @@ __global__ void __launch_bounds__(kScanThreads)
   __syncthreads();
   for (int s0 = beg; s0 < end; s0 += 32) {
     const int s = s0 + lane;
-    int e2 = (s < end) ? idx[s] : -1;
-    if (e2 < 0 || e2 >= E) e2 = -1;
+    const int e2 = (s < end) ? local_group(idx[s], e_base, E) : -1;
     const unsigned m = __match_any_sync(0xffffffffu, e2);
     const int rank = __popc(m & ((1u << lane) - 1u));
     const int base = (e2 >= 0) ? my[e2] : 0;
@@ -262,7 +272,7 @@ __global__ void __launch_bounds__(kScanThreads)
       pos[s] = p;
       if (lane == __ffs(m) - 1) my[e2] = base + __popc(m);
     } else if (s < end) {
-      pos[s] = -1;   // a skipped (out-of-range) slot: no position, left out of the combine
+      pos[s] = -1;   // a skipped slot: no position, left out of the combine
     }
     __syncwarp();
   }
@@ -274,19 +284,21 @@ cudaError_t launch_dispatch(const Ctx& c, const int32_t* topk_idx, int T, int nb
                             int32_t* blk_hist, int32_t* counts, int32_t* offsets, int32_t* perm,
                             int32_t* pos, int32_t* sched, int* status, cudaStream_t st) {
   const int n = T * c.k;
+  const int e_all = c.e_all();
   if (n <= kDispatchChunk && c.E <= kSingleMaxExperts) {
     return launch_pdl(dispatch_single_kernel, dim3(1), dim3(kScanThreads),
-                      kSingleWarps * c.E * sizeof(int32_t), st, 1, topk_idx, n, c.E, c.S, T,
-                      counts, offsets, perm, pos, sched, status);
+                      kSingleWarps * c.E * sizeof(int32_t), st, 1, topk_idx, n, c.E, c.e_base,
+                      e_all, c.S, T, counts, offsets, perm, pos, sched, status);
   }
   cudaError_t err = launch_pdl(dispatch_count_kernel, dim3(nblk), dim3(kCountThreads),
-                               c.E * sizeof(int32_t), st, 1, topk_idx, n, c.E, blk_hist, status);
+                               c.E * sizeof(int32_t), st, 1, topk_idx, n, c.E, c.e_base, e_all,
+                               blk_hist, status);
   if (err != cudaSuccess) return err;
   err = launch_pdl(dispatch_scan_kernel, dim3(1), dim3(kScanThreads), 0, st, 1, blk_hist, nblk,
                    c.E, c.S, T, counts, offsets, sched);
   if (err != cudaSuccess) return err;
   return launch_pdl(dispatch_scatter_kernel, dim3(nblk), dim3(kScatterWarps * 32),
-                    kScatterWarps * c.E * sizeof(int32_t), st, 1, topk_idx, n, c.E,
+                    kScatterWarps * c.E * sizeof(int32_t), st, 1, topk_idx, n, c.E, c.e_base,
                     static_cast<const int32_t*>(blk_hist), perm, pos);
 }
 

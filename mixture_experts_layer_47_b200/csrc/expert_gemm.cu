@@ -470,8 +470,10 @@ GemmTiling gemm_tiling(const Ctx& c, int T) {
     case TilesMode::kSwapPair: return GemmTiling::kSwapPair;
     case TilesMode::kAuto: break;
   }
-  return int64_t(T) * c.k >= int64_t(kSwapPairMinRowsPerExpert) * c.E ? GemmTiling::kSwapPair
-                                                                        : GemmTiling::kSwap;
+  // the average load of a routed expert: the layer's T*k slots over all its experts
+  return int64_t(T) * c.k >= int64_t(kSwapPairMinRowsPerExpert) * c.e_all()
+             ? GemmTiling::kSwapPair
+             : GemmTiling::kSwap;
 }
 
 moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,

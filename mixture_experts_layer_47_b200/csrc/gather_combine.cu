@@ -12,7 +12,11 @@
 //             y[t] = sum_s Y[T*k + s*T + t] + sum_i w[t][i] * Y[pos[t*k + i]]
 //           in fp32, in that fixed order, then rounded once to bf16.  Each
 //           thread owns 8 consecutive features of one token.  Y is fp32 for
-//           moe_combine and bf16 inside moe_forward (half the traffic).
+//           moe_combine and bf16 inside moe_forward (half the traffic).  For a
+//           shard of the layer (moe_forward_partial) the sum is written in fp32
+//           unrounded, and
+//  reduce   adds the shards' fp32 partial outputs in rank order and rounds the
+//           total once to bf16 (moe_reduce_partials).
 #include "common.cuh"
 #include "internal.h"
 
@@ -114,12 +118,27 @@ struct RowBF16 {
   }
 };
 
+// Store 8 fp32 sums: rounded once to bf16, or (partial output) as they are.
+__device__ __forceinline__ void store8(const float (&acc)[8], uint16_t* __restrict__ out) {
+  uint4 o;
+  o.x = pack_bf16x2(acc[0], acc[1]);
+  o.y = pack_bf16x2(acc[2], acc[3]);
+  o.z = pack_bf16x2(acc[4], acc[5]);
+  o.w = pack_bf16x2(acc[6], acc[7]);
+  *reinterpret_cast<uint4*>(out) = o;
+}
+__device__ __forceinline__ void store8(const float (&acc)[8], float* __restrict__ out) {
+  *reinterpret_cast<float4*>(out) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  *reinterpret_cast<float4*>(out + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
 // TY = float (Y in fp32) or uint16_t (Y in bf16); the sums are fp32 either way.
-template <typename TY, typename Row>
+// TOut = uint16_t (y in bf16) or float (a shard's unrounded partial output).
+template <typename TY, typename Row, typename TOut>
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const TY* __restrict__ Y, const float* __restrict__ topk_w,
                    const int32_t* __restrict__ pos, int T, int k, int S, int d,
-                   uint16_t* __restrict__ y) {
+                   TOut* __restrict__ y) {
   pdl_wait();
   pdl_launch_dependents();
   const int t = blockIdx.x;
@@ -141,12 +160,25 @@ __global__ void __launch_bounds__(kCombineThreads)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = fmaf(w, v[j], acc[j]);
   }
-  uint4 out;
-  out.x = pack_bf16x2(acc[0], acc[1]);
-  out.y = pack_bf16x2(acc[2], acc[3]);
-  out.z = pack_bf16x2(acc[4], acc[5]);
-  out.w = pack_bf16x2(acc[6], acc[7]);
-  *reinterpret_cast<uint4*>(y + size_t(t) * d + c) = out;
+  store8(acc, y + size_t(t) * d + c);
+}
+
+// y[i] = bf16(sum_{r < n} part_r[i]) in fp32, r in order; 8 elements per thread per step.
+__global__ void __launch_bounds__(kCombineThreads)
+    reduce_partials_kernel(PartialPtrs parts, int n, size_t n_vec8, uint16_t* __restrict__ y) {
+  pdl_wait();
+  pdl_launch_dependents();
+  for (size_t v = size_t(blockIdx.x) * kCombineThreads + threadIdx.x; v < n_vec8;
+       v += size_t(gridDim.x) * kCombineThreads) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int r = 0; r < n; ++r) {
+      float x[8];
+      RowF32::load8(parts.p[r] + v * 8, x);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] += x[j];
+    }
+    store8(acc, y + v * 8);
+  }
 }
 
 }  // namespace
@@ -181,15 +213,34 @@ cudaError_t launch_gather_tokens(const Ctx& c, const uint16_t* x, const int32_t*
 cudaError_t launch_combine(const Ctx& c, const float* Y, const float* topk_w, const int32_t* pos,
                            int T, uint16_t* y, cudaStream_t st) {
   dim3 grid(T, (c.d / 8 + kCombineThreads - 1) / kCombineThreads);
-  return launch_pdl(combine_kernel<float, RowF32>, grid, dim3(kCombineThreads), 0, st, 1, Y,
-                    topk_w, pos, T, c.k, c.S, c.d, y);
+  return launch_pdl(combine_kernel<float, RowF32, uint16_t>, grid, dim3(kCombineThreads), 0, st,
+                    1, Y, topk_w, pos, T, c.k, c.S, c.d, y);
 }
 
 cudaError_t launch_combine_bf16(const Ctx& c, const uint16_t* Y, const float* topk_w,
                                 const int32_t* pos, int T, uint16_t* y, cudaStream_t st) {
   dim3 grid(T, (c.d / 8 + kCombineThreads - 1) / kCombineThreads);
-  return launch_pdl(combine_kernel<uint16_t, RowBF16>, grid, dim3(kCombineThreads), 0, st, 1, Y,
-                    topk_w, pos, T, c.k, c.S, c.d, y);
+  return launch_pdl(combine_kernel<uint16_t, RowBF16, uint16_t>, grid, dim3(kCombineThreads), 0,
+                    st, 1, Y, topk_w, pos, T, c.k, c.S, c.d, y);
+}
+
+cudaError_t launch_combine_partial(const Ctx& c, const uint16_t* Y, const float* topk_w,
+                                   const int32_t* pos, int T, float* y_partial,
+                                   cudaStream_t st) {
+  dim3 grid(T, (c.d / 8 + kCombineThreads - 1) / kCombineThreads);
+  return launch_pdl(combine_kernel<uint16_t, RowBF16, float>, grid, dim3(kCombineThreads), 0, st,
+                    1, Y, topk_w, pos, T, c.k, c.S, c.d, y_partial);
+}
+
+cudaError_t launch_reduce_partials(const PartialPtrs& parts, int n, size_t elems, uint16_t* y,
+                                   int num_sms, cudaStream_t st) {
+  const size_t n_vec8 = elems / 8;
+  size_t blocks = (n_vec8 + kCombineThreads - 1) / kCombineThreads;
+  const size_t cap = size_t(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return launch_pdl(reduce_partials_kernel, dim3(unsigned(blocks)), dim3(kCombineThreads), 0, st,
+                    1, parts, n, n_vec8, y);
 }
 
 }  // namespace moe

@@ -47,10 +47,16 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 enum class RouterMode { kAuto, kTensorCore, kFfma };
 enum class TilesMode { kAuto, kSingle, kPair, kSwap, kSwapPair };
 
+// A layer shape.  For a shard of the layer (moe_forward_partial) the expert
+// stages see E = the local experts e_base .. e_base + E - 1 of the layer's
+// E_all routed experts and S = the shared experts computed on this GPU.
 struct Ctx {
   int d, E, k, F, S;
   RouterMode router = RouterMode::kAuto;
   TilesMode tiles = TilesMode::kAuto;
+  int e_base = 0;   // first local expert
+  int E_all = 0;    // routed experts of the whole layer (0: E)
+  int e_all() const { return E_all > 0 ? E_all : E; }
 };
 
 // Geometry of the router's split-K partial sums for T tokens.
@@ -116,6 +122,16 @@ cudaError_t launch_combine(const Ctx& c, const float* Y, const float* topk_w, co
                            int T, uint16_t* y, cudaStream_t st);
 cudaError_t launch_combine_bf16(const Ctx& c, const uint16_t* Y, const float* topk_w,
                                 const int32_t* pos, int T, uint16_t* y, cudaStream_t st);
+cudaError_t launch_combine_partial(const Ctx& c, const uint16_t* Y, const float* topk_w,
+                                   const int32_t* pos, int T, float* y_partial, cudaStream_t st);
+
+// Up to this many fp32 partial outputs are added by one moe_reduce_partials call.
+constexpr int kMaxPartials = 16;
+struct PartialPtrs {
+  const float* p[kMaxPartials];
+};
+cudaError_t launch_reduce_partials(const PartialPtrs& parts, int n, size_t elems, uint16_t* y,
+                                   int num_sms, cudaStream_t st);
 
 struct FfnArgs {
   const uint16_t* x;        // [T][d]

@@ -375,10 +375,33 @@ moe_status moe_combine(moe_handle h, const float* Y, const float* topk_w, const 
       launch_combine(h->c, Y, topk_w, pos, T, y, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// A shard of the layer for tensor or expert parallelism: the routed experts
+// e_base .. e_base + n_local - 1 (the caller's weights hold just those), with or
+// without the shared experts, and an unrounded fp32 output.
+struct Shard {
+  int e_base, n_local;
+  bool shared;
+  float* y_partial;
+};
+
+// The shape the expert stages see: the whole layer, or one shard of it.
+static Ctx stage_shape(const Ctx& c, const Shard* sh) {
+  Ctx cl = c;
+  if (sh) {
+    cl.e_base = sh->e_base;
+    cl.E = sh->n_local;
+    cl.E_all = c.E;
+    if (!sh->shared) cl.S = 0;
+  }
+  return cl;
+}
+
 static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W_router,
                                  const float* bias, const Weights& w, int T, uint16_t* y,
-                                 uint8_t* ws, const Layout& L, DeviceInfo* dev, cudaStream_t st) {
+                                 uint8_t* ws, const Layout& L, DeviceInfo* dev, cudaStream_t st,
+                                 const Shard* shard = nullptr) {
   const Ctx& c = h->c;
+  const Ctx cl = stage_shape(c, shard);   // dispatch, gather, GEMMs and combine
   moe_status s;
   int* status = reinterpret_cast<int*>(ws + L.status);
   int32_t* topk_idx = reinterpret_cast<int32_t*>(ws + L.topk_idx);
@@ -402,12 +425,12 @@ static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W
                                      dev->num_sms, topk_idx, topk_w, st))))
     return s;
   if ((s = mark(1))) return s;
-  if ((s = cuda_status(launch_dispatch(c, topk_idx, T, L.nblk,
+  if ((s = cuda_status(launch_dispatch(cl, topk_idx, T, L.nblk,
                                        reinterpret_cast<int32_t*>(ws + L.blk_hist), counts,
                                        offsets, perm, pos, sched, status, st))))
     return s;
   if ((s = mark(2))) return s;
-  if ((s = cuda_status(launch_gather_tokens(c, x, pos, T, x_perm, dev->num_sms, st)))) return s;
+  if ((s = cuda_status(launch_gather_tokens(cl, x, pos, T, x_perm, dev->num_sms, st)))) return s;
   if ((s = mark(3))) return s;
   FfnArgs a;
   a.x = x;
@@ -421,9 +444,13 @@ static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W
   a.T = T;
   a.y_bf16 = true;
   a.after_gate_up = prof ? h->stage_events[4] : nullptr;
-  if ((s = launch_expert_ffn(c, a, *dev, st))) return s;
+  if ((s = launch_expert_ffn(cl, a, *dev, st))) return s;
   if ((s = mark(5))) return s;
-  if ((s = cuda_status(launch_combine_bf16(c, Y, topk_w, pos, T, y, st)))) return s;
+  if (shard)
+    s = cuda_status(launch_combine_partial(cl, Y, topk_w, pos, T, shard->y_partial, st));
+  else
+    s = cuda_status(launch_combine_bf16(c, Y, topk_w, pos, T, y, st));
+  if (s) return s;
   return mark(6);
 }
 
@@ -511,6 +538,56 @@ moe_status moe_forward_fp8_host(moe_handle h, const uint16_t* x_host, const floa
   if (!routed) return MOE_ERR_INVALID_ARG;
   return forward_host_impl(h, x_host, W_router, bias, fp8_weights(routed, shared), T, y_host,
                            workspace, ws_bytes, stream);
+}
+
+moe_status moe_forward_partial(moe_handle h, const uint16_t* x, const float* W_router,
+                               const float* bias, int expert_begin, int n_local_experts,
+                               const uint16_t* W_gate, const uint16_t* W_up,
+                               const uint16_t* W_down, const uint16_t* Ws_gate,
+                               const uint16_t* Ws_up, const uint16_t* Ws_down, int T,
+                               float* y_partial, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_T(h->c, T);
+  if (s) return s;
+  if (expert_begin < 0 || n_local_experts < 1 ||
+      (long long)expert_begin + n_local_experts > h->c.E)
+    return MOE_ERR_INVALID_ARG;
+  const int n_shared_ptrs = (Ws_gate != nullptr) + (Ws_up != nullptr) + (Ws_down != nullptr);
+  if (n_shared_ptrs != 0 && n_shared_ptrs != 3) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  const Shard shard{expert_begin, n_local_experts, n_shared_ptrs == 3 && h->c.S > 0, y_partial};
+  const Ctx cl = stage_shape(h->c, &shard);
+  const Weights w = bf16_weights(W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down);
+  if (!x || !W_router || !y_partial) return MOE_ERR_INVALID_ARG;
+  if ((s = check_weights(cl, w))) return s;
+  if (!aligned16(x) || !aligned16(W_router) || !aligned16(y_partial)) return MOE_ERR_ALIGNMENT;
+  if ((s = check_ws(h, T, workspace, ws_bytes))) return s;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  const Layout L = make_layout(h->c, T, kPlanSms);
+  return forward_device(h, x, W_router, bias, w, T, nullptr, aligned_base(workspace), L, dev,
+                        reinterpret_cast<cudaStream_t>(stream), &shard);
+}
+
+moe_status moe_reduce_partials(moe_handle h, const float* const* partials, int n_partials, int T,
+                               uint16_t* y, void* stream) {
+  if (!h || !partials || !y) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_T(h->c, T);
+  if (s) return s;
+  if (n_partials < 1 || n_partials > kMaxPartials) return MOE_ERR_INVALID_ARG;
+  PartialPtrs parts = {};
+  for (int r = 0; r < n_partials; ++r) {
+    if (!partials[r]) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(partials[r])) return MOE_ERR_ALIGNMENT;
+    parts.p[r] = partials[r];
+  }
+  if (!aligned16(y)) return MOE_ERR_ALIGNMENT;
+  if (T == 0) return MOE_OK;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  return cuda_status(launch_reduce_partials(parts, n_partials, size_t(T) * h->c.d, y,
+                                            dev->num_sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_device_status(moe_handle h, int T, const void* workspace, void* stream,

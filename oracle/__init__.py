@@ -269,6 +269,39 @@ def forward(inp, tokens: Optional[Sequence[int]] = None, idx_override=None,
                 tokens=np.arange(wl.T) if tokens is None else np.asarray(tokens))
 
 
+def shard_output(x, idx, w, W_gate, W_up, W_down, Ws_gate=None, Ws_up=None, Ws_down=None,
+                 expert_begin: int = 0, tokens: Optional[Sequence[int]] = None) -> np.ndarray:
+    """One shard's part of the layer output, fp64, for the sharded deployments the pages name
+    (gpuvram.cloud "Tencent Hy4 preview" model card: vLLM TP8 on eight GPUs; pgsm.cn Hy4
+    preview hands-on, vLLM section: expert parallelism for MoE).  A shard holds routed experts
+    expert_begin .. expert_begin + n - 1 (W_gate, W_up [n, F, d], W_down [n, d, F], possibly
+    only a slice of d_ff: rows of W_gate/W_up and the matching columns of W_down) and, if
+    Ws_* are given, the shared experts (or their slices):
+
+        part[t] = sum_s FFN_s(x_t) + sum over i with expert_begin <= idx[t, i] < expert_begin + n
+                  of w[t, i] * FFN_{idx[t, i]}(x_t)
+
+    summed in that order, each FFN term computed by ``expert_one``.  Summing the parts of
+    all shards gives the layer (SwiGLU acts feature by feature, and every slot's expert lives
+    on exactly one shard)."""
+    xs = _np(x, np.uint16)
+    idx = np.asarray(idx)
+    w = np.asarray(w, np.float64)
+    T, d = xs.shape
+    n = W_gate.shape[0]
+    toks = range(T) if tokens is None else [int(t) for t in tokens]
+    out = np.zeros((len(toks), d), np.float64)
+    for row, t in enumerate(toks):
+        if Ws_gate is not None:
+            for s in range(Ws_gate.shape[0]):
+                out[row] += expert_one(xs[t], Ws_gate[s], Ws_up[s], Ws_down[s])[1]
+        for i in range(idx.shape[1]):
+            e = int(idx[t, i]) - expert_begin
+            if 0 <= e < n:
+                out[row] += w[t, i] * expert_one(xs[t], W_gate[e], W_up[e], W_down[e])[1]
+    return out
+
+
 def renormalised_gates(logits: np.ndarray, idx: np.ndarray) -> np.ndarray:
     """Gate weights for a given expert choice: softmax over all logits, renormalised over idx."""
     logits = np.asarray(logits, np.float64)

@@ -111,3 +111,65 @@ def test_gpus_n_starts_n_ranks_through_torchrun_or_fails_loudly():
     r = subprocess.run([sys.executable, bench.__file__, "--gpus", "2"], capture_output=True,
                        text=True, env=env, timeout=300)
     assert r.returncode != 0 and "--gpus 2 asked for" in r.stderr
+
+
+def _shard_worker(rank: int, world: int, port: int, parallel: str, out):
+    """One rank of a sharded layer on the CPU: its shard of the tiny workload through the
+    oracle, the parts exchanged with the collective bench.py uses, added in rank order."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import numpy as np
+    import bench
+    import oracle
+    from workloads import WORKLOADS, make_inputs
+    bench.init_dist(world, "gloo")
+    wl = WORKLOADS["tiny"]
+    inp = make_inputs(wl)
+    plan = bench.shard_plan(parallel, rank, world, wl.E, wl.F)
+    (Wg, Wu, Wd), (Sg, Su, Sd) = bench.shard_weights(inp, plan)
+    logits = oracle.router_logits(inp.x, inp.W_router, inp.bias)
+    idx, w, _ = oracle.route(logits, wl.k)
+    part = oracle.shard_output(inp.x, idx, w, Wg, Wu, Wd, Sg, Su, Sd, expert_begin=plan["e0"])
+    parts = bench.gather_parts(torch.from_numpy(part), world)
+    total = np.zeros_like(part)
+    for p in parts:                      # rank order, as moe_reduce_partials adds them
+        total += p.numpy()
+    out[rank] = (plan, total)
+    torch.distributed.destroy_process_group()
+
+
+def test_sharded_layer_on_two_gloo_ranks():
+    """tp and ep shard plans over two ranks: the shards cover the layer exactly once, and the
+    all-gathered parts add up on every rank to the oracle's whole layer."""
+    import numpy as np
+    import oracle
+    from workloads import WORKLOADS, make_inputs
+    wl = WORKLOADS["tiny"]
+    full = oracle.forward(make_inputs(wl))["y"]
+    for parallel in ("tp", "ep"):
+        world, port = 2, _free_port()
+        mgr = mp.get_context("spawn").Manager()
+        out = mgr.dict()
+        mp.spawn(_shard_worker, args=(world, port, parallel, out), nprocs=world, join=True)
+        plans = [out[r][0] for r in range(world)]
+        if parallel == "tp":
+            assert [(p["f0"], p["f1"]) for p in plans] == [(0, 64), (64, 128)]
+            assert all(p["shared"] and p["n"] == wl.E for p in plans)
+        else:
+            assert [(p["e0"], p["n"]) for p in plans] == [(0, 8), (8, 8)]
+            assert [p["shared"] for p in plans] == [True, False]
+        for r in range(world):
+            np.testing.assert_allclose(out[r][1], full, rtol=1e-11, atol=1e-12)
+
+
+def test_shard_plans_cover_the_hy4_layer():
+    import bench
+    for world in (1, 2, 4, 8):
+        tp = [bench.shard_plan("tp", r, world, 256, 2048) for r in range(world)]
+        assert tp[0]["f0"] == 0 and tp[-1]["f1"] == 2048
+        assert all(a["f1"] == b["f0"] for a, b in zip(tp, tp[1:]))
+        ep = [bench.shard_plan("ep", r, world, 256, 2048) for r in range(world)]
+        assert sum(p["n"] for p in ep) == 256 and sum(p["shared"] for p in ep) == 1
+    import pytest
+    with pytest.raises(ValueError):
+        bench.shard_plan("tp", 0, 3, 256, 2048)     # 2048 / 3 is not a multiple of 64

@@ -347,3 +347,65 @@ def test_fp8_layer_is_the_bf16_layer_on_decoded_weights():
                  torch_dec(routed.down, routed.down_scale), torch_dec(shared.gate, shared.gate_scale),
                  torch_dec(shared.up, shared.up_scale), torch_dec(shared.down, shared.down_scale))
     np.testing.assert_array_equal(via_oracle, oracle.forward(alt)["y"])
+
+
+def _slice(inp, f0, f1):
+    """Rows f0:f1 of every W_gate / W_up and the matching columns of every W_down."""
+    def rows(W):
+        return W[:, f0:f1, :].contiguous()
+
+    def cols(W):
+        return W[:, :, f0:f1].contiguous()
+    return (rows(inp.W_gate), rows(inp.W_up), cols(inp.W_down),
+            rows(inp.Ws_gate), rows(inp.Ws_up), cols(inp.Ws_down))
+
+
+def test_shard_of_one_expert_slice_is_the_dense_ffn_slice():
+    """E=1, k=1, S=0: one d_ff slice's part is the dense SwiGLU FFN restricted to that slice
+    (torch float64), and the parts of all slices add up to the dense FFN."""
+    inp = make_small(T=11, d=128, E=1, k=1, F=256, S=0, seed=61)
+    idx = np.zeros((11, 1), np.int32)
+    w = np.ones((11, 1))
+    total = np.zeros((11, 128))
+    for f0 in range(0, 256, 64):
+        Wg, Wu, Wd, _, _, _ = _slice(inp, f0, f0 + 64)
+        part = oracle.shard_output(inp.x, idx, w, Wg, Wu, Wd)
+        ref = _dense_swiglu_f64(inp.x, Wg[0], Wu[0], Wd[0]).numpy()
+        np.testing.assert_allclose(part, ref, rtol=1e-12, atol=1e-12)
+        total += part
+    ref = _dense_swiglu_f64(inp.x, inp.W_gate[0], inp.W_up[0], inp.W_down[0]).numpy()
+    np.testing.assert_allclose(total, ref, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("n_slices", [2, 4])
+def test_d_ff_slices_add_up_to_the_layer(n_slices):
+    """Tensor parallelism over d_ff: every shard holds a slice of every routed and shared
+    expert; the parts add up to the whole layer."""
+    inp = make_small(T=20, d=64, E=6, k=2, F=256, S=1, seed=62, bias_scale=0.2)
+    full = oracle.forward(inp)
+    width = 256 // n_slices
+    total = np.zeros_like(full["y"])
+    for r in range(n_slices):
+        Wg, Wu, Wd, Sg, Su, Sd = _slice(inp, r * width, (r + 1) * width)
+        total += oracle.shard_output(inp.x, full["idx"], full["w"], Wg, Wu, Wd, Sg, Su, Sd)
+    np.testing.assert_allclose(total, full["y"], rtol=1e-11, atol=1e-12)
+
+
+def test_expert_ranges_add_up_to_the_layer():
+    """Expert parallelism: shards hold 3, 2 and 3 of 8 routed experts, the first one also the
+    shared expert; the parts add up to the layer, and a part leaves out the other shards'
+    experts (without the shared expert, a shard whose experts no token picked gives 0)."""
+    inp = make_small(T=30, d=64, E=8, k=3, F=64, S=1, seed=63, bias_scale=0.3)
+    full = oracle.forward(inp)
+    total = np.zeros_like(full["y"])
+    for r, (e0, n) in enumerate([(0, 3), (3, 2), (5, 3)]):
+        sl = slice(e0, e0 + n)
+        shared = (inp.Ws_gate, inp.Ws_up, inp.Ws_down) if r == 0 else (None, None, None)
+        total += oracle.shard_output(inp.x, full["idx"], full["w"], inp.W_gate[sl],
+                                     inp.W_up[sl], inp.W_down[sl], *shared, expert_begin=e0)
+    np.testing.assert_allclose(total, full["y"], rtol=1e-11, atol=1e-12)
+    idx = np.full_like(full["idx"], 7)
+    idx[:, 1:] = 6
+    none = oracle.shard_output(inp.x, idx, full["w"], inp.W_gate[:3], inp.W_up[:3],
+                               inp.W_down[:3], expert_begin=0)
+    assert np.all(none == 0.0)
