@@ -181,11 +181,12 @@ def algorithmic_work(wl: Workload, counts: np.ndarray) -> dict:
     rows = wl.T * wl.k + wl.S * wl.T
     gate_up_bytes = int((touched + wl.S) * 2 * wl.F * wl.d * bpe)
     down_bytes = int((touched + wl.S) * wl.F * wl.d * bpe)
+    dense = wl.layer == "dense"     # no router: weights, x and y only
     return {
         "touched_experts": touched,
-        "layer_bytes": w_bytes + wl.E * wl.d * 4 + 2 * wl.T * wl.d * 2,
+        "layer_bytes": w_bytes + (0 if dense else wl.E * wl.d * 4) + 2 * wl.T * wl.d * 2,
         "expert_flops": 6 * wl.d * wl.F * rows,
-        "router_flops": 2 * wl.T * wl.d * wl.E,
+        "router_flops": 0 if dense else 2 * wl.T * wl.d * wl.E,
         "gate_up_bytes": gate_up_bytes,
         "gate_up_flops": 4 * wl.d * wl.F * rows,
         "down_bytes": down_bytes,
@@ -229,7 +230,7 @@ def hbm_bound(wl: Workload, work: dict, peaks: dict) -> bool:
 # (--workload, decode by default) and, in "workloads", the others.  Each is created,
 # timed and freed before the next (19.4 GB of weights each).
 EXTRA_WORKLOADS = ("batched_decode", "prefill", "skewed_prefill", "decode_fp8",
-                   "batched_decode_fp8")
+                   "batched_decode_fp8", "dense_decode", "dense_prefill")
 
 
 def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds: float,
@@ -259,9 +260,20 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
         inp.Ws_gate = inp.Ws_up = inp.Ws_down = None
         torch.cuda.empty_cache()
     weights = (inp.W_gate, inp.W_up, inp.W_down, inp.Ws_gate, inp.Ws_up, inp.Ws_down)
+    dense = wl.layer == "dense"
+    x_stage = torch.empty_like(inp.x) if dense else None
+    y_stage = torch.empty_like(y) if dense else None
 
     def forward(x_arg, y_arg, host=False):
-        if fp8 is not None:
+        if dense:   # the dense FFN layer; host activations go through two copies around it
+            if host:
+                x_stage.copy_(x_arg, non_blocking=True)
+                moe.moe_dense_ffn(h, x_stage, inp.W_gate, inp.W_up, inp.W_down, y_stage, ws,
+                                  stream)
+                y_arg.copy_(y_stage, non_blocking=True)
+            else:
+                moe.moe_dense_ffn(h, x_arg, inp.W_gate, inp.W_up, inp.W_down, y_arg, ws, stream)
+        elif fp8 is not None:
             f = moe.moe_forward_fp8_host if host else moe.moe_forward_fp8
             f(h, x_arg, inp.W_router, inp.bias, fp8[0], fp8[1], y_arg, ws, stream)
         else:
@@ -278,7 +290,8 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
     st, detail = moe.moe_device_status(h, wl.T, ws, stream)
     if st != moe.MOE_OK:
         raise RuntimeError(f"{wl.name}: device status {st} ({detail:#x}) after warm-up")
-    counts = moe.workspace_views(h, wl.T, ws)["counts"].cpu().numpy()
+    counts = (np.array([wl.T]) if dense else
+              moe.workspace_views(h, wl.T, ws)["counts"].cpu().numpy())
 
     # ---- the timed steps (headline): events around each whole forward only ----
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -333,12 +346,12 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
 
     raw = {"step_ms": step_ms, "stage_ms": stage_ms.mean(0).tolist(), "e2e_ms": e2e_ms,
            "counts": counts, "clocks": clocks.summary(),
-           "kernels_per_step": moe.moe_forward_kernel_count(h, wl.T),
+           "kernels_per_step": 3 if dense else moe.moe_forward_kernel_count(h, wl.T),
            "h2d_bytes": int(x_host.numel() * x_host.element_size()),
            "d2h_bytes": int(y_host.numel() * y_host.element_size()), "fp8": fp8 is not None}
     if rank == 0 and world == 1 and cpu_seconds > 0:
         raw["cpu_baseline"] = cpu_baseline(inp, cpu_seconds, fp8, cpu_tokens)
-    del inp, fp8, weights, ws, y, flush, x_host, y_host
+    del inp, fp8, weights, ws, y, flush, x_host, y_host, x_stage, y_stage
     moe.moe_destroy(h)
     torch.cuda.synchronize(device)
     torch.cuda.empty_cache()
@@ -376,8 +389,8 @@ def workload_config(wl: Workload, world: int) -> dict:
     """The "config" of a bench line (the same for both arms)."""
     return {"workload": wl.name, "T": wl.T, "d_model": wl.d, "n_experts": wl.E,
             "top_k": wl.k, "d_ff": wl.F, "n_shared": wl.S, "router": wl.router,
-            "zipf_s": wl.zipf_s, "weights": wl.weights, "global_batch": wl.T * world,
-            "parallelism": f"replicas{world}",
+            "zipf_s": wl.zipf_s, "weights": wl.weights, "layer": wl.layer,
+            "global_batch": wl.T * world, "parallelism": f"replicas{world}",
             "l2": "flushed before every step (1 GB write, outside the timed interval)"}
 
 
@@ -410,8 +423,9 @@ def report_workload(wl: Workload, raw: dict, args, world: int, device, stage_nam
         "config": workload_config(wl, world),
         "e2e": {"value": round(tokens_all / (e2e_total / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": raw["h2d_bytes"], "d2h_bytes_per_step": raw["d2h_bytes"],
-                "api": ("moe_forward_fp8_host" if raw["fp8"] else "moe_forward_host")
-                       + " (pinned host x in, host y out)"},
+                "api": ("moe_dense_ffn between pinned host copies" if wl.layer == "dense" else
+                        ("moe_forward_fp8_host" if raw["fp8"] else "moe_forward_host")
+                        + " (pinned host x in, host y out)")},
         "gpu_launches": raw["kernels_per_step"] * args.steps,
         "roofline": roofline(wl, work, stage_mean, peaks),
         "layer": layer,

@@ -314,6 +314,26 @@ moe_status moe_reduce_partials(moe_handle h, const float *const *partials, int n
                                uint16_t *y, void *stream);
 
 /*
+ * The dense FFN layer.  Of the model's 78 layers the first uses a standard
+ * dense FFN and the other 77 the MoE FFN (ZAKER Hy4 Preview release news,
+ * architecture paragraph); the pages give the dense layer no width.  Reading:
+ * the SwiGLU form of the experts,
+ *   y[t] = W_down (silu(W_gate x[t]) * (W_up x[t]))
+ * which is the MoE layer with one routed expert chosen with weight 1 and no
+ * shared expert, and is computed as that layer without its router, dispatch,
+ * gather and combine (the expert GEMMs read x and write y directly).
+ * h: a context created with n_experts = 1, top_k = 1, n_shared = 0 and the
+ * dense layer's d_model and d_ff (others give MOE_ERR_INVALID_ARG);
+ * x: bf16 [T][d]; W_gate, W_up: bf16 [F][d]; W_down: bf16 [d][F];
+ * y: bf16 [T][d] (output); workspace: moe_workspace_size(h, T) bytes.
+ * The activation is rounded to bf16 before the down projection, and the
+ * output rows once from the fp32 accumulator.
+ */
+moe_status moe_dense_ffn(moe_handle h, const uint16_t *x, const uint16_t *W_gate,
+                         const uint16_t *W_up, const uint16_t *W_down, int T, uint16_t *y,
+                         void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Synchronise the stream and read the workspace's device status word, which
  * the last call on this workspace wrote: MOE_OK, MOE_ERR_TIMEOUT or
  * MOE_ERR_BAD_INDEX.  *device_detail receives the raw word (0 if none).
@@ -323,12 +343,14 @@ moe_status moe_device_status(moe_handle h, int T, const void *workspace, void *s
 
 /*
  * Profiling hook.  With n_events == MOE_STAGE_EVENTS and events non-NULL,
- * every later moe_forward / moe_forward_host call on this context records
- * events[0..6] (cudaEvent_t handles the caller created) on its stream at the
- * stage boundaries: before the router, after the router, after dispatch,
- * after the gather, after the gate/up GEMM, after the down GEMM, after the
- * combine.  The elapsed time between consecutive events is then the device
- * time of one stage.  events == NULL (n_events == 0) switches it off.  The
+ * every later moe_forward / moe_forward_host / moe_dense_ffn call on this
+ * context records events[0..6] (cudaEvent_t handles the caller created) on
+ * its stream at the stage boundaries: before the router, after the router,
+ * after dispatch, after the gather, after the gate/up GEMM, after the down
+ * GEMM, after the combine.  The elapsed time between consecutive events is
+ * then the device time of one stage (moe_dense_ffn: its one-group schedule
+ * counts as dispatch; router, gather and combine are empty).  events == NULL
+ * (n_events == 0) switches it off.  The
  * context keeps the handles only; the caller keeps the events alive.
  */
 #define MOE_STAGE_EVENTS 7

@@ -38,7 +38,7 @@ EXPORTS = ("moe_create", "moe_destroy", "moe_workspace_size", "moe_get_workspace
            "moe_forward_host", "moe_device_status", "moe_set_stage_events",
            "moe_dispatch_noalloc", "moe_selftest_wait_timeout", "moe_forward_kernel_count",
            "moe_status_string", "moe_expert_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_host",
-           "moe_forward_partial", "moe_reduce_partials")
+           "moe_forward_partial", "moe_reduce_partials", "moe_dense_ffn")
 MOE_STAGE_EVENTS = 7
 STAGE_NAMES = ("router", "dispatch", "gather", "gate_up_gemm", "down_gemm", "combine")
 
@@ -100,6 +100,7 @@ def load_library() -> ctypes.CDLL:
                                   ctypes.POINTER(Fp8ExpertWeights), I, P, P, Z, P], I),
         "moe_forward_partial": ([P, P, P, P, I, I, P, P, P, P, P, P, I, P, P, Z, P], I),
         "moe_reduce_partials": ([P, ctypes.POINTER(P), I, I, P, P], I),
+        "moe_dense_ffn": ([P, P, P, P, P, I, P, P, Z, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -369,6 +370,21 @@ def moe_forward_partial(h: Handle, x, W_router, bias, expert_begin: int, W_gate,
         _ptr(Ws_down, torch.bfloat16, "Ws_down", (h.S, h.d, h.F)) if shared else None, T,
         _ptr(y_partial, torch.float32, "y_partial", (T, h.d)), wp, wn, _stream(stream)),
         "moe_forward_partial")
+
+
+def moe_dense_ffn(h: Handle, x, W_gate, W_up, W_down, y, workspace, stream=None) -> None:
+    """The dense SwiGLU FFN layer (h created with n_experts=1, top_k=1, n_shared=0).
+    W_gate, W_up: [F, d] or [1, F, d]; W_down: [d, F] or [1, d, F]."""
+    T = x.shape[0]
+    wp, wn = _ws(workspace)
+    Wg, Wu, Wd = (W.reshape(W.shape[-2:]) if W.dim() == 3 else W
+                  for W in (W_gate, W_up, W_down))
+    _check(load_library().moe_dense_ffn(
+        h.value, _ptr(x, torch.bfloat16, "x", (T, h.d)),
+        _ptr(Wg, torch.bfloat16, "W_gate", (h.F, h.d)),
+        _ptr(Wu, torch.bfloat16, "W_up", (h.F, h.d)),
+        _ptr(Wd, torch.bfloat16, "W_down", (h.d, h.F)), T,
+        _ptr(y, torch.bfloat16, "y", (T, h.d)), wp, wn, _stream(stream)), "moe_dense_ffn")
 
 
 def moe_reduce_partials(h: Handle, partials, y, stream=None) -> None:

@@ -151,6 +151,20 @@ __global__ void __launch_bounds__(kScanThreads)
   write_schedule(c, E, S, T, sched, warp_sums);
 }
 
+// The dense FFN as a one-group layer: offsets = {0, T} and the schedules of
+// one routed group of T rows and no shared group.
+__global__ void __launch_bounds__(kScanThreads)
+    dense_schedule_kernel(int T, int32_t* __restrict__ offsets, int32_t* __restrict__ sched) {
+  __shared__ int warp_sums[32];
+  pdl_wait();
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    offsets[0] = 0;
+    offsets[1] = T;
+  }
+  write_schedule(threadIdx.x == 0 ? T : 0, 1, 0, T, sched, warp_sums);
+}
+
 __global__ void __launch_bounds__(kScatterWarps * 32)
     dispatch_scatter_kernel(const int32_t* __restrict__ idx, int n, int E, int e_base,
                             const int32_t* __restrict__ blk_base, int32_t* __restrict__ perm,
@@ -300,6 +314,11 @@ cudaError_t launch_dispatch(const Ctx& c, const int32_t* topk_idx, int T, int nb
   return launch_pdl(dispatch_scatter_kernel, dim3(nblk), dim3(kScatterWarps * 32),
                     kScatterWarps * c.E * sizeof(int32_t), st, 1, topk_idx, n, c.E, c.e_base,
                     static_cast<const int32_t*>(blk_hist), perm, pos);
+}
+
+cudaError_t launch_dense_schedule(int T, int32_t* offsets, int32_t* sched, cudaStream_t st) {
+  return launch_pdl(dense_schedule_kernel, dim3(1), dim3(kScanThreads), 0, st, 1, T, offsets,
+                    sched);
 }
 
 cudaError_t launch_schedule_from_offsets(const Ctx& c, const int32_t* offsets, int T,

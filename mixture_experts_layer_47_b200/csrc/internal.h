@@ -108,6 +108,8 @@ cudaError_t launch_dispatch(const Ctx& c, const int32_t* topk_idx, int T, int nb
                             int32_t* blk_hist, int32_t* counts, int32_t* offsets, int32_t* perm,
                             int32_t* pos, int32_t* sched, int* status, cudaStream_t st);
 
+cudaError_t launch_dense_schedule(int T, int32_t* offsets, int32_t* sched, cudaStream_t st);
+
 cudaError_t launch_schedule_from_offsets(const Ctx& c, const int32_t* offsets, int T,
                                          int32_t* sched, cudaStream_t st);
 

@@ -570,6 +570,57 @@ moe_status moe_forward_partial(moe_handle h, const uint16_t* x, const float* W_r
                         reinterpret_cast<cudaStream_t>(stream), &shard);
 }
 
+moe_status moe_dense_ffn(moe_handle h, const uint16_t* x, const uint16_t* W_gate,
+                         const uint16_t* W_up, const uint16_t* W_down, int T, uint16_t* y,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  if (c.E != 1 || c.k != 1 || c.S != 0) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_T(c, T);
+  if (s) return s;
+  if (T == 0) return MOE_OK;
+  if (!x || !W_gate || !W_up || !W_down || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down) ||
+      !aligned16(y))
+    return MOE_ERR_ALIGNMENT;
+  if ((s = check_ws(h, T, workspace, ws_bytes))) return s;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Layout L = make_layout(c, T, kPlanSms);
+  uint8_t* ws = aligned_base(workspace);
+  int* status = reinterpret_cast<int*>(ws + L.status);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* sched = reinterpret_cast<int32_t*>(ws + L.sched);
+  const bool prof = h->n_stage_events == MOE_STAGE_EVENTS;
+  auto mark = [&](int i) -> moe_status {
+    return prof ? cuda_status(cudaEventRecord(h->stage_events[i], st)) : MOE_OK;
+  };
+  if ((s = cuda_status(cudaMemsetAsync(status, 0, sizeof(int), st)))) return s;
+  if ((s = mark(0))) return s;
+  if ((s = mark(1))) return s;   // no router
+  if ((s = cuda_status(launch_dense_schedule(T, offsets, sched, st)))) return s;
+  if ((s = mark(2))) return s;   // the one-group schedule in place of dispatch
+  if ((s = mark(3))) return s;   // no gather
+  // One group holding every token in order: the GEMMs read x itself as the group's rows and
+  // the down GEMM's rows are y (weight 1, nothing to combine).
+  FfnArgs a;
+  a.x = x;
+  a.x_perm = x;
+  a.offsets = offsets;
+  a.sched = sched;
+  set_weights(a, bf16_weights(W_gate, W_up, W_down, nullptr, nullptr, nullptr));
+  a.h_act = reinterpret_cast<uint16_t*>(ws + L.h_act);
+  a.Y = y;
+  a.y_bf16 = true;
+  a.status = status;
+  a.T = T;
+  a.after_gate_up = prof ? h->stage_events[4] : nullptr;
+  if ((s = launch_expert_ffn(c, a, *dev, st))) return s;
+  if ((s = mark(5))) return s;
+  return mark(6);   // no combine
+}
+
 moe_status moe_reduce_partials(moe_handle h, const float* const* partials, int n_partials, int T,
                                uint16_t* y, void* stream) {
   if (!h || !partials || !y) return MOE_ERR_INVALID_ARG;

@@ -100,3 +100,17 @@ def test_replica_batches_differ_per_rank_and_are_reproducible(name):
     a1, a2, b1 = bench.rank_batch(wl, 1), bench.rank_batch(wl, 1), bench.rank_batch(wl, 2)
     assert a1.shape == (wl.T, wl.d)
     assert a1.equal(a2) and not a1.equal(b1)
+
+
+def test_algorithmic_work_dense_layer():
+    """The dense first layer: all of its weights, x and y; no router."""
+    wl = WORKLOADS["dense_decode"]
+    w = bench.algorithmic_work(wl, np.array([wl.T]))
+    assert w["touched_experts"] == 1
+    assert w["layer_bytes"] == 3 * 18432 * 6144 * 2 + 2 * 16 * 6144 * 2
+    assert w["router_flops"] == 0
+    assert w["expert_flops"] == 6 * 6144 * 18432 * 16
+    peaks = {"hbm_gbs": 6546.9, "bf16_tflops": 1676.5}
+    assert bench.hbm_bound(wl, w, peaks)
+    pre = WORKLOADS["dense_prefill"]
+    assert not bench.hbm_bound(pre, bench.algorithmic_work(pre, np.array([pre.T])), peaks)

@@ -8,7 +8,7 @@ of tokens the fp64 oracle computes one by one, with only the experts those
 tokens use copied to the host.  At decode the sample is every token; at the
 larger batches it holds, for every routed expert, the last token routed to it
 (the group's last, ragged token tile), the first token of the most loaded
-expert, and 128 evenly spaced tokens.
+expert, and 256 evenly spaced tokens.
 """
 import numpy as np
 import pytest
@@ -40,7 +40,7 @@ def test_full_size_workload(name):
     assert np.isfinite(yg).all()
 
     idx_use = np.where(exempt[:, None], idx_g, idx_o)
-    tokens = coverage_tokens(idx_g, wl.T, 128)
+    tokens = coverage_tokens(idx_g, wl.T, 256)
     assert len(set(idx_g[tokens].reshape(-1).tolist())) == int((c_o > 0).sum())
     w_use = oracle.renormalised_gates(logits, idx_use)
     used = sorted(set(idx_use[tokens].reshape(-1).tolist()))

@@ -49,6 +49,7 @@ class Workload:
     seed: int = 0
     description: str = ""
     weights: str = "bf16"           # "bf16", or "fp8": the same draws stored as e4m3 + block scales
+    layer: str = "moe"              # "moe", or "dense": the dense FFN layer (E = 1, k = 1, S = 0)
 
     @property
     def slots(self) -> int:
@@ -91,6 +92,17 @@ WORKLOADS = {
         "batched_decode_fp8", T=256, d=6144, E=256, k=8, F=2048, S=1, router="uniform", seed=0,
         weights="fp8",
         description="the batched decode workload with FP8 expert weights"),
+    # The model's first layer is a standard dense FFN (ZAKER release news, architecture
+    # paragraph); its width is not printed.  Reading: SwiGLU of width (8 + 1) * 2048 = 18432,
+    # the FFN width one token passes through in an MoE layer (8 routed + 1 shared experts).
+    "dense_decode": Workload(
+        "dense_decode", T=16, d=6144, E=1, k=1, F=18432, S=0, router="normal", seed=0,
+        layer="dense",
+        description="the dense first layer at decode: T=16, d_model=6144, SwiGLU d_ff=18432"),
+    "dense_prefill": Workload(
+        "dense_prefill", T=8192, d=6144, E=1, k=1, F=18432, S=0, router="normal", seed=0,
+        layer="dense",
+        description="the dense first layer at prefill: T=8192, d_model=6144, SwiGLU d_ff=18432"),
 }
 
 # Reduced cases of the same kernels for profiler captures that must stay a few GB on the
