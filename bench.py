@@ -351,11 +351,32 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
            "d2h_bytes": int(y_host.numel() * y_host.element_size()), "fp8": fp8 is not None}
     if rank == 0 and world == 1 and cpu_seconds > 0:
         raw["cpu_baseline"] = cpu_baseline(inp, cpu_seconds, fp8, cpu_tokens)
+    if hbm_bound(wl, algorithmic_work(wl, counts), load_peaks()):
+        raw["read_only_gbs"] = read_only_peak(device)
     del inp, fp8, weights, ws, y, flush, x_host, y_host, x_stage, y_stage
     moe.moe_destroy(h)
     torch.cuda.synchronize(device)
     torch.cuda.empty_cache()
     return raw
+
+
+def read_only_peak(device) -> float:
+    """GB/s of a read-only stream on this GPU, measured live: a sum over a 4 GiB buffer
+    (reads only, a few bytes written), best of 5 with CUDA events.  The HBM-bound kernels
+    here mostly read, so this is shown beside the copy peak (read + write) that
+    MEASURED_PEAKS.json holds."""
+    buf = torch.ones(1 << 30, dtype=torch.int32, device=device)
+    best = 0.0
+    for _ in range(6):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        buf.sum(dtype=torch.int64)
+        b.record()
+        b.synchronize()
+        best = max(best, buf.numel() * 4 / (a.elapsed_time(b) / 1e3) / 1e9)
+    del buf
+    torch.cuda.empty_cache()
+    return round(best, 1)
 
 
 def roofline(wl: Workload, work: dict, stage_mean: dict, peaks: dict) -> dict:
@@ -369,6 +390,9 @@ def roofline(wl: Workload, work: dict, stage_mean: dict, peaks: dict) -> dict:
         achieved = work[key + "_bytes"] / (dom_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4)}
+        if peaks.get("read_only_gbs"):
+            roof["peak_read_only"] = peaks["read_only_gbs"]
+            roof["frac_read_only"] = round(achieved / peaks["read_only_gbs"], 4)
     else:
         achieved = work[key + "_flops"] / (dom_ms / 1e3) / 1e12
         peak = peaks["bf16_tflops"]
@@ -403,7 +427,7 @@ def report_workload(wl: Workload, raw: dict, args, world: int, device, stage_nam
     stage_mean = {n: max_over_ranks(float(v), world, device)
                   for n, v in zip(stage_names, raw["stage_ms"])}
     e2e_total = max_over_ranks(sum(raw["e2e_ms"]), world, device)
-    peaks = load_peaks()
+    peaks = dict(load_peaks(), read_only_gbs=raw.get("read_only_gbs"))
     counts = raw["counts"]
     work = algorithmic_work(wl, counts)
     layer = {
