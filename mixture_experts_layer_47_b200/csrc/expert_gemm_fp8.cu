@@ -34,6 +34,19 @@
 // TMEM columns: [0, 128) two double-buffered accumulators of 2 x 32 columns,
 // [128, 512) six A stages of 2 x 32 columns (64 bf16 K values per row each), one
 // per shared-memory stage, so one MMA commit per K block frees both.
+//
+// 2-SM form (kPair, optional): at decode the token tile is 16 or 32 wide, so an
+// M=128 MMA moves little work per instruction and the MMA issue rate, not HBM,
+// bounds the 1-SM kernel.  A CTA pair halves the instructions per weight byte:
+// each CTA stages and decodes its own 128 rows of each A tile (gate / up rows
+// f0 + 128 r, or W_down rows f0 + 128 r and f0 + 256 + 128 r) into its own
+// TMEM, stages half of the token tile, and the pair's leader issues
+// tcgen05.mma.cta_group::2 (M = 256) with A from both CTAs' TMEM.  The token
+// halves are counted on the leader's barrier; the decoders of both CTAs arrive
+// on the leader's "A tile written" barrier; MMA completions are multicast to
+// both CTAs' barriers; both CTAs' epilogues arrive on the leader's
+// "accumulator free" barrier.  Measured, each 2-SM MMA of this shape costs about
+// twice a 1-SM one, so the pair is not faster; it is kept selectable, not default.
 // Every wait is bounded; on expiry the kernel records the fault, drains its
 // own copies and MMAs, frees TMEM and returns.
 #include <cudaTypedefs.h>
@@ -71,6 +84,7 @@ constexpr uint32_t A_COL0 = 2 * ACC_COLS;   // first A-stage column
 constexpr uint32_t A_STAGE_COLS = 2 * (BK / 2);   // two A tiles, 32 columns each
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_GROUPS = 1024 + 8;
+constexpr int A_TX = 2 * RAW_A + 2 * RAW_S;  // one CTA's codes and scales per stage
 static_assert(STAGE_TX <= STAGE_BYTES, "stage size");
 static_assert(A_COL0 + A_STAGES * A_STAGE_COLS <= TMEM_COLS, "TMEM budget");
 
@@ -93,7 +107,8 @@ struct __align__(64) Fp8Params {
 };
 
 struct SharedStorage {
-  uint64_t full[STAGES];
+  uint64_t full[STAGES];             // 1-SM: the whole stage; pair: this CTA's codes and scales
+  uint64_t bfull[STAGES];            // pair (leader): both CTAs' token rows
   uint64_t empty[STAGES];            // every decoder warp has read its codes and scales
   uint64_t a_full[A_STAGES];         // every decoder warp has written its rows to TMEM
   uint64_t mma_free[STAGES];         // the stage's MMAs are done (token tile and A tile read)
@@ -173,7 +188,7 @@ __device__ void build_schedule(SharedStorage& ss, int E, int S, int T, int lane)
   if (lane == 0) ss.sched[G] = carry;
 }
 
-template <bool kGateUp>
+template <bool kGateUp, bool kPair>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_fp8_kernel(const __grid_constant__ Fp8Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -184,17 +199,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = p.E + p.S;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;   // CTA rank inside the pair
+  const bool leader = rank == 0;
+  const int unit = kPair ? int(blockIdx.x >> 1) : int(blockIdx.x);
+  const int n_units = kPair ? int(gridDim.x >> 1) : int(gridDim.x);
+  constexpr int kCtas = kPair ? 2 : 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&ss.full[s], 1);
+      mbar_init(&ss.bfull[s], 1);
       mbar_init(&ss.empty[s], DEC_WARPS);
-      mbar_init(&ss.a_full[s], DEC_WARPS);
+      mbar_init(&ss.a_full[s], kCtas * DEC_WARPS);
       mbar_init(&ss.mma_free[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&ss.tmem_full[a], 1);
-      mbar_init(&ss.tmem_empty[a], 128);
+      mbar_init(&ss.tmem_empty[a], kCtas * 128);
     }
     mbar_init(&ss.mma_done, 1);
     ss.abort_flag = 0;
@@ -215,8 +236,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(&ss.tmem_base, TMEM_COLS);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(&ss.tmem_base, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&ss.tmem_base, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   pdl_wait();   // the offsets and token operands come from earlier kernels
   pdl_launch_dependents();
@@ -224,11 +250,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   if (warp == 0) build_schedule(ss, p.E, p.S, p.T, lane);
   tc_fence_before();
-  __syncthreads();
+  if (kPair) cluster_sync_all(); else __syncthreads();   // barriers of both CTAs initialised
   tc_fence_after();
   const uint32_t tmem_base = ss.tmem_base;
 
-  constexpr int kFeat = kGateUp ? WM : 2 * WM;   // output features per weight tile
+  // Output features per weight tile: gate/up 128 per CTA, down 256 per CTA (two A tiles).
+  constexpr int kFeat = (kGateUp ? WM : 2 * WM) * kCtas;
+  constexpr int kHalf2 = WM * kCtas;             // down: offset of the second A tile's rows
+  const int rofs = int(rank) * WM;               // this CTA's first row inside an A tile
   const int n_wt = (p.n_out + kFeat - 1) / kFeat;
   const int total = ss.sched[G] * n_wt;
   const int kblocks = p.K / BK;
@@ -242,7 +271,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
-      for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
+      for (int t = unit; t < total && !aborted; t += n_units) {
         if (*abort_flag) { aborted = true; break; }
         const wm::Tile tl = wm::decode_tile<TN, kFeat, kGateUp>(t, n_wt, G, ss.sched, ss.offsets,
                                                                 p.E, p.T, p.k, p.w_rows);
@@ -251,8 +280,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const CUtensorMap* mS0 = tl.shared ? &p.ss0 : &p.ws0;
         const CUtensorMap* mW1 = kGateUp ? (tl.shared ? &p.s1 : &p.w1) : mW0;
         const CUtensorMap* mS1 = kGateUp ? (tl.shared ? &p.ss1 : &p.ws1) : mS0;
-        const int w1_row = kGateUp ? tl.w_row : tl.w_row + WM;   // down: second 128 rows
-        const int f1 = kGateUp ? tl.f0 : tl.f0 + WM;
+        const int w0_row = tl.w_row + rofs;
+        const int w1_row = kGateUp ? w0_row : tl.w_row + kHalf2 + rofs;   // down: second tile
+        const int f0 = tl.f0 + rofs;
+        const int f1 = kGateUp ? f0 : tl.f0 + kHalf2 + rofs;
+        const int t_row = tl.tok_row + (kPair ? int(rank) * (tl.n >> 1) : 0);
         const int srow = tl.g_local * kscales;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&ss.empty[stage], phase ^ 1) ||
@@ -265,11 +297,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint8_t* dst = ring + stage * STAGE_BYTES;
           const int kc = kb * BK;
           const int kbs = srow + kb * (BK / FP8_BLOCK);
-          mbar_arrive_expect_tx(&ss.full[stage], STAGE_TX);
-          tma_load_2d_nohint(dst, mT, &ss.full[stage], kc, tl.tok_row);
-          tma_load_2d_nohint(dst + OFF_A0, mW0, &ss.full[stage], kc, tl.w_row);
+          if (kPair) {
+            // codes and scales for this CTA's decoders; the token half for the leader's MMA
+            mbar_arrive_expect_tx(&ss.full[stage], A_TX);
+            const uint32_t bbar = mapa_shared(smem_u32(&ss.bfull[stage]), 0);
+            if (leader) mbar_arrive_expect_tx(&ss.bfull[stage], 2 * (TN / 2) * BK * 2);
+            tma_load_2d_pair(dst, mT, bbar, kc, t_row);
+          } else {
+            mbar_arrive_expect_tx(&ss.full[stage], STAGE_TX);
+            tma_load_2d_nohint(dst, mT, &ss.full[stage], kc, t_row);
+          }
+          tma_load_2d_nohint(dst + OFF_A0, mW0, &ss.full[stage], kc, w0_row);
           tma_load_2d_nohint(dst + OFF_A1, mW1, &ss.full[stage], kc, w1_row);
-          tma_load_2d_nohint(dst + OFF_S0, mS0, &ss.full[stage], tl.f0, kbs);
+          tma_load_2d_nohint(dst + OFF_S0, mS0, &ss.full[stage], f0, kbs);
           tma_load_2d_nohint(dst + OFF_S1, mS1, &ss.full[stage], f1, kbs);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -279,10 +319,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
+      // Drain: this CTA's own loads must land before it exits (the leader also sees the
+      // token halves on its barrier; the other CTA waits out its halves at the end).
       for (int s = 0; s < STAGES; ++s)
-        if (issued_mask & (1u << s))
+        if (issued_mask & (1u << s)) {
           if (!mbar_wait(&ss.full[s], (issued_parity >> s) & 1u, kDrainTimeoutNs))
             report_error(p.status, kDevTimeout, kSiteDrain);
+          if (kPair && leader &&
+              !mbar_wait(&ss.bfull[s], (issued_parity >> s) & 1u, kDrainTimeoutNs))
+            report_error(p.status, kDevTimeout, kSiteDrain);
+        }
     }
     __syncwarp();
   } else if (warp >= 2 && warp < 2 + DEC_WARPS) {
@@ -294,7 +340,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
     int stage = 0;
     uint32_t phase = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    for (int t = unit; t < total; t += n_units) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) { aborted = true; break; }
       for (int kb = 0; kb < kblocks; ++kb) {
         bool ok = __all_sync(0xffffffffu, mbar_wait(&ss.mma_free[stage], phase ^ 1));
@@ -333,7 +379,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ss.a_full[stage]);
+        if (lane == 0) {
+          if (kPair)
+            mbar_arrive_cluster(mapa_shared(smem_u32(&ss.a_full[stage]), 0));
+          else
+            mbar_arrive(&ss.a_full[stage]);
+        }
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
@@ -344,17 +395,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ---------------- MMA issuer: A from TMEM, token tile from shared memory ----------------
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
+      for (int t = unit; t < total && !aborted; t += n_units) {
         if (*abort_flag) { aborted = true; break; }
         const wm::Tile tl = wm::decode_tile<TN, kFeat, kGateUp>(t, n_wt, G, ss.sched, ss.offsets,
                                                                 p.E, p.T, p.k, p.w_rows);
-        const uint32_t idesc = umma_idesc_bf16_f32(WM, tl.n);
-        if (!mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1)) {
+        const uint32_t idesc = umma_idesc_bf16_f32(WM * kCtas, tl.n);
+        const bool e_ok = kPair ? mbar_wait_cluster(&ss.tmem_empty[acc], acc_phase ^ 1)
+                                : mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1);
+        if (!e_ok) {
           report_error(p.status, kDevTimeout, kSiteMma);
           *abort_flag = 1;
           aborted = true;
@@ -364,7 +417,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t d0 = tmem_base + uint32_t(acc) * ACC_COLS;
         const uint32_t d1 = d0 + uint32_t(TN);
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&ss.a_full[stage], phase) || !mbar_wait(&ss.full[stage], phase)) {
+          const bool a_ok = kPair ? mbar_wait_cluster(&ss.a_full[stage], phase)
+                                  : mbar_wait(&ss.a_full[stage], phase);
+          if (!a_ok || !mbar_wait(kPair ? &ss.bfull[stage] : &ss.full[stage], phase)) {
             report_error(p.status, kDevTimeout, kSiteMma);
             *abort_flag = 1;
             aborted = true;
@@ -377,23 +432,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-            umma_bf16_tmem_a(d0, a0 + uint32_t(8 * kk), b + uint64_t(2 * kk), idesc, accum);
-            umma_bf16_tmem_a(d1, a1 + uint32_t(8 * kk), b + uint64_t(2 * kk), idesc, accum);
+            if (kPair) {
+              umma_bf16_pair_tmem_a(d0, a0 + uint32_t(8 * kk), b + uint64_t(2 * kk), idesc,
+                                    accum);
+              umma_bf16_pair_tmem_a(d1, a1 + uint32_t(8 * kk), b + uint64_t(2 * kk), idesc,
+                                    accum);
+            } else {
+              umma_bf16_tmem_a(d0, a0 + uint32_t(8 * kk), b + uint64_t(2 * kk), idesc, accum);
+              umma_bf16_tmem_a(d1, a1 + uint32_t(8 * kk), b + uint64_t(2 * kk), idesc, accum);
+            }
           }
-          umma_commit(&ss.mma_free[stage]);
+          if (kPair) umma_commit_pair(&ss.mma_free[stage], 0x3); else umma_commit(&ss.mma_free[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (aborted) break;
-        umma_commit(&ss.tmem_full[acc]);
+        if (kPair) umma_commit_pair(&ss.tmem_full[acc], 0x3); else umma_commit(&ss.tmem_full[acc]);
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1;
         }
       }
-      umma_commit(&ss.mma_done);
+      if (kPair) umma_commit_pair(&ss.mma_done, 0x1); else umma_commit(&ss.mma_done);
       if (!mbar_wait(&ss.mma_done, 0, kDrainTimeoutNs))
         report_error(p.status, kDevTimeout, kSiteDrain);
     }
@@ -405,7 +467,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float* stg = ss.stage_t[quarter];
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    for (int t = unit; t < total; t += n_units) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) { aborted = true; break; }  // warp-uniform
       const wm::Tile tl = wm::decode_tile<TN, kFeat, kGateUp>(t, n_wt, G, ss.sched, ss.offsets,
                                                               p.E, p.T, p.k, p.w_rows);
@@ -419,7 +481,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + lane_addr + uint32_t(acc) * ACC_COLS;
       if (kGateUp) {
-        const int col0 = tl.f0 + quarter * 32;      // this warp's 32 features
+        const int col0 = tl.f0 + rofs + quarter * 32;   // this warp's 32 features
         uint32_t g[32], u[32];
         tmem_ld_32cols(tbase, g);
         tmem_ld_32cols(tbase + uint32_t(TN), u);
@@ -435,7 +497,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else {
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
-          const int col0 = tl.f0 + half * WM + quarter * 32;
+          const int col0 = tl.f0 + half * kHalf2 + rofs + quarter * 32;
           uint32_t r[32];
           tmem_ld_32cols(tbase + uint32_t(half * TN), r);
           tmem_ld_wait();
@@ -453,7 +515,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&ss.tmem_empty[acc]);
+      if (kPair)
+        mbar_arrive_cluster(mapa_shared(smem_u32(&ss.tmem_empty[acc]), 0));
+      else
+        mbar_arrive(&ss.tmem_empty[acc]);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -461,28 +526,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
 
+  if (kPair && aborted) {
+    // The token halves of the non-leader CTA are counted on the leader's barrier,
+    // so it cannot observe their completion: give copies in flight time to land.
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 100000ull) {
+    }
+  }
   tc_fence_before();
-  __syncthreads();
+  if (kPair) cluster_sync_all(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (kPair) tmem_dealloc_pair(tmem_base, TMEM_COLS); else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
-template <bool kGateUp>
+template <bool kGateUp, bool kPair>
 cudaError_t launch_fp8(const Fp8Params& fp, int num_sms, cudaStream_t st) {
   static thread_local int attrs_device = -1;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (attrs_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_fp8_kernel<kGateUp>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_fp8_kernel<kGateUp, kPair>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          int(fp8_smem_bytes()));
     if (e != cudaSuccess) return e;
     attrs_device = dev;
   }
-  return launch_pdl(grouped_gemm_fp8_kernel<kGateUp>, dim3(unsigned(num_sms)), dim3(NUM_THREADS),
-                    fp8_smem_bytes(), st, 1, fp);
+  const unsigned grid = kPair ? unsigned(num_sms & ~1) : unsigned(num_sms);
+  return launch_pdl(grouped_gemm_fp8_kernel<kGateUp, kPair>, dim3(grid), dim3(NUM_THREADS),
+                    fp8_smem_bytes(), st, kPair ? 2 : 1, fp);
 }
 
 // Codes [n*rows][K] (box 128 rows x 64 bytes, 64-byte swizzle) and scales
@@ -505,12 +578,17 @@ moe_status launch_expert_ffn_fp8(const Ctx& c, const FfnArgs& a, const DeviceInf
   const int T = a.T;
   const uint64_t nslots = uint64_t(T) * c.k;
   const uint64_t rows = nslots + uint64_t(c.S) * T;
+  // The 1-SM form unless the 2-SM weight-major tiling is asked for (MOE_GEMM_TILES=swap_pair):
+  // measured on B200 at decode, a cta_group::2 MMA with A in TMEM and N = 16 costs about
+  // twice a 1-SM one, so the pair takes twice as long (2.0 against 1.03 ms per layer).
+  const bool pair = c.tiles == TilesMode::kSwapPair;
+  const int tok_box = pair ? TN / 2 : TN;   // token rows one CTA stages per K block
 
   // ---- gate/up + SwiGLU ----
   Fp8Params gp;
   memset(&gp, 0, sizeof gp);
-  bool ok = encode_bf16_2d(&gp.tok_routed, a.x_perm, nslots, c.d, TN) &&
-            encode_bf16_2d(&gp.tok_shared, a.x, uint64_t(T), c.d, TN) &&
+  bool ok = encode_bf16_2d(&gp.tok_routed, a.x_perm, nslots, c.d, tok_box) &&
+            encode_bf16_2d(&gp.tok_shared, a.x, uint64_t(T), c.d, tok_box) &&
             encode_set(&gp.w0, &gp.ws0, R.gate, R.gate_scale, c.E, c.F, c.d) &&
             encode_set(&gp.w1, &gp.ws1, R.up, R.up_scale, c.E, c.F, c.d);
   if (c.S > 0)
@@ -534,13 +612,15 @@ moe_status launch_expert_ffn_fp8(const Ctx& c, const FfnArgs& a, const DeviceInf
   gp.n_out = c.F;
   gp.w_rows = c.F;
   gp.out_rows = int(rows);
-  if (launch_fp8<true>(gp, dev.num_sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((pair ? launch_fp8<true, true>(gp, dev.num_sms, st)
+            : launch_fp8<true, false>(gp, dev.num_sms, st)) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (a.after_gate_up && cudaEventRecord(a.after_gate_up, st) != cudaSuccess) return MOE_ERR_CUDA;
 
   // ---- down projection ----
   Fp8Params dp;
   memset(&dp, 0, sizeof dp);
-  ok = encode_bf16_2d(&dp.tok_routed, a.h_act, rows, c.F, TN) &&
+  ok = encode_bf16_2d(&dp.tok_routed, a.h_act, rows, c.F, tok_box) &&
        encode_set(&dp.w0, &dp.ws0, R.down, R.down_scale, c.E, c.d, c.F);
   if (c.S > 0)
     ok = ok && encode_set(&dp.s0, &dp.ss0, Sh->down, Sh->down_scale, c.S, c.d, c.F);
@@ -566,7 +646,9 @@ moe_status launch_expert_ffn_fp8(const Ctx& c, const FfnArgs& a, const DeviceInf
   dp.n_out = c.d;
   dp.w_rows = c.d;
   dp.out_rows = int(rows);
-  if (launch_fp8<false>(dp, dev.num_sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((pair ? launch_fp8<false, true>(dp, dev.num_sms, st)
+            : launch_fp8<false, false>(dp, dev.num_sms, st)) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

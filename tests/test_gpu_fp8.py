@@ -2,9 +2,10 @@
 
 The reference is the fp64 oracle run on the decoded FP8 weights (oracle.fp8_inputs:
 E4M3 codes decoded from the format definition, times the block scales).  Shapes span
-several tiles and ragged tails: d and d_ff that are not multiples of the 128- or
-256-feature weight tiles, groups that are not multiples of the 16-token N step, more
-than one token tile per group, two shared experts and none.
+several tiles and ragged tails: d and d_ff that are not multiples of the 128- to
+512-feature weight tiles, groups that are not multiples of the 16-token N step, more
+than one token tile per group, two shared experts and none.  Both forms of the FP8
+kernel run: the 1-SM form (the default) and the 2-SM pair (MOE_GEMM_TILES=swap_pair).
 """
 import numpy as np
 import pytest
@@ -53,10 +54,22 @@ def _forward_fp8(dev: Inputs, routed, shared):
     return y.cpu(), {k: v.cpu() for k, v in moe.workspace_views(h, wl.T, ws).items()}
 
 
+FORMS = ["pair", "swap"]
+
+
+def _form(form, monkeypatch):
+    if form == "pair":
+        monkeypatch.setenv("MOE_GEMM_TILES", "swap_pair")
+    else:
+        monkeypatch.delenv("MOE_GEMM_TILES", raising=False)
+
+
+@pytest.mark.parametrize("form", FORMS)
 @pytest.mark.parametrize("shape", FP8_SHAPES, ids=_ids(FP8_SHAPES))
-def test_fp8_expert_ffn_stage(shape):
+def test_fp8_expert_ffn_stage(shape, form, monkeypatch):
     """fp32 Y rows and the bf16 activations against the oracle on the decoded weights,
     given the oracle's dispatch."""
+    _form(form, monkeypatch)
     T, d, E, k, F, S, bs = shape
     inp = make_small(T, d, E, k, F, S, seed=700 + T, bias_scale=bs)
     routed, shared = make_fp8(inp)
@@ -83,8 +96,10 @@ def test_fp8_expert_ffn_stage(shape):
     assert rel_err(Yg, Yr) < Y_REL_TOL, rel_err(Yg, Yr)
 
 
+@pytest.mark.parametrize("form", FORMS)
 @pytest.mark.parametrize("shape", FP8_SHAPES, ids=_ids(FP8_SHAPES))
-def test_fp8_forward_matches_oracle(shape):
+def test_fp8_forward_matches_oracle(shape, form, monkeypatch):
+    _form(form, monkeypatch)
     T, d, E, k, F, S, bs = shape
     inp = make_small(T, d, E, k, F, S, seed=800 + T, bias_scale=bs)
     routed, shared = make_fp8(inp)
@@ -174,8 +189,12 @@ def test_fp8_special_codes_decode_exactly(monkeypatch):
         flat[where] = codes[torch.randint(0, len(SPECIAL_CODES), (4096,), generator=g)]
     routed.gate_scale[0, 0, :8] = 134           # largest scale byte decoded exactly
     ref_inp = decoded_inputs(inp, routed, shared)
-    y8, v8 = _forward_fp8(to_device(inp, "cuda"), routed.to("cuda"), shared.to("cuda"))
+    monkeypatch.setenv("MOE_GEMM_TILES", "swap_pair")
+    y8_pair, v8p = _forward_fp8(to_device(inp, "cuda"), routed.to("cuda"), shared.to("cuda"))
+    ref_p = oracle.forward(ref_inp, idx_override=v8p["topk_idx"].numpy())
+    assert rel_err(y8_pair.float().numpy(), ref_p["y"]) < Y_REL_TOL
     monkeypatch.setenv("MOE_GEMM_TILES", "swap")
+    y8, v8 = _forward_fp8(to_device(inp, "cuda"), routed.to("cuda"), shared.to("cuda"))
     dec = to_device(ref_inp, "cuda")
     h = moe.moe_create(d, E, k, F, S)
     ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
@@ -186,3 +205,22 @@ def test_fp8_special_codes_decode_exactly(monkeypatch):
     assert torch.equal(y8.view(torch.int16), y16.cpu().view(torch.int16))
     ref = oracle.forward(ref_inp, idx_override=v8["topk_idx"].numpy())
     assert rel_err(y8.float().numpy(), ref["y"]) < Y_REL_TOL
+
+
+@pytest.mark.parametrize("name", ["decode_fp8"])
+def test_fp8_pair_and_single_forms_agree_at_full_size(name, monkeypatch):
+    """The 2-SM and 1-SM FP8 kernels on the Hy4 decode workload: the same routing and
+    outputs within the layer's tolerance of each other (the pair's M = 256 MMAs may order
+    the tensor core's partial sums differently from two M = 128 ones)."""
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl, device="cuda")
+    routed, shared = make_fp8(inp)
+    monkeypatch.setenv("MOE_GEMM_TILES", "swap_pair")
+    y_pair, v_pair = _forward_fp8(inp, routed, shared)
+    monkeypatch.delenv("MOE_GEMM_TILES", raising=False)
+    y_one, v_one = _forward_fp8(inp, routed, shared)
+    assert torch.equal(v_pair["topk_idx"], v_one["topk_idx"])
+    err = rel_err(y_pair.float().numpy(), y_one.float().numpy())
+    same = torch.equal(y_pair.view(torch.int16), y_one.view(torch.int16))
+    print(f"{name}: pair vs 1-SM FP8 rel diff {err:.3e}, bit-identical {same}")
+    assert err < Y_REL_TOL
