@@ -346,7 +346,8 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
 
     raw = {"step_ms": step_ms, "stage_ms": stage_ms.mean(0).tolist(), "e2e_ms": e2e_ms,
            "counts": counts, "clocks": clocks.summary(),
-           "kernels_per_step": 3 if dense else moe.moe_forward_kernel_count(h, wl.T),
+           "kernels_per_step": (moe.moe_dense_ffn_kernel_count(h, wl.T) if dense
+                                else moe.moe_forward_kernel_count(h, wl.T)),
            "h2d_bytes": int(x_host.numel() * x_host.element_size()),
            "d2h_bytes": int(y_host.numel() * y_host.element_size()), "fp8": fp8 is not None}
     if rank == 0 and world == 1 and cpu_seconds > 0:
@@ -361,19 +362,19 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
 
 
 def read_only_peak(device) -> float:
-    """GB/s of a read-only stream on this GPU, measured live: a sum over a 4 GiB buffer
-    (reads only, a few bytes written), best of 5 with CUDA events.  The HBM-bound kernels
-    here mostly read, so this is shown beside the copy peak (read + write) that
-    MEASURED_PEAKS.json holds."""
-    buf = torch.ones(1 << 30, dtype=torch.int32, device=device)
+    """GB/s of a read-only stream on this GPU, measured live: a max-reduction over a 4 GiB
+    int64 buffer (reads only, one value written; of the reductions tried on B200 the fastest
+    reader), best of 5 with CUDA events.  The HBM-bound kernels here mostly read, so this is
+    shown beside the copy peak (read + write) that MEASURED_PEAKS.json holds."""
+    buf = torch.ones(1 << 29, dtype=torch.int64, device=device)
     best = 0.0
     for _ in range(6):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        buf.sum(dtype=torch.int64)
+        buf.max()
         b.record()
         b.synchronize()
-        best = max(best, buf.numel() * 4 / (a.elapsed_time(b) / 1e3) / 1e9)
+        best = max(best, buf.numel() * 8 / (a.elapsed_time(b) / 1e3) / 1e9)
     del buf
     torch.cuda.empty_cache()
     return round(best, 1)

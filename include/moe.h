@@ -327,7 +327,10 @@ moe_status moe_reduce_partials(moe_handle h, const float *const *partials, int n
  * x: bf16 [T][d]; W_gate, W_up: bf16 [F][d]; W_down: bf16 [d][F];
  * y: bf16 [T][d] (output); workspace: moe_workspace_size(h, T) bytes.
  * The activation is rounded to bf16 before the down projection, and the
- * output rows once from the fp32 accumulator.
+ * output rows once from the fp32 accumulator.  At up to 128 tokens the down
+ * projection's K is split into ranges whose fp32 parts are added in range
+ * order (deterministic) before that rounding, so that enough SMs stream the
+ * weights.
  */
 moe_status moe_dense_ffn(moe_handle h, const uint16_t *x, const uint16_t *W_gate,
                          const uint16_t *W_up, const uint16_t *W_down, int T, uint16_t *y,
@@ -404,6 +407,11 @@ moe_status moe_selftest_wait_timeout(void *workspace, size_t ws_bytes,
 /* Number of kernels one moe_forward call with T tokens launches (for launch
  * accounting), or -1 for invalid arguments. */
 int moe_forward_kernel_count(moe_handle h, int T);
+
+/* Number of kernels one moe_dense_ffn call with T tokens launches, or -1 for
+ * invalid arguments (including a context that is not the dense E=1, k=1, S=0
+ * layer). */
+int moe_dense_ffn_kernel_count(moe_handle h, int T);
 
 /* Static text for a status code. */
 const char *moe_status_string(moe_status s);

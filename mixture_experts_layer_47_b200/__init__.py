@@ -38,7 +38,8 @@ EXPORTS = ("moe_create", "moe_destroy", "moe_workspace_size", "moe_get_workspace
            "moe_forward_host", "moe_device_status", "moe_set_stage_events",
            "moe_dispatch_noalloc", "moe_selftest_wait_timeout", "moe_forward_kernel_count",
            "moe_status_string", "moe_expert_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_host",
-           "moe_forward_partial", "moe_reduce_partials", "moe_dense_ffn")
+           "moe_forward_partial", "moe_reduce_partials", "moe_dense_ffn",
+           "moe_dense_ffn_kernel_count")
 MOE_STAGE_EVENTS = 7
 STAGE_NAMES = ("router", "dispatch", "gather", "gate_up_gemm", "down_gemm", "combine")
 
@@ -101,6 +102,7 @@ def load_library() -> ctypes.CDLL:
         "moe_forward_partial": ([P, P, P, P, I, I, P, P, P, P, P, P, I, P, P, Z, P], I),
         "moe_reduce_partials": ([P, ctypes.POINTER(P), I, I, P, P], I),
         "moe_dense_ffn": ([P, P, P, P, P, I, P, P, Z, P], I),
+        "moe_dense_ffn_kernel_count": ([P, I], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -426,6 +428,10 @@ def moe_selftest_wait_timeout(workspace, timeout_ns: int, stream=None) -> None:
 
 def moe_forward_kernel_count(h: Handle, T: int) -> int:
     return int(load_library().moe_forward_kernel_count(h.value, int(T)))
+
+
+def moe_dense_ffn_kernel_count(h: Handle, T: int) -> int:
+    return int(load_library().moe_dense_ffn_kernel_count(h.value, int(T)))
 
 
 def moe_status_string(status: int) -> str:

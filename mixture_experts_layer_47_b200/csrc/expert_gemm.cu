@@ -476,6 +476,23 @@ GemmTiling gemm_tiling(const Ctx& c, int T) {
              : GemmTiling::kSwap;
 }
 
+// The dense layer (E = 1, k = 1, S = 0) at up to 128 tokens runs the 1-SM weight-major
+// GEMMs, whose down projection has d / 256 output tiles (24 at d = 6144) for the SMs'
+// 148: split its K so that about 148 CTAs stream the weights (planned for a 148-SM part,
+// so the summation order is the same on every device).
+int dense_down_ksplit(const Ctx& c, int T) {
+  if (c.E != 1 || c.k != 1 || c.S != 0 || T < 1 || T > kDenseSplitMaxT) return 1;
+  if (gemm_tiling(c, T) != GemmTiling::kSwap) return 1;
+  const int tiles = (c.d + 255) / 256;
+  int ks = 148 / tiles;
+  ks = ks < 1 ? 1 : (ks > kDenseSplitMax ? kDenseSplitMax : ks);
+  const int kblocks = c.F / 64;
+  if (ks > kblocks) ks = kblocks;
+  // every range non-empty: ranges are ceil(kblocks / ks) blocks long, the last the rest
+  while (ks > 1 && (ks - 1) * ((kblocks + ks - 1) / ks) >= kblocks) --ks;
+  return ks;
+}
+
 moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                              cudaStream_t st) {
   if (!tensor_map_encoder()) return MOE_ERR_CUDA;

@@ -94,6 +94,8 @@ struct __align__(64) SwapParams {
   int n_out;               // output features per group (F or d)
   int w_rows;              // weight rows per expert in the w maps (F or d)
   int out_rows;            // rows of the output buffer (T*k + S*T)
+  int ksplit;              // down, 1-SM only: K ranges per output tile (1 = no split)
+  float* part;             // with ksplit > 1: fp32 parts [ksplit][out_rows][n_out]
 };
 
 struct SharedStorage {
@@ -178,8 +180,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = ss.tmem_base;
 
   const int n_wt = (p.n_out + C::FEAT - 1) / C::FEAT;
-  const int total = ss.sched[G] * n_wt;
+  // Split over K (down projection of the 1-SM tiling only): tile t covers output tile
+  // t / ksplit and K blocks [kper * (t % ksplit), ...); each writes an fp32 part.
+  const int ksplit = (!kGateUp && !kPair && p.ksplit > 1) ? p.ksplit : 1;
+  const int total = ss.sched[G] * n_wt * ksplit;
   const int kblocks = p.K / BK;
+  const int kper = (kblocks + ksplit - 1) / ksplit;
   volatile int* abort_flag = &ss.abort_flag;
   bool aborted = false;
 
@@ -191,8 +197,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t issued_mask = 0, issued_parity = 0;
       for (int t = unit; t < total && !aborted; t += n_units) {
         if (*abort_flag) { aborted = true; break; }
+        const int ks = t % ksplit;
         const wm::Tile tl = wm::decode_tile<C::TN, C::FEAT, kGateUp>(
-            t, n_wt, G, ss.sched, ss.offsets, p.E, p.T, p.k, p.w_rows);
+            t / ksplit, n_wt, G, ss.sched, ss.offsets, p.E, p.T, p.k, p.w_rows);
+        const int kb0 = ks * kper, kb1 = min(kblocks, kb0 + kper);
         const CUtensorMap* mT = tl.shared ? &p.tok_shared : &p.tok_routed;
         const CUtensorMap* mW0 = tl.shared ? &p.s0 : &p.w0;
         const CUtensorMap* mW1 = kGateUp ? (tl.shared ? &p.s1 : &p.w1) : mW0;
@@ -200,7 +208,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int w0_row = tl.w_row + (kPair ? int(rank) * WM : 0);
         const int w1_row = kGateUp ? w0_row : w0_row + WM;   // 1-SM down: second 128 rows
         const int t_row = tl.tok_row + (kPair ? int(rank) * (tl.n >> 1) : 0);
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&ss.empty[stage], phase ^ 1)) {
             report_error(p.status, kDevTimeout, kSiteProducer);
             *abort_flag = 1;
@@ -249,8 +257,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t acc_phase = 0;
       for (int t = unit; t < total && !aborted; t += n_units) {
         if (*abort_flag) { aborted = true; break; }
+        const int ks = t % ksplit;
         const wm::Tile tl = wm::decode_tile<C::TN, C::FEAT, kGateUp>(
-            t, n_wt, G, ss.sched, ss.offsets, p.E, p.T, p.k, p.w_rows);
+            t / ksplit, n_wt, G, ss.sched, ss.offsets, p.E, p.T, p.k, p.w_rows);
+        const int kb0 = ks * kper, kb1 = min(kblocks, kb0 + kper);
         const uint32_t idesc = umma_idesc_bf16_f32(C::MMA_M, tl.n);
         if (!mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1)) {
           report_error(p.status, kDevTimeout, kSiteMma);
@@ -261,7 +271,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d0 = tmem_base + uint32_t(acc * C::ACC_STRIDE);
         const uint32_t d1 = d0 + uint32_t(C::SECOND);
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&ss.full[stage], phase)) {
             report_error(p.status, kDevTimeout, kSiteMma);
             *abort_flag = 1;
@@ -275,7 +285,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t b = umma_desc_sw128_kmajor(base + C::NUM_A * W_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            const uint32_t accum = (kb != kb0 || kk != 0) ? 1u : 0u;
             if (kPair) {
               umma_bf16_pair(d0, a0 + uint64_t(2 * kk), b + uint64_t(2 * kk), idesc, accum);
               if (C::NUM_A == 2)
@@ -315,8 +325,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t acc_phase = 0;
     for (int t = unit; t < total; t += n_units) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) { aborted = true; break; }  // warp-uniform
+      const int ks = t % ksplit;
       const wm::Tile tl = wm::decode_tile<C::TN, C::FEAT, kGateUp>(
-            t, n_wt, G, ss.sched, ss.offsets, p.E, p.T, p.k, p.w_rows);
+            t / ksplit, n_wt, G, ss.sched, ss.offsets, p.E, p.T, p.k, p.w_rows);
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&ss.tmem_full[acc], acc_phase));
       if (!ok) {
         if (lane == 0) report_error(p.status, kDevTimeout, kSiteEpilogue);
@@ -409,7 +420,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
             if (c + 64 < tl.n) tmem_ld_32cols(hbase + uint32_t(c + 64), r);
             if (cols_ok) {
-              if (p.out_bf16)
+              if (ksplit > 1)   // this K range's fp32 part; the parts are added afterwards
+                wm::store_block_transposed<false>(
+                    stg, v, lane, p.part + size_t(ks) * p.out_rows * p.n_out, p.n_out,
+                    tl.out_row + c, tl.cnt - c, col0, p.out_rows);
+              else if (p.out_bf16)
                 wm::store_block_transposed<true>(stg, v, lane, p.out, p.n_out, tl.out_row + c,
                                              tl.cnt - c, col0, p.out_rows);
               else
@@ -533,9 +548,19 @@ moe_status launch_expert_ffn_swap(const Ctx& c, const FfnArgs& a, const DeviceIn
   dp.n_out = c.d;
   dp.w_rows = c.d;
   dp.out_rows = int(rows);
+  const bool split = !pair && a.down_ksplit > 1 && a.down_part && a.y_bf16;
+  dp.ksplit = split ? a.down_ksplit : 1;
+  dp.part = split ? a.down_part : nullptr;
   err = pair ? launch_swap<false, true>(dp, dev.num_sms, st)
              : launch_swap<false, false>(dp, dev.num_sms, st);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
+  if (split) {   // y = bf16(sum of the K ranges' parts, in range order)
+    PartialPtrs parts = {};
+    for (int j = 0; j < dp.ksplit; ++j) parts.p[j] = a.down_part + size_t(j) * rows * c.d;
+    if (launch_reduce_partials(parts, dp.ksplit, size_t(rows) * c.d,
+                               static_cast<uint16_t*>(a.Y), dev.num_sms, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   return MOE_OK;
 }
 

@@ -71,7 +71,7 @@ RouterPlan router_plan(const Ctx& c, int T, int num_sms);
 // Workspace carve-up for T tokens (offsets from the 1024-aligned base).
 struct Layout {
   size_t status, part, wparts, topk_idx, topk_w, counts, offsets, perm, pos, blk_hist, sched,
-      x_perm, h_act, y_rows, x_stage, y_stage, end;
+      x_perm, h_act, y_rows, x_stage, y_stage, down_part, end;
   int nblk;           // dispatch blocks
   RouterPlan rplan;
 };
@@ -103,6 +103,11 @@ enum class GemmTiling { kSingle, kPair, kSwap, kSwapPair };
 // Average routed rows per expert from which the 2-SM weight-major kernel is used.
 constexpr int kSwapPairMinRowsPerExpert = 96;
 GemmTiling gemm_tiling(const Ctx& c, int T);
+// K ranges the dense layer's down projection is split into at small batches (1 = none): its
+// d / 256 output tiles alone would leave most SMs idle.
+constexpr int kDenseSplitMaxT = 128;
+constexpr int kDenseSplitMax = 8;
+int dense_down_ksplit(const Ctx& c, int T);
 
 cudaError_t launch_dispatch(const Ctx& c, const int32_t* topk_idx, int T, int nblk,
                             int32_t* blk_hist, int32_t* counts, int32_t* offsets, int32_t* perm,
@@ -151,6 +156,10 @@ struct FfnArgs {
   // (nullptr when S == 0); both nullptr for bf16 weights.
   const moe_fp8_expert_weights* fp8_routed = nullptr;
   const moe_fp8_expert_weights* fp8_shared = nullptr;
+  // Down projection split over K (1-SM weight-major tiling, bf16 Y): fp32 parts
+  // [down_ksplit][rows][d] in the workspace, added in order into Y.
+  int down_ksplit = 1;
+  float* down_part = nullptr;
 };
 moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                              cudaStream_t st);

@@ -91,6 +91,8 @@ Layout make_layout(const Ctx& c, int T, int num_sms) {
   L.y_rows = take(rows * c.d * sizeof(uint16_t));  // bf16 rows of moe_forward
   L.x_stage = take(size_t(T) * c.d * sizeof(uint16_t));
   L.y_stage = take(size_t(T) * c.d * sizeof(uint16_t));
+  L.down_part = take(size_t(dense_down_ksplit(c, T) > 1 ? dense_down_ksplit(c, T) : 0) * T * c.d *
+                     sizeof(float));
   L.end = off;
   return L;
 }
@@ -616,6 +618,8 @@ moe_status moe_dense_ffn(moe_handle h, const uint16_t* x, const uint16_t* W_gate
   a.status = status;
   a.T = T;
   a.after_gate_up = prof ? h->stage_events[4] : nullptr;
+  a.down_ksplit = dense_down_ksplit(c, T);
+  a.down_part = reinterpret_cast<float*>(ws + L.down_part);
   if ((s = launch_expert_ffn(c, a, *dev, st))) return s;
   if ((s = mark(5))) return s;
   return mark(6);   // no combine
@@ -670,6 +674,14 @@ int moe_forward_kernel_count(moe_handle h, int T) {
   const int router = rp.tc ? 3 : 2;  // [weight split +] score GEMM + top-k
   const int dispatch = (int64_t(T) * c.k <= kDispatchChunk && c.E <= 256) ? 1 : 3;
   return router + dispatch + 1 /*gather*/ + 2 /*GEMMs*/ + 1 /*combine*/;
+}
+
+int moe_dense_ffn_kernel_count(moe_handle h, int T) {
+  if (!h || T < 0 || check_T(h->c, T) != MOE_OK) return -1;
+  const Ctx& c = h->c;
+  if (c.E != 1 || c.k != 1 || c.S != 0) return -1;
+  if (T == 0) return 0;
+  return 3 + (dense_down_ksplit(c, T) > 1 ? 1 : 0);   // schedule, GEMMs [, K-range sum]
 }
 
 moe_status moe_set_stage_events(moe_handle h, void* const* events, int n_events) {

@@ -3,8 +3,10 @@
 The dense layer is the MoE layer with one routed expert chosen with weight 1 and no shared
 expert, which the oracle computes as such (pinned against a float64 dense SwiGLU in
 tests/test_oracle.py).  moe_dense_ffn runs the same expert GEMM kernels without router,
-dispatch, gather and combine, so its output must also equal moe_forward's on that one-expert
-layer bit for bit (the combine of one weight-1 row reproduces the row's bf16 value).
+dispatch, gather and combine, so where it does not split the down projection over K its
+output equals moe_forward's on that one-expert layer bit for bit (the combine of one
+weight-1 row reproduces the row's bf16 value); with the split (up to 128 tokens, 1-SM
+tiling) the fp32 parts are added before the one rounding, so the two agree within the bar.
 """
 import numpy as np
 import pytest
@@ -17,7 +19,8 @@ from workloads import WORKLOADS, make_inputs, make_small, to_device
 
 pytestmark = pytest.mark.gpu
 
-SHAPES = [(1, 64, 64), (64, 256, 640), (300, 192, 384), (1000, 128, 192), (517, 256, 2304)]
+SHAPES = [(1, 64, 64), (64, 256, 640), (40, 128, 576), (300, 192, 384), (1000, 128, 192),
+          (517, 256, 2304)]
 
 
 def _dense(inp, T):
@@ -46,7 +49,10 @@ def test_dense_ffn_matches_oracle_and_the_one_expert_layer(shape, tiles, monkeyp
     moe.moe_forward(h, dev.x, dev.W_router, None, dev.W_gate, dev.W_up, dev.W_down, None, None,
                     None, y2, ws)
     torch.cuda.synchronize()
-    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    if moe.moe_dense_ffn_kernel_count(h, T) == 3:      # no split over K
+        assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    else:
+        assert rel_err(y.float().cpu().numpy(), y2.float().cpu().numpy()) < Y_REL_TOL
 
 
 def test_dense_ffn_rejects_a_moe_context():
