@@ -68,10 +68,13 @@ typedef int moe_status;
  * 1 <= E <= 1024; 1 <= k <= min(E, 32); 0 <= S <= 8.  Shapes outside it give
  * MOE_ERR_UNSUPPORTED, impossible ones MOE_ERR_INVALID_ARG.  No CUDA call is
  * made here; the device is checked (sm_100 required) at the first launch.
- * Two tuning overrides are read from the environment here, once, and fixed for
- * the context's lifetime: MOE_ROUTER=tc|ffma (router path) and
- * MOE_GEMM_TILES=single|pair|swap|swap_pair (expert GEMM tiling); all choices
- * compute the same result.
+ * Three tuning overrides are read from the environment here, once, and fixed
+ * for the context's lifetime: MOE_ROUTER=tc|ffma (router path),
+ * MOE_GEMM_TILES=single|pair|swap|swap_pair (expert GEMM tiling) and
+ * MOE_FUSED_COMBINE=1 (moe_forward merges the experts' rows into y inside the
+ * down GEMM kernel, after a grid-wide barrier, instead of in a separate
+ * kernel; weight-major tilings only, the same order of additions, so the
+ * same bits).  All choices compute the same result.
  */
 moe_status moe_create(int d_model, int n_experts, int top_k, int d_ff, int n_shared,
                       moe_handle *out);

@@ -24,6 +24,7 @@ enum DeviceErrorSite : int {
   kSiteEpilogue = 3,
   kSiteDrain = 4,
   kSiteDispatch = 5,
+  kSiteGridSync = 6,   // the down GEMM's grid-wide barrier before its fused combine
 };
 
 __device__ __forceinline__ void report_error(int* status, int kind, int site) {

@@ -96,6 +96,13 @@ struct __align__(64) SwapParams {
   int out_rows;            // rows of the output buffer (T*k + S*T)
   int ksplit;              // down, 1-SM only: K ranges per output tile (1 = no split)
   float* part;             // with ksplit > 1: fp32 parts [ksplit][out_rows][n_out]
+  // Fused combine (down, bf16 Y rows): after all tiles and a grid-wide barrier,
+  //   y[t] = sum_s Y[T*k + s*T + t] + sum_i topk_w[t][i] * Y[pos[t*k + i]]
+  int fuse_combine;
+  const float* topk_w;     // [T][k]
+  const int32_t* pos;      // [T*k]
+  uint16_t* y;             // [T][n_out] bf16
+  unsigned int* grid_count;  // zero at launch; every CTA adds 1 when its tiles are done
 };
 
 struct SharedStorage {
@@ -106,6 +113,7 @@ struct SharedStorage {
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
+  int grid_done;    // fused combine: every CTA passed the grid-wide barrier in time
   int sched[MAX_GROUPS + 1];
   int offsets[MAX_GROUPS + 1];
   float stage_t[EPI_WARPS][16 * wm::STG_LD];   // per epilogue warp: one 16-token x 32 block
@@ -119,6 +127,73 @@ constexpr size_t swap_smem_bytes() {
 static_assert(swap_smem_bytes<true, false>() <= 227 * 1024, "shared memory budget");
 static_assert(swap_smem_bytes<true, true>() <= 227 * 1024, "shared memory budget");
 static_assert(swap_smem_bytes<false, true>() <= 227 * 1024, "shared memory budget");
+
+// The merge of the layer's output (m.xxqk.cn Hy4-preview MoE explainer, section 2.2)
+// inside the down GEMM.  Every CTA has stored its Y rows; a grid-wide barrier (one counter,
+// bounded wait; the grid is at most one CTA per SM, all resident) makes all rows visible,
+// then the CTAs share the tokens: 8 features per thread, the shared rows and then the k
+// weighted rows added in fp32 in the same order as the separate combine kernel, rounded
+// once.  Y is read through L2 (__ldcg): other SMs wrote it.
+__device__ __noinline__ void fused_combine(const SwapParams& p, int& all_done) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(p.grid_count, 1u);
+    const uint64_t t0 = globaltimer_ns();
+    int ok = 1;
+    while (true) {
+      unsigned int n;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(n) : "l"(p.grid_count) : "memory");
+      if (n >= gridDim.x) break;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        report_error(p.status, kDevTimeout, kSiteGridSync);
+        ok = 0;
+        break;
+      }
+    }
+    all_done = ok;
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+  if (!all_done) return;
+  const int d = p.n_out, k = p.k, S = p.S, T = p.T;
+  const size_t nslots = size_t(T) * k;
+  const uint16_t* Y = static_cast<const uint16_t*>(p.out);
+  const int vec = d / 8;
+  for (int64_t item = int64_t(blockIdx.x) * NUM_THREADS + threadIdx.x; item < int64_t(T) * vec;
+       item += int64_t(gridDim.x) * NUM_THREADS) {
+    const int t = int(item / vec);
+    const int c = int(item - int64_t(t) * vec) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < S; ++s) {
+      const uint4 a = __ldcg(reinterpret_cast<const uint4*>(Y + (nslots + size_t(s) * T + t) * d + c));
+      const uint32_t w4[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[2 * q] += bf16_bits_to_float(w4[q] & 0xFFFFu);
+        acc[2 * q + 1] += bf16_bits_to_float(w4[q] >> 16);
+      }
+    }
+    for (int i = 0; i < k; ++i) {
+      const int r = p.pos[size_t(t) * k + i];
+      if (r < 0 || size_t(r) >= nslots) continue;
+      const float w = p.topk_w[size_t(t) * k + i];
+      const uint4 a = __ldcg(reinterpret_cast<const uint4*>(Y + size_t(r) * d + c));
+      const uint32_t w4[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[2 * q] = fmaf(w, bf16_bits_to_float(w4[q] & 0xFFFFu), acc[2 * q]);
+        acc[2 * q + 1] = fmaf(w, bf16_bits_to_float(w4[q] >> 16), acc[2 * q + 1]);
+      }
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(p.y + size_t(t) * d + c) = o;
+  }
+}
 
 template <bool kGateUp, bool kPair>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -171,7 +246,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
   pdl_wait();   // the schedule, offsets and token operands come from earlier kernels
-  pdl_launch_dependents();
+  // With the fused combine every CTA waits for all the others, so the next kernel may not
+  // take an SM before all of them are resident: its launch is released after the barrier.
+  if (kGateUp || !p.fuse_combine) pdl_launch_dependents();
   for (int i = threadIdx.x; i <= G; i += NUM_THREADS) ss.sched[i] = p.sched[i];
   for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) ss.offsets[i] = p.offsets[i];
   tc_fence_before();
@@ -461,6 +538,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     if (kPair) tmem_dealloc_pair(tmem_base, TMEM_COLS); else tmem_dealloc(tmem_base, TMEM_COLS);
   }
+  if (!kGateUp && p.fuse_combine) fused_combine(p, ss.grid_done);
 }
 
 template <bool kGateUp, bool kPair>
@@ -481,6 +559,60 @@ cudaError_t launch_swap(const SwapParams& sp, int num_sms, cudaStream_t st) {
 }
 
 }  // namespace
+
+// Whether every CTA of the weight-major down GEMM's grid can be resident at once on the
+// current device (one CTA per SM by its shared memory; for the pair, as many 2-CTA clusters
+// as the grid has), which the fused combine's grid-wide barrier needs.
+bool swap_down_all_resident(bool pair) {
+  static thread_local int cached_dev = -1, cached[2] = {-1, -1};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (cached_dev != dev) {
+    cached[0] = cached[1] = -1;
+    cached_dev = dev;
+  }
+  if (cached[pair] < 0) {
+    int sms = 0;
+    bool ok = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess;
+    const unsigned grid = pair ? unsigned(sms & ~1) : unsigned(sms);
+    const size_t smem = pair ? swap_smem_bytes<false, true>() : swap_smem_bytes<false, false>();
+    if (ok && pair) {
+      ok = cudaFuncSetAttribute(grouped_gemm_swap_kernel<false, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) ==
+           cudaSuccess;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(grid);
+      cfg.blockDim = dim3(NUM_THREADS);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 2;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      ok = ok && cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_swap_kernel<false, true>,
+                                                &cfg) == cudaSuccess;
+      ok = ok && unsigned(clusters) * 2u >= grid;
+    } else if (ok) {
+      ok = cudaFuncSetAttribute(grouped_gemm_swap_kernel<false, false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) ==
+           cudaSuccess;
+      int per_sm = 0;
+      ok = ok && cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                     &per_sm, grouped_gemm_swap_kernel<false, false>, NUM_THREADS, smem) ==
+                     cudaSuccess;
+      ok = ok && unsigned(per_sm) * unsigned(sms) >= grid;
+    }
+    if (!ok) cudaGetLastError();
+    cached[pair] = ok ? 1 : 0;
+  }
+  return cached[pair] == 1;
+}
 
 moe_status launch_expert_ffn_swap(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                                   bool pair, cudaStream_t st) {
@@ -551,6 +683,13 @@ moe_status launch_expert_ffn_swap(const Ctx& c, const FfnArgs& a, const DeviceIn
   const bool split = !pair && a.down_ksplit > 1 && a.down_part && a.y_bf16;
   dp.ksplit = split ? a.down_ksplit : 1;
   dp.part = split ? a.down_part : nullptr;
+  if (a.fuse_combine && a.y_bf16 && !split) {   // grid_count was zeroed with the status word
+    dp.fuse_combine = 1;
+    dp.topk_w = a.topk_w;
+    dp.pos = a.pos;
+    dp.y = a.y_out;
+    dp.grid_count = a.grid_count;
+  }
   err = pair ? launch_swap<false, true>(dp, dev.num_sms, st)
              : launch_swap<false, false>(dp, dev.num_sms, st);
   if (err != cudaSuccess) return MOE_ERR_CUDA;

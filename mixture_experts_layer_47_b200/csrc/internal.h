@@ -54,6 +54,7 @@ struct Ctx {
   int d, E, k, F, S;
   RouterMode router = RouterMode::kAuto;
   TilesMode tiles = TilesMode::kAuto;
+  bool fused_combine = false;   // MOE_FUSED_COMBINE=1 at moe_create
   int e_base = 0;   // first local expert
   int E_all = 0;    // routed experts of the whole layer (0: E)
   int e_all() const { return E_all > 0 ? E_all : E; }
@@ -71,7 +72,7 @@ RouterPlan router_plan(const Ctx& c, int T, int num_sms);
 // Workspace carve-up for T tokens (offsets from the 1024-aligned base).
 struct Layout {
   size_t status, part, wparts, topk_idx, topk_w, counts, offsets, perm, pos, blk_hist, sched,
-      x_perm, h_act, y_rows, x_stage, y_stage, down_part, end;
+      x_perm, h_act, y_rows, x_stage, y_stage, down_part, grid_count, end;
   int nblk;           // dispatch blocks
   RouterPlan rplan;
 };
@@ -160,9 +161,17 @@ struct FfnArgs {
   // [down_ksplit][rows][d] in the workspace, added in order into Y.
   int down_ksplit = 1;
   float* down_part = nullptr;
+  // The combine fused into the down GEMM (weight-major tilings, bf16 Y rows): the down
+  // kernel writes y itself after a grid-wide barrier on grid_count (workspace).
+  bool fuse_combine = false;
+  const float* topk_w = nullptr;
+  const int32_t* pos = nullptr;
+  uint16_t* y_out = nullptr;
+  unsigned int* grid_count = nullptr;
 };
 moe_status launch_expert_ffn(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                              cudaStream_t st);
+bool swap_down_all_resident(bool pair);
 moe_status launch_expert_ffn_swap(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                                   bool pair, cudaStream_t st);
 moe_status launch_expert_ffn_fp8(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,

@@ -93,6 +93,7 @@ Layout make_layout(const Ctx& c, int T, int num_sms) {
   L.y_stage = take(size_t(T) * c.d * sizeof(uint16_t));
   L.down_part = take(size_t(dense_down_ksplit(c, T) > 1 ? dense_down_ksplit(c, T) : 0) * T * c.d *
                      sizeof(float));
+  L.grid_count = L.status + 64;   // inside the status block, cleared with the status word
   L.end = off;
   return L;
 }
@@ -155,6 +156,8 @@ moe_status moe_create(int d_model, int n_experts, int top_k, int d_ff, int n_sha
     if (strcmp(v, "tc") == 0) h->c.router = RouterMode::kTensorCore;
     if (strcmp(v, "ffma") == 0) h->c.router = RouterMode::kFfma;
   }
+  if (const char* v = getenv("MOE_FUSED_COMBINE"))
+    h->c.fused_combine = strcmp(v, "1") == 0;
   if (const char* v = getenv("MOE_GEMM_TILES")) {
     if (strcmp(v, "single") == 0) h->c.tiles = TilesMode::kSingle;
     if (strcmp(v, "pair") == 0) h->c.tiles = TilesMode::kPair;
@@ -377,6 +380,16 @@ moe_status moe_combine(moe_handle h, const float* Y, const float* topk_w, const 
       launch_combine(h->c, Y, topk_w, pos, T, y, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// Whether moe_forward runs the combine inside the down GEMM (context option
+// MOE_FUSED_COMBINE=1; only the weight-major tilings have the fused form).
+static bool combine_fused(const Ctx& c, int T) {
+  if (!c.fused_combine) return false;
+  const GemmTiling t = gemm_tiling(c, T);
+  if (t != GemmTiling::kSwap && t != GemmTiling::kSwapPair) return false;
+  // its grid-wide barrier needs every CTA of the down GEMM resident at once
+  return swap_down_all_resident(t == GemmTiling::kSwapPair);
+}
+
 // A shard of the layer for tensor or expert parallelism: the routed experts
 // e_base .. e_base + n_local - 1 (the caller's weights hold just those), with or
 // without the shared experts, and an unrounded fp32 output.
@@ -419,7 +432,8 @@ static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W
   auto mark = [&](int i) -> moe_status {
     return prof ? cuda_status(cudaEventRecord(h->stage_events[i], st)) : MOE_OK;
   };
-  if ((s = cuda_status(cudaMemsetAsync(status, 0, sizeof(int), st)))) return s;
+  // the status word and the fused combine's grid counter (same 256-byte block)
+  if ((s = cuda_status(cudaMemsetAsync(status, 0, 128, st)))) return s;
   if ((s = mark(0))) return s;
   if ((s = cuda_status(launch_router(c, L.rplan, x, W_router, bias, T,
                                      reinterpret_cast<float*>(ws + L.part),
@@ -446,11 +460,17 @@ static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W
   a.T = T;
   a.y_bf16 = true;
   a.after_gate_up = prof ? h->stage_events[4] : nullptr;
+  const bool fuse = combine_fused(c, T) && !shard && !w.r8;
+  a.fuse_combine = fuse;
+  a.topk_w = topk_w;
+  a.pos = pos;
+  a.y_out = y;
+  a.grid_count = reinterpret_cast<unsigned int*>(ws + L.grid_count);
   if ((s = launch_expert_ffn(cl, a, *dev, st))) return s;
   if ((s = mark(5))) return s;
   if (shard)
     s = cuda_status(launch_combine_partial(cl, Y, topk_w, pos, T, shard->y_partial, st));
-  else
+  else if (!fuse)
     s = cuda_status(launch_combine_bf16(c, Y, topk_w, pos, T, y, st));
   if (s) return s;
   return mark(6);
@@ -673,7 +693,8 @@ int moe_forward_kernel_count(moe_handle h, int T) {
   const RouterPlan rp = router_plan(c, T, kPlanSms);
   const int router = rp.tc ? 3 : 2;  // [weight split +] score GEMM + top-k
   const int dispatch = (int64_t(T) * c.k <= kDispatchChunk && c.E <= 256) ? 1 : 3;
-  return router + dispatch + 1 /*gather*/ + 2 /*GEMMs*/ + 1 /*combine*/;
+  const int combine = combine_fused(c, T) ? 0 : 1;
+  return router + dispatch + 1 /*gather*/ + 2 /*GEMMs*/ + combine;
 }
 
 int moe_dense_ffn_kernel_count(moe_handle h, int T) {
