@@ -220,3 +220,73 @@ def test_tuning_overrides_are_fixed_when_the_context_is_created(lib, monkeypatch
     monkeypatch.delenv("MOE_ROUTER")
     assert moe.moe_workspace_size(h_tc, T) == size_tc
     assert moe.moe_workspace_size(h_ffma, T) == size_ffma
+
+
+def test_shard_and_dense_entry_points_validate_on_the_host(lib):
+    """moe_forward_partial (expert range, partial shared pointers, alignment, workspace),
+    moe_reduce_partials (count, null or misaligned parts) and moe_dense_ffn (a context that is
+    not the one-expert layer), all decided before any CUDA call."""
+    L = moe.load_library()
+    A = 1 << 20
+    T = 32
+    h = moe.moe_create(256, 16, 2, 128, 1)
+    hv = h.value
+    ws = moe.moe_workspace_size(h, T)
+    fp = L.moe_forward_partial
+    # expert range outside [0, E), empty range
+    assert fp(hv, A, A, None, -1, 4, A, A, A, A, A, A, T, A, A, ws, None) == moe.MOE_ERR_INVALID_ARG
+    assert fp(hv, A, A, None, 14, 4, A, A, A, A, A, A, T, A, A, ws, None) == moe.MOE_ERR_INVALID_ARG
+    assert fp(hv, A, A, None, 0, 0, A, A, A, A, A, A, T, A, A, ws, None) == moe.MOE_ERR_INVALID_ARG
+    # the shared experts' pointers all or none
+    assert fp(hv, A, A, None, 0, 4, A, A, A, A, None, A, T, A, A, ws, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    # misaligned part, small workspace, no output
+    assert fp(hv, A, A, None, 0, 4, A, A, A, None, None, None, T, A + 4, A, ws, None) == \
+        moe.MOE_ERR_ALIGNMENT
+    assert fp(hv, A, A, None, 0, 4, A, A, A, None, None, None, T, A, A, ws - 1, None) == \
+        moe.MOE_ERR_WORKSPACE
+    assert fp(hv, A, A, None, 0, 4, A, A, A, None, None, None, T, None, A, ws, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert fp(hv, None, None, None, 0, 4, None, None, None, None, None, None, 0, None, None, 0,
+              None) == moe.MOE_OK
+    # reduce: 1..16 parts, each non-null and aligned
+    P = ctypes.c_void_p
+    parts = (P * 17)(*([A] * 17))
+    assert L.moe_reduce_partials(hv, parts, 0, T, A, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_reduce_partials(hv, parts, 17, T, A, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_reduce_partials(hv, None, 2, T, A, None) == moe.MOE_ERR_INVALID_ARG
+    holed = (P * 2)(A, None)
+    assert L.moe_reduce_partials(hv, holed, 2, T, A, None) == moe.MOE_ERR_INVALID_ARG
+    skew = (P * 2)(A, A + 4)
+    assert L.moe_reduce_partials(hv, skew, 2, T, A, None) == moe.MOE_ERR_ALIGNMENT
+    assert L.moe_reduce_partials(hv, parts, 2, T, A + 2, None) == moe.MOE_ERR_ALIGNMENT
+    assert L.moe_reduce_partials(hv, parts, 2, 0, A, None) == moe.MOE_OK
+    # dense layer: only the E=1, k=1, S=0 context
+    assert L.moe_dense_ffn(hv, A, A, A, A, T, A, A, ws, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_dense_ffn_kernel_count(hv, T) == -1
+    hd = moe.moe_create(256, 1, 1, 640, 0)
+    wsd = moe.moe_workspace_size(hd, T)
+    assert L.moe_dense_ffn(hd.value, A, A, A + 2, A, T, A, A, wsd, None) == moe.MOE_ERR_ALIGNMENT
+    assert L.moe_dense_ffn(hd.value, A, A, A, A, T, A, A, wsd - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert L.moe_dense_ffn(hd.value, None, None, None, None, 0, None, None, 0, None) == moe.MOE_OK
+    # up to 128 tokens the down projection is split over K (one launch more)
+    assert L.moe_dense_ffn_kernel_count(hd.value, 16) == 4
+    assert L.moe_dense_ffn_kernel_count(hd.value, 4096) == 3
+
+
+def test_fused_combine_option_is_fixed_at_create(lib, monkeypatch):
+    """MOE_FUSED_COMBINE=1 at moe_create takes the combine out of moe_forward's launch list
+    where it applies; the count of another context is unchanged (no device is needed to
+    count).  Without a GPU the occupancy check cannot pass, so the fused form is not chosen
+    and the counts agree."""
+    monkeypatch.delenv("MOE_FUSED_COMBINE", raising=False)
+    h0 = moe.moe_create(6144, 256, 8, 2048, 1)
+    monkeypatch.setenv("MOE_FUSED_COMBINE", "1")
+    h1 = moe.moe_create(6144, 256, 8, 2048, 1)
+    monkeypatch.delenv("MOE_FUSED_COMBINE")
+    n0 = moe.moe_forward_kernel_count(h0, 16)
+    n1 = moe.moe_forward_kernel_count(h1, 16)
+    assert n0 == 7
+    assert n1 in (n0, n0 - 1)
+    if not torch.cuda.is_available():
+        assert n1 == n0
