@@ -134,7 +134,7 @@ static_assert(swap_smem_bytes<false, true>() <= 227 * 1024, "shared memory budge
 // then the CTAs share the tokens: 8 features per thread, the shared rows and then the k
 // weighted rows added in fp32 in the same order as the separate combine kernel, rounded
 // once.  Y is read through L2 (__ldcg): other SMs wrote it.
-__device__ __noinline__ void fused_combine(const SwapParams& p, int& all_done) {
+__device__ __forceinline__ void fused_combine(const SwapParams& p, int& all_done) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -156,42 +156,97 @@ __device__ __noinline__ void fused_combine(const SwapParams& p, int& all_done) {
   __syncthreads();
   pdl_launch_dependents();
   if (!all_done) return;
+  // Only NUM_THREADS threads per SM do the merge, so each keeps many rows in flight: two
+  // items (token, 8 features) at a time, and every row of a chunk of up to 4 slots is loaded
+  // before the chunk's additions, which stay in the separate combine's order.
+  constexpr int kChunk = 4;
   const int d = p.n_out, k = p.k, S = p.S, T = p.T;
   const size_t nslots = size_t(T) * k;
   const uint16_t* Y = static_cast<const uint16_t*>(p.out);
   const int vec = d / 8;
-  for (int64_t item = int64_t(blockIdx.x) * NUM_THREADS + threadIdx.x; item < int64_t(T) * vec;
-       item += int64_t(gridDim.x) * NUM_THREADS) {
-    const int t = int(item / vec);
-    const int c = int(item - int64_t(t) * vec) * 8;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < S; ++s) {
-      const uint4 a = __ldcg(reinterpret_cast<const uint4*>(Y + (nslots + size_t(s) * T + t) * d + c));
-      const uint32_t w4[4] = {a.x, a.y, a.z, a.w};
+  const int64_t n_items = int64_t(T) * vec;
+  const int64_t stride = int64_t(gridDim.x) * NUM_THREADS;
+  for (int64_t item0 = int64_t(blockIdx.x) * NUM_THREADS + threadIdx.x; item0 < n_items;
+       item0 += 2 * stride) {
+    int t[2], c[2];
+    bool live[2];
+    float acc[2][8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        acc[2 * q] += bf16_bits_to_float(w4[q] & 0xFFFFu);
-        acc[2 * q + 1] += bf16_bits_to_float(w4[q] >> 16);
-      }
-    }
-    for (int i = 0; i < k; ++i) {
-      const int r = p.pos[size_t(t) * k + i];
-      if (r < 0 || size_t(r) >= nslots) continue;
-      const float w = p.topk_w[size_t(t) * k + i];
-      const uint4 a = __ldcg(reinterpret_cast<const uint4*>(Y + size_t(r) * d + c));
-      const uint32_t w4[4] = {a.x, a.y, a.z, a.w};
+    for (int u = 0; u < 2; ++u) {
+      const int64_t item = item0 + u * stride;
+      live[u] = item < n_items;
+      t[u] = live[u] ? int(item / vec) : 0;
+      c[u] = live[u] ? int(item - int64_t(t[u]) * vec) * 8 : 0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        acc[2 * q] = fmaf(w, bf16_bits_to_float(w4[q] & 0xFFFFu), acc[2 * q]);
-        acc[2 * q + 1] = fmaf(w, bf16_bits_to_float(w4[q] >> 16), acc[2 * q + 1]);
-      }
+      for (int j = 0; j < 8; ++j) acc[u][j] = 0.f;
     }
-    uint4 o;
-    o.x = pack_bf16x2(acc[0], acc[1]);
-    o.y = pack_bf16x2(acc[2], acc[3]);
-    o.z = pack_bf16x2(acc[4], acc[5]);
-    o.w = pack_bf16x2(acc[6], acc[7]);
-    *reinterpret_cast<uint4*>(p.y + size_t(t) * d + c) = o;
+    for (int s0 = 0; s0 < S; s0 += kChunk) {
+      uint4 v[2][kChunk];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j)
+          if (live[u] && s0 + j < S)
+            v[u][j] = __ldcg(reinterpret_cast<const uint4*>(
+                Y + (nslots + size_t(s0 + j) * T + t[u]) * d + c[u]));
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j)
+          if (live[u] && s0 + j < S) {
+            const uint32_t w4[4] = {v[u][j].x, v[u][j].y, v[u][j].z, v[u][j].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              acc[u][2 * q] += bf16_bits_to_float(w4[q] & 0xFFFFu);
+              acc[u][2 * q + 1] += bf16_bits_to_float(w4[q] >> 16);
+            }
+          }
+    }
+    for (int i0 = 0; i0 < k; i0 += kChunk) {
+      int r[2][kChunk];
+      float wt[2][kChunk];
+      uint4 v[2][kChunk];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) {
+          r[u][j] = -1;
+          if (live[u] && i0 + j < k) {
+            const int rr = p.pos[size_t(t[u]) * k + i0 + j];
+            r[u][j] = (rr >= 0 && size_t(rr) < nslots) ? rr : -1;
+            wt[u][j] = p.topk_w[size_t(t[u]) * k + i0 + j];
+          }
+        }
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j)
+          if (r[u][j] >= 0)
+            v[u][j] = __ldcg(reinterpret_cast<const uint4*>(Y + size_t(r[u][j]) * d + c[u]));
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j)
+          if (r[u][j] >= 0) {
+            const uint32_t w4[4] = {v[u][j].x, v[u][j].y, v[u][j].z, v[u][j].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              acc[u][2 * q] = fmaf(wt[u][j], bf16_bits_to_float(w4[q] & 0xFFFFu), acc[u][2 * q]);
+              acc[u][2 * q + 1] =
+                  fmaf(wt[u][j], bf16_bits_to_float(w4[q] >> 16), acc[u][2 * q + 1]);
+            }
+          }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      if (live[u]) {
+        uint4 o;
+        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+        *reinterpret_cast<uint4*>(p.y + size_t(t[u]) * d + c[u]) = o;
+      }
   }
 }
 
