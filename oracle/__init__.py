@@ -302,6 +302,55 @@ def shard_output(x, idx, w, W_gate, W_up, W_down, Ws_gate=None, Ws_up=None, Ws_d
     return out
 
 
+# ----------------------------------------------------------------------------
+# iHC: the layer inside four parallel residual streams.  ZAKER "Tencent releases and
+# open-sources Hy4 Preview", iHC paragraphs: identity Hyper-Connections widen the single
+# residual stream to 4 parallel streams that are recombined at every layer, and keep a stable
+# identity path under the learned exchange between streams.  The pages give no formula; the
+# reading (static hyper-connections with the identity term kept exactly):
+#   layer input   x[t]     = sum_j alpha[j] * H[t, j]
+#   stream update H'[t, i] = H[t, i] + sum_j B[i, j] * H[t, j] + gamma[i] * y[t]
+# with y = the MoE layer on x, and alpha [n], B [n, n], gamma [n] the learned coefficients.
+# ----------------------------------------------------------------------------
+def ihc_mix_in(H, alpha) -> np.ndarray:
+    """x[t] = sum_j alpha[j] * H[t, j] in fp64, j in order.  H: [T, n, d] bf16 (uint16 bits
+    or a CPU bf16 tensor) or float; returns [T, d] fp64."""
+    Hf = _as_f64(H)
+    alpha = np.asarray(alpha, np.float64)
+    T, n, d = Hf.shape
+    x = np.zeros((T, d), np.float64)
+    for j in range(n):
+        x += alpha[j] * Hf[:, j, :]
+    return x
+
+
+def ihc_update(H, B, gamma, y) -> np.ndarray:
+    """H'[t, i] = H[t, i] + sum_j B[i, j] * H[t, j] + gamma[i] * y[t] in fp64: the identity
+    path, then the exchange terms j in order, then the layer's output."""
+    Hf = _as_f64(H)
+    B = np.asarray(B, np.float64)
+    gamma = np.asarray(gamma, np.float64)
+    y = np.asarray(y, np.float64)
+    T, n, d = Hf.shape
+    out = np.empty_like(Hf)
+    for i in range(n):
+        acc = Hf[:, i, :].copy()
+        for j in range(n):
+            acc += B[i, j] * Hf[:, j, :]
+        out[:, i, :] = acc + gamma[i] * y
+    return out
+
+
+def _as_f64(a) -> np.ndarray:
+    """bf16 bit patterns (uint16) or a bf16 tensor -> exact fp64; float arrays as they are."""
+    if hasattr(a, "dtype") and str(a.dtype) == "torch.bfloat16":
+        a = a.view(dtype=__import__("torch").int16).numpy().view(np.uint16)
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
 def renormalised_gates(logits: np.ndarray, idx: np.ndarray) -> np.ndarray:
     """Gate weights for a given expert choice: softmax over all logits, renormalised over idx."""
     logits = np.asarray(logits, np.float64)

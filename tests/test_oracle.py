@@ -409,3 +409,53 @@ def test_expert_ranges_add_up_to_the_layer():
     none = oracle.shard_output(inp.x, idx, full["w"], inp.W_gate[:3], inp.W_up[:3],
                                inp.W_down[:3], expert_begin=0)
     assert np.all(none == 0.0)
+
+
+def test_ihc_update_hand_worked():
+    """Two streams, two features, one token, by hand:
+    H = [[1, 2], [4, 8]] (stream 0, stream 1), B = [[0, 0.5], [0.25, 0]], gamma = [1, -2],
+    y = [10, 20]:
+      H'_0 = H_0 + 0 * H_0 + 0.5 * H_1 + 1 * y = [1 + 2 + 10, 2 + 4 + 20] = [13, 26]
+      H'_1 = H_1 + 0.25 * H_0 + 0 * H_1 - 2 * y = [4 + 0.25 - 20, 8 + 0.5 - 40] = [-15.75, -31.5]
+    and the layer input with alpha = [0.5, 0.25] is x = [0.5 + 1, 1 + 2] = [1.5, 3]."""
+    H = np.array([[[1.0, 2.0], [4.0, 8.0]]])
+    out = oracle.ihc_update(H, [[0.0, 0.5], [0.25, 0.0]], [1.0, -2.0], [[10.0, 20.0]])
+    np.testing.assert_array_equal(out[0], [[13.0, 26.0], [-15.75, -31.5]])
+    np.testing.assert_array_equal(oracle.ihc_mix_in(H, [0.5, 0.25]), [[1.5, 3.0]])
+
+
+def test_ihc_with_one_stream_is_the_residual_connection():
+    """n = 1, alpha = 1, B = 0, gamma = 1: H' = H + layer(H), the ordinary residual block."""
+    inp = make_small(T=12, d=64, E=4, k=2, F=64, S=1, seed=71)
+    H = inp.x.view(12, 1, 64)
+    x = oracle.ihc_mix_in(H, [1.0])
+    xf = torch.tensor(x).float().to(torch.bfloat16)
+    assert torch.equal(xf.view(torch.int16), inp.x.view(torch.int16))   # exact: weight 1
+    y = oracle.forward(inp)["y"]
+    out = oracle.ihc_update(H, [[0.0]], [1.0], y)
+    np.testing.assert_allclose(out[:, 0, :], inp.x.double().numpy() + y, rtol=0, atol=0)
+
+
+def test_ihc_identity_path_and_stream_relabelling():
+    """B = 0 keeps every stream: H'_i - H_i = gamma_i y exactly.  Relabelling the streams
+    (alpha, the rows and columns of B, gamma, the stream axis of H) relabels the result,
+    with an asymmetric B so a transposed exchange would fail."""
+    g = torch.Generator().manual_seed(3)
+    H = torch.randn(5, 4, 32, generator=g).to(torch.bfloat16)
+    y = torch.randn(5, 32, generator=g).double().numpy()
+    gamma = np.array([0.5, -1.0, 2.0, 0.25])
+    out = oracle.ihc_update(H, np.zeros((4, 4)), gamma, y)
+    Hf = H.double().numpy()
+    for i in range(4):
+        np.testing.assert_array_equal(out[:, i] - Hf[:, i], gamma[i] * y)
+    B = np.arange(16, dtype=np.float64).reshape(4, 4) / 32.0
+    alpha = np.array([0.1, 0.2, 0.3, 0.4])
+    base = oracle.ihc_update(H, B, gamma, y)
+    pi = np.array([2, 0, 3, 1])             # new stream i is old stream pi[i]
+    perm = oracle.ihc_update(H[:, pi], B[np.ix_(pi, pi)], gamma[pi], y)
+    np.testing.assert_allclose(perm, base[:, pi], rtol=1e-15, atol=1e-15)
+    np.testing.assert_allclose(oracle.ihc_mix_in(H[:, pi], alpha[pi]),
+                               oracle.ihc_mix_in(H, alpha), rtol=1e-15, atol=1e-15)
+    # B against its transpose: stream 0 takes 1/32 of stream 1 in B, 4/32 in B^T
+    bt = oracle.ihc_update(H, B.T, gamma, y)
+    assert not np.allclose(bt, base)
