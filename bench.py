@@ -38,7 +38,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import ALL_WORKLOADS, Workload, make_fp8, make_inputs  # noqa: E402
+from workloads import ALL_WORKLOADS, Workload, make_fp8, make_ihc, make_inputs  # noqa: E402
 
 DEFAULT_WORKLOAD = "decode"
 
@@ -182,9 +182,10 @@ def algorithmic_work(wl: Workload, counts: np.ndarray) -> dict:
     gate_up_bytes = int((touched + wl.S) * 2 * wl.F * wl.d * bpe)
     down_bytes = int((touched + wl.S) * wl.F * wl.d * bpe)
     dense = wl.layer == "dense"     # no router: weights, x and y only
+    act = wl.n_streams if wl.layer == "ihc" else 1   # iHC: n streams in and out
     return {
         "touched_experts": touched,
-        "layer_bytes": w_bytes + (0 if dense else wl.E * wl.d * 4) + 2 * wl.T * wl.d * 2,
+        "layer_bytes": w_bytes + (0 if dense else wl.E * wl.d * 4) + 2 * act * wl.T * wl.d * 2,
         "expert_flops": 6 * wl.d * wl.F * rows,
         "router_flops": 0 if dense else 2 * wl.T * wl.d * wl.E,
         "gate_up_bytes": gate_up_bytes,
@@ -230,7 +231,7 @@ def hbm_bound(wl: Workload, work: dict, peaks: dict) -> bool:
 # (--workload, decode by default) and, in "workloads", the others.  Each is created,
 # timed and freed before the next (19.4 GB of weights each).
 EXTRA_WORKLOADS = ("batched_decode", "prefill", "skewed_prefill", "decode_fp8",
-                   "batched_decode_fp8", "dense_decode", "dense_prefill")
+                   "batched_decode_fp8", "dense_decode", "dense_prefill", "decode_ihc")
 
 
 def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds: float,
@@ -261,11 +262,24 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
         torch.cuda.empty_cache()
     weights = (inp.W_gate, inp.W_up, inp.W_down, inp.Ws_gate, inp.Ws_up, inp.Ws_down)
     dense = wl.layer == "dense"
+    ihc = make_ihc(wl, device) if wl.layer == "ihc" else None
     x_stage = torch.empty_like(inp.x) if dense else None
     y_stage = torch.empty_like(y) if dense else None
+    if ihc is not None:   # the activations are the residual streams H [T, n, d]
+        inp.x = ihc[0]
+        y = torch.empty_like(ihc[0])
+        x_stage, y_stage = torch.empty_like(ihc[0]), torch.empty_like(ihc[0])
 
     def forward(x_arg, y_arg, host=False):
-        if dense:   # the dense FFN layer; host activations go through two copies around it
+        if ihc is not None:   # the layer inside iHC streams; host streams copied around it
+            H_in, H_out = (x_stage, y_stage) if host else (x_arg, y_arg)
+            if host:
+                x_stage.copy_(x_arg, non_blocking=True)
+            moe.moe_forward_ihc(h, H_in, ihc[1], ihc[2], ihc[3], inp.W_router, inp.bias,
+                                *weights, H_out, ws, stream)
+            if host:
+                y_arg.copy_(y_stage, non_blocking=True)
+        elif dense:   # the dense FFN layer; host activations go through two copies around it
             if host:
                 x_stage.copy_(x_arg, non_blocking=True)
                 moe.moe_dense_ffn(h, x_stage, inp.W_gate, inp.W_up, inp.W_down, y_stage, ws,
@@ -329,7 +343,7 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
 
     # ---- end to end: pinned host x in, host y out, through moe_forward_host ----
     x_host = inp.x.cpu().pin_memory()
-    y_host = torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory()
+    y_host = torch.empty(y.shape, dtype=torch.bfloat16).pin_memory()
     for _ in range(max(1, args.warmup)):
         forward(x_host, y_host, host=True)
     torch.cuda.synchronize(device)
@@ -347,14 +361,15 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
     raw = {"step_ms": step_ms, "stage_ms": stage_ms.mean(0).tolist(), "e2e_ms": e2e_ms,
            "counts": counts, "clocks": clocks.summary(),
            "kernels_per_step": (moe.moe_dense_ffn_kernel_count(h, wl.T) if dense
-                                else moe.moe_forward_kernel_count(h, wl.T)),
+                                else moe.moe_forward_kernel_count(h, wl.T)
+                                + (1 if ihc is not None else 0)),   # + the iHC mix
            "h2d_bytes": int(x_host.numel() * x_host.element_size()),
            "d2h_bytes": int(y_host.numel() * y_host.element_size()), "fp8": fp8 is not None}
-    if rank == 0 and world == 1 and cpu_seconds > 0:
+    if rank == 0 and world == 1 and cpu_seconds > 0 and ihc is None:
         raw["cpu_baseline"] = cpu_baseline(inp, cpu_seconds, fp8, cpu_tokens)
     if hbm_bound(wl, algorithmic_work(wl, counts), load_peaks()):
         raw["read_only_gbs"] = read_only_peak(device)
-    del inp, fp8, weights, ws, y, flush, x_host, y_host, x_stage, y_stage
+    del inp, fp8, weights, ws, y, flush, x_host, y_host, x_stage, y_stage, ihc
     moe.moe_destroy(h)
     torch.cuda.synchronize(device)
     torch.cuda.empty_cache()
@@ -449,6 +464,8 @@ def report_workload(wl: Workload, raw: dict, args, world: int, device, stage_nam
         "e2e": {"value": round(tokens_all / (e2e_total / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": raw["h2d_bytes"], "d2h_bytes_per_step": raw["d2h_bytes"],
                 "api": ("moe_dense_ffn between pinned host copies" if wl.layer == "dense" else
+                "moe_forward_ihc between pinned host copies of the streams" if wl.layer == "ihc"
+                else
                         ("moe_forward_fp8_host" if raw["fp8"] else "moe_forward_host")
                         + " (pinned host x in, host y out)")},
         "gpu_launches": raw["kernels_per_step"] * args.steps,

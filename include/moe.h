@@ -317,6 +317,41 @@ moe_status moe_reduce_partials(moe_handle h, const float *const *partials, int n
                                uint16_t *y, void *stream);
 
 /*
+ * iHC wrapper: the layer inside n parallel residual streams.  The pages'
+ * model widens the residual stream to 4 parallel streams that are
+ * recombined at every layer and keeps a stable identity path under the
+ * learned exchange between them (ZAKER Hy4 Preview release news, iHC
+ * paragraphs: identity Hyper-Connections); they give no formula.  Reading:
+ *   layer input   x[t]     = sum_j alpha[j] * H[t][j]
+ *   stream update H'[t][i] = H[t][i] + sum_j B[i][j] * H[t][j] + gamma[i] * y[t]
+ * with y the MoE layer on x (as in moe_forward), alpha [n], B [n][n] and
+ * gamma [n] the learned coefficients.  Arithmetic: fp32, in the order written
+ * (identity term, exchange terms in j order, layer output); x is rounded to
+ * bf16 as the layer's input, y stays in fp32 (the combine's sum) and each
+ * H' element is rounded once to bf16.
+ *
+ * moe_ihc_mix: x only.  H: bf16 [T][n][d]; alpha: fp32 [n] (device);
+ * x: bf16 [T][d] (output); 1 <= n_streams <= 8.
+ */
+moe_status moe_ihc_mix(moe_handle h, const uint16_t *H, int n_streams, const float *alpha, int T,
+                       uint16_t *x, void *stream);
+
+/*
+ * moe_forward_ihc: the whole wrapped layer: the mix, then moe_forward on x
+ * (x kept in the workspace), with the combine writing the updated streams
+ * H_out instead of y (y never leaves the combine's registers).  B: fp32
+ * [n][n] row-major (B[i][j] is stream j's share in stream i); gamma: fp32 [n]
+ * (device pointers); H_out: bf16 [T][n][d], may be H itself.  Other
+ * arguments and the workspace as in moe_forward.
+ */
+moe_status moe_forward_ihc(moe_handle h, const uint16_t *H, int n_streams, const float *alpha,
+                           const float *B, const float *gamma, const float *W_router,
+                           const float *bias, const uint16_t *W_gate, const uint16_t *W_up,
+                           const uint16_t *W_down, const uint16_t *Ws_gate,
+                           const uint16_t *Ws_up, const uint16_t *Ws_down, int T,
+                           uint16_t *H_out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * The dense FFN layer.  Of the model's 78 layers the first uses a standard
  * dense FFN and the other 77 the MoE FFN (ZAKER Hy4 Preview release news,
  * architecture paragraph); the pages give the dense layer no width.  Reading:

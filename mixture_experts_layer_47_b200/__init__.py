@@ -39,7 +39,7 @@ EXPORTS = ("moe_create", "moe_destroy", "moe_workspace_size", "moe_get_workspace
            "moe_dispatch_noalloc", "moe_selftest_wait_timeout", "moe_forward_kernel_count",
            "moe_status_string", "moe_expert_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_host",
            "moe_forward_partial", "moe_reduce_partials", "moe_dense_ffn",
-           "moe_dense_ffn_kernel_count")
+           "moe_dense_ffn_kernel_count", "moe_ihc_mix", "moe_forward_ihc")
 MOE_STAGE_EVENTS = 7
 STAGE_NAMES = ("router", "dispatch", "gather", "gate_up_gemm", "down_gemm", "combine")
 
@@ -103,6 +103,8 @@ def load_library() -> ctypes.CDLL:
         "moe_reduce_partials": ([P, ctypes.POINTER(P), I, I, P, P], I),
         "moe_dense_ffn": ([P, P, P, P, P, I, P, P, Z, P], I),
         "moe_dense_ffn_kernel_count": ([P, I], I),
+        "moe_ihc_mix": ([P, P, I, P, I, P, P], I),
+        "moe_forward_ihc": ([P, P, I, P, P, P, P, P, P, P, P, P, P, P, I, P, P, Z, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -428,6 +430,32 @@ def moe_selftest_wait_timeout(workspace, timeout_ns: int, stream=None) -> None:
 
 def moe_forward_kernel_count(h: Handle, T: int) -> int:
     return int(load_library().moe_forward_kernel_count(h.value, int(T)))
+
+
+def moe_ihc_mix(h: Handle, H, alpha, x, stream=None) -> None:
+    """x = bf16(sum_j alpha[j] H[:, j]) for streams H [T, n, d] (bf16) and alpha [n] (fp32)."""
+    T, n = H.shape[0], H.shape[1]
+    _check(load_library().moe_ihc_mix(
+        h.value, _ptr(H, torch.bfloat16, "H", (T, n, h.d)), n,
+        _ptr(alpha, torch.float32, "alpha", (n,)), T, _ptr(x, torch.bfloat16, "x", (T, h.d)),
+        _stream(stream)), "moe_ihc_mix")
+
+
+def moe_forward_ihc(h: Handle, H, alpha, B, gamma, W_router, bias, W_gate, W_up, W_down,
+                    Ws_gate, Ws_up, Ws_down, H_out, workspace, stream=None) -> None:
+    """The layer inside n residual streams: H_out[:, i] = H[:, i] + sum_j B[i, j] H[:, j]
+    + gamma[i] * layer(sum_j alpha[j] H[:, j])."""
+    T, n = H.shape[0], H.shape[1]
+    wp, wn = _ws(workspace)
+    _check(load_library().moe_forward_ihc(
+        h.value, _ptr(H, torch.bfloat16, "H", (T, n, h.d)), n,
+        _ptr(alpha, torch.float32, "alpha", (n,)), _ptr(B, torch.float32, "B", (n, n)),
+        _ptr(gamma, torch.float32, "gamma", (n,)),
+        _ptr(W_router, torch.float32, "W_router", (h.E, h.d)),
+        _ptr(bias, torch.float32, "bias", (h.E,)),
+        *_weights(h, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down), T,
+        _ptr(H_out, torch.bfloat16, "H_out", (T, n, h.d)), wp, wn, _stream(stream)),
+        "moe_forward_ihc")
 
 
 def moe_dense_ffn_kernel_count(h: Handle, T: int) -> int:

@@ -17,6 +17,12 @@
 //           unrounded, and
 //  reduce   adds the shards' fp32 partial outputs in rank order and rounds the
 //           total once to bf16 (moe_reduce_partials).
+//  iHC      the layer inside n parallel residual streams H [T][n][d] (ZAKER Hy4
+//           Preview release news, iHC paragraphs: identity Hyper-Connections, four
+//           streams recombined at every layer, the identity path kept):
+//             mix     x[t]     = sum_j alpha[j] H[t][j]                    -> bf16
+//             update  H'[t][i] = H[t][i] + sum_j B[i][j] H[t][j] + gamma[i] y[t]
+//           where the update is done by the combine itself, with y[t] its fp32 sum.
 #include "common.cuh"
 #include "internal.h"
 
@@ -132,20 +138,16 @@ __device__ __forceinline__ void store8(const float (&acc)[8], float* __restrict_
   *reinterpret_cast<float4*>(out + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
 }
 
-// TY = float (Y in fp32) or uint16_t (Y in bf16); the sums are fp32 either way.
-// TOut = uint16_t (y in bf16) or float (a shard's unrounded partial output).
-template <typename TY, typename Row, typename TOut>
-__global__ void __launch_bounds__(kCombineThreads)
-    combine_kernel(const TY* __restrict__ Y, const float* __restrict__ topk_w,
-                   const int32_t* __restrict__ pos, int T, int k, int S, int d,
-                   TOut* __restrict__ y) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const int t = blockIdx.x;
-  const int c = (blockIdx.y * kCombineThreads + threadIdx.x) * 8;
-  if (c >= d) return;
+// The merge of token t's rows for features c .. c+7, in fp32: the shared experts' rows,
+// then the k weighted rows in order.  TY = float (Y in fp32) or uint16_t (Y in bf16).
+template <typename TY, typename Row>
+__device__ __forceinline__ void combine_sum8(const TY* __restrict__ Y,
+                                             const float* __restrict__ topk_w,
+                                             const int32_t* __restrict__ pos, int T, int k,
+                                             int S, int d, int t, int c, float (&acc)[8]) {
   const size_t nslots = size_t(T) * k;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
   float v[8];
   for (int s = 0; s < S; ++s) {
     Row::load8(Y + (nslots + size_t(s) * T + t) * d + c, v);
@@ -160,7 +162,84 @@ __global__ void __launch_bounds__(kCombineThreads)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = fmaf(w, v[j], acc[j]);
   }
+}
+
+// TOut = uint16_t (y in bf16) or float (a shard's unrounded partial output).
+template <typename TY, typename Row, typename TOut>
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_kernel(const TY* __restrict__ Y, const float* __restrict__ topk_w,
+                   const int32_t* __restrict__ pos, int T, int k, int S, int d,
+                   TOut* __restrict__ y) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int t = blockIdx.x;
+  const int c = (blockIdx.y * kCombineThreads + threadIdx.x) * 8;
+  if (c >= d) return;
+  float acc[8];
+  combine_sum8<TY, Row>(Y, topk_w, pos, T, k, S, d, t, c, acc);
   store8(acc, y + size_t(t) * d + c);
+}
+
+// The iHC stream update done by the combine: y[t] stays in fp32 registers, every stream's
+// 8 features are read once, and H'[t][i] = H[t][i] + sum_j B[i][j] H[t][j] + gamma[i] y[t]
+// (identity term, then the exchange terms in j order, then the layer output) is rounded once
+// to bf16.  H_out may be H: each thread reads its elements of all streams before writing.
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_ihc_kernel(const uint16_t* __restrict__ Y, const float* __restrict__ topk_w,
+                       const int32_t* __restrict__ pos, int T, int k, int S, int d,
+                       const uint16_t* H, const float* __restrict__ Bm,
+                       const float* __restrict__ gamma, int n, uint16_t* H_out) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int t = blockIdx.x;
+  const int c = (blockIdx.y * kCombineThreads + threadIdx.x) * 8;
+  if (c >= d) return;
+  float acc[8];
+  combine_sum8<uint16_t, RowBF16>(Y, topk_w, pos, T, k, S, d, t, c, acc);
+  float h[kMaxStreams][8];
+#pragma unroll
+  for (int j = 0; j < kMaxStreams; ++j)
+    if (j < n) RowBF16::load8(H + (size_t(t) * n + j) * d + c, h[j]);
+#pragma unroll
+  for (int i = 0; i < kMaxStreams; ++i) {
+    if (i < n) {
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = h[i][e];
+#pragma unroll
+      for (int j = 0; j < kMaxStreams; ++j) {
+        if (j < n) {
+          const float b = Bm[i * n + j];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[e] = fmaf(b, h[j][e], o[e]);
+        }
+      }
+      const float g = gamma[i];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = fmaf(g, acc[e], o[e]);
+      store8(o, H_out + (size_t(t) * n + i) * d + c);
+    }
+  }
+}
+
+// iHC layer input: x[t] = bf16(sum_j alpha[j] H[t][j]), fp32 in j order.
+__global__ void __launch_bounds__(kCombineThreads)
+    ihc_mix_kernel(const uint16_t* __restrict__ H, const float* __restrict__ alpha, int n,
+                   int d, uint16_t* __restrict__ x) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int t = blockIdx.x;
+  const int c = (blockIdx.y * kCombineThreads + threadIdx.x) * 8;
+  if (c >= d) return;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int j = 0; j < n; ++j) {
+    float v[8];
+    RowBF16::load8(H + (size_t(t) * n + j) * d + c, v);
+    const float a = alpha[j];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = fmaf(a, v[e], acc[e]);
+  }
+  store8(acc, x + size_t(t) * d + c);
 }
 
 // y[i] = bf16(sum_{r < n} part_r[i]) in fp32, r in order; 8 elements per thread per step.
@@ -171,11 +250,14 @@ __global__ void __launch_bounds__(kCombineThreads)
   for (size_t v = size_t(blockIdx.x) * kCombineThreads + threadIdx.x; v < n_vec8;
        v += size_t(gridDim.x) * kCombineThreads) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int r = 0; r < n; ++r) {
-      float x[8];
-      RowF32::load8(parts.p[r] + v * 8, x);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[j] += x[j];
+    for (int r = 0; r < kMaxPartials; ++r) {   // unrolled: the pointers stay in registers
+      if (r < n) {
+        float x[8];
+        RowF32::load8(parts.p[r] + v * 8, x);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] += x[j];
+      }
     }
     store8(acc, y + v * 8);
   }
@@ -230,6 +312,20 @@ cudaError_t launch_combine_partial(const Ctx& c, const uint16_t* Y, const float*
   dim3 grid(T, (c.d / 8 + kCombineThreads - 1) / kCombineThreads);
   return launch_pdl(combine_kernel<uint16_t, RowBF16, float>, grid, dim3(kCombineThreads), 0, st,
                     1, Y, topk_w, pos, T, c.k, c.S, c.d, y_partial);
+}
+
+cudaError_t launch_ihc_mix(const Ctx& c, const uint16_t* H, const float* alpha, int n, int T,
+                           uint16_t* x, cudaStream_t st) {
+  dim3 grid(T, (c.d / 8 + kCombineThreads - 1) / kCombineThreads);
+  return launch_pdl(ihc_mix_kernel, grid, dim3(kCombineThreads), 0, st, 1, H, alpha, n, c.d, x);
+}
+
+cudaError_t launch_combine_ihc(const Ctx& c, const uint16_t* Y, const float* topk_w,
+                               const int32_t* pos, int T, const uint16_t* H, const float* B,
+                               const float* gamma, int n, uint16_t* H_out, cudaStream_t st) {
+  dim3 grid(T, (c.d / 8 + kCombineThreads - 1) / kCombineThreads);
+  return launch_pdl(combine_ihc_kernel, grid, dim3(kCombineThreads), 0, st, 1, Y, topk_w, pos, T,
+                    c.k, c.S, c.d, H, B, gamma, n, H_out);
 }
 
 cudaError_t launch_reduce_partials(const PartialPtrs& parts, int n, size_t elems, uint16_t* y,

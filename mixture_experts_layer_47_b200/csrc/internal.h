@@ -133,6 +133,14 @@ cudaError_t launch_combine_bf16(const Ctx& c, const uint16_t* Y, const float* to
 cudaError_t launch_combine_partial(const Ctx& c, const uint16_t* Y, const float* topk_w,
                                    const int32_t* pos, int T, float* y_partial, cudaStream_t st);
 
+// iHC: parallel residual streams per token (the pages' model uses 4).
+constexpr int kMaxStreams = 8;
+cudaError_t launch_ihc_mix(const Ctx& c, const uint16_t* H, const float* alpha, int n, int T,
+                           uint16_t* x, cudaStream_t st);
+cudaError_t launch_combine_ihc(const Ctx& c, const uint16_t* Y, const float* topk_w,
+                               const int32_t* pos, int T, const uint16_t* H, const float* B,
+                               const float* gamma, int n, uint16_t* H_out, cudaStream_t st);
+
 // Up to this many fp32 partial outputs are added by one moe_reduce_partials call.
 constexpr int kMaxPartials = 16;
 struct PartialPtrs {

@@ -399,6 +399,15 @@ struct Shard {
   float* y_partial;
 };
 
+// The iHC wrapper's stream update, done by the combine (moe_forward_ihc).
+struct IhcArgs {
+  const uint16_t* H;     // [T][n][d] streams in
+  const float* B;        // [n][n] exchange between streams
+  const float* gamma;    // [n] weight of the layer output per stream
+  int n;
+  uint16_t* H_out;       // [T][n][d] streams out (may be H)
+};
+
 // The shape the expert stages see: the whole layer, or one shard of it.
 static Ctx stage_shape(const Ctx& c, const Shard* sh) {
   Ctx cl = c;
@@ -414,7 +423,7 @@ static Ctx stage_shape(const Ctx& c, const Shard* sh) {
 static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W_router,
                                  const float* bias, const Weights& w, int T, uint16_t* y,
                                  uint8_t* ws, const Layout& L, DeviceInfo* dev, cudaStream_t st,
-                                 const Shard* shard = nullptr) {
+                                 const Shard* shard = nullptr, const IhcArgs* ihc = nullptr) {
   const Ctx& c = h->c;
   const Ctx cl = stage_shape(c, shard);   // dispatch, gather, GEMMs and combine
   moe_status s;
@@ -460,7 +469,7 @@ static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W
   a.T = T;
   a.y_bf16 = true;
   a.after_gate_up = prof ? h->stage_events[4] : nullptr;
-  const bool fuse = combine_fused(c, T) && !shard && !w.r8;
+  const bool fuse = combine_fused(c, T) && !shard && !w.r8 && !ihc;
   a.fuse_combine = fuse;
   a.topk_w = topk_w;
   a.pos = pos;
@@ -470,6 +479,9 @@ static moe_status forward_device(moe_handle h, const uint16_t* x, const float* W
   if ((s = mark(5))) return s;
   if (shard)
     s = cuda_status(launch_combine_partial(cl, Y, topk_w, pos, T, shard->y_partial, st));
+  else if (ihc)
+    s = cuda_status(launch_combine_ihc(c, Y, topk_w, pos, T, ihc->H, ihc->B, ihc->gamma, ihc->n,
+                                       ihc->H_out, st));
   else if (!fuse)
     s = cuda_status(launch_combine_bf16(c, Y, topk_w, pos, T, y, st));
   if (s) return s;
@@ -643,6 +655,50 @@ moe_status moe_dense_ffn(moe_handle h, const uint16_t* x, const uint16_t* W_gate
   if ((s = launch_expert_ffn(c, a, *dev, st))) return s;
   if ((s = mark(5))) return s;
   return mark(6);   // no combine
+}
+
+moe_status moe_ihc_mix(moe_handle h, const uint16_t* H, int n_streams, const float* alpha, int T,
+                       uint16_t* x, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_T(h->c, T);
+  if (s) return s;
+  if (n_streams < 1 || n_streams > kMaxStreams) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!H || !alpha || !x) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(H) || !aligned16(alpha) || !aligned16(x)) return MOE_ERR_ALIGNMENT;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  return cuda_status(
+      launch_ihc_mix(h->c, H, alpha, n_streams, T, x, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_forward_ihc(moe_handle h, const uint16_t* H, int n_streams, const float* alpha,
+                           const float* B, const float* gamma, const float* W_router,
+                           const float* bias, const uint16_t* W_gate, const uint16_t* W_up,
+                           const uint16_t* W_down, const uint16_t* Ws_gate,
+                           const uint16_t* Ws_up, const uint16_t* Ws_down, int T,
+                           uint16_t* H_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_T(h->c, T);
+  if (s) return s;
+  if (n_streams < 1 || n_streams > kMaxStreams) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!H || !alpha || !B || !gamma || !H_out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(H) || !aligned16(alpha) || !aligned16(B) || !aligned16(gamma) ||
+      !aligned16(H_out))
+    return MOE_ERR_ALIGNMENT;
+  const Weights w = bf16_weights(W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down);
+  // the layer input x is made by the mix below; H stands in for it in the checks
+  if ((s = check_forward_args(h, H, W_router, w, T, H_out, false, workspace, ws_bytes))) return s;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Layout L = make_layout(h->c, T, kPlanSms);
+  uint8_t* ws = aligned_base(workspace);
+  uint16_t* x = reinterpret_cast<uint16_t*>(ws + L.x_stage);
+  if ((s = cuda_status(launch_ihc_mix(h->c, H, alpha, n_streams, T, x, st)))) return s;
+  const IhcArgs ihc{H, B, gamma, n_streams, H_out};
+  return forward_device(h, x, W_router, bias, w, T, nullptr, ws, L, dev, st, nullptr, &ihc);
 }
 
 moe_status moe_reduce_partials(moe_handle h, const float* const* partials, int n_partials, int T,

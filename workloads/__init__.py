@@ -49,7 +49,9 @@ class Workload:
     seed: int = 0
     description: str = ""
     weights: str = "bf16"           # "bf16", or "fp8": the same draws stored as e4m3 + block scales
-    layer: str = "moe"              # "moe", or "dense": the dense FFN layer (E = 1, k = 1, S = 0)
+    layer: str = "moe"              # "moe"; "dense": the dense FFN layer (E = 1, k = 1, S = 0);
+                                    # "ihc": the MoE layer inside n_streams residual streams
+    n_streams: int = 0              # iHC streams (the pages' model: 4)
 
     @property
     def slots(self) -> int:
@@ -92,6 +94,13 @@ WORKLOADS = {
         "batched_decode_fp8", T=256, d=6144, E=256, k=8, F=2048, S=1, router="uniform", seed=0,
         weights="fp8",
         description="the batched decode workload with FP8 expert weights"),
+    # The MoE layer inside the iHC wrapper's four residual streams (ZAKER release news, iHC
+    # paragraphs); streams H ~ N(0, 1), alpha ~ U(0.1, 0.5), B ~ N(0, 0.1^2), gamma ~ U(0.5, 1.5)
+    # drawn after the layer's inputs (make_ihc).
+    "decode_ihc": Workload(
+        "decode_ihc", T=16, d=6144, E=256, k=8, F=2048, S=1, router="normal", seed=0,
+        layer="ihc", n_streams=4,
+        description="the decode workload inside four iHC residual streams"),
     # The model's first layer is a standard dense FFN (ZAKER release news, architecture
     # paragraph); its width is not printed.  Reading: SwiGLU of width (8 + 1) * 2048 = 18432,
     # the FFN width one token passes through in an MoE layer (8 routed + 1 shared experts).
@@ -341,3 +350,16 @@ def make_fp8(inp: Inputs) -> tuple:
         dn, ds = quantize_fp8(Wd)
         return Fp8Set(g, gs, u, us, dn, ds)
     return one(inp.W_gate, inp.W_up, inp.W_down), one(inp.Ws_gate, inp.Ws_up, inp.Ws_down)
+
+
+def make_ihc(wl: Workload, device="cpu") -> tuple:
+    """(H [T, n, d] bf16, alpha [n], B [n, n], gamma [n] fp32) for an iHC workload, drawn with
+    a CPU generator seeded with seed + 17: H ~ N(0, 1), alpha ~ U(0.1, 0.5),
+    B ~ N(0, 0.1^2), gamma ~ U(0.5, 1.5)."""
+    n = wl.n_streams
+    g = torch.Generator().manual_seed(wl.seed + 17)
+    H = torch.randn(wl.T, n, wl.d, generator=g).to(torch.bfloat16)
+    alpha = (0.1 + 0.4 * torch.rand(n, generator=g)).float()
+    B = (0.1 * torch.randn(n, n, generator=g)).float()
+    gamma = (0.5 + torch.rand(n, generator=g)).float()
+    return tuple(t.to(device) for t in (H, alpha, B, gamma))
