@@ -86,8 +86,8 @@ moe_status moe_destroy(moe_handle h);
  * Bytes of device workspace that any call below needs for T tokens
  * (0 when h is NULL or T < 0).  One workspace of this size serves every
  * call; it holds intermediates only and may be reused across calls that the
- * stream orders.  At the Hy4 shape it is about 2.2 GB at T = 8192 and about
- * 5 MB at T = 16.
+ * stream orders.  At the Hy4 shape it is about 2.3 GB at T = 8192 and about
+ * 6 MB at T = 16.
  */
 size_t moe_workspace_size(moe_handle h, int T);
 
@@ -194,10 +194,16 @@ moe_status moe_forward(moe_handle h, const uint16_t *x, const float *W_router, c
 /*
  * moe_forward with the activations in HOST memory: copies x_host (bf16
  * [T][d]) to the device, runs the layer, copies y back to y_host (bf16
- * [T][d]), all on the stream; returns once the copies are enqueued (the
- * caller synchronises the stream before reading y_host).  Host buffers
- * should be page-locked for the copies to be asynchronous.  Weights and the
- * workspace are device memory as in moe_forward.
+ * [T][d]); returns once everything is enqueued.  y_host holds the result
+ * when the stream has reached the end of the call (the caller synchronises
+ * the stream before reading it).  The input copy runs on a helper stream of
+ * the context (made at its first host-activation call on a device) into one
+ * of two staging slots of the workspace used in turn, so it can start before
+ * the stream reaches the call -- while the previous call's layer still runs;
+ * x_host must therefore stay unchanged from the call until the stream has
+ * passed it.  Host buffers should be page-locked for the copies to be
+ * asynchronous.  Weights and the workspace are device memory as in
+ * moe_forward.
  */
 moe_status moe_forward_host(moe_handle h, const uint16_t *x_host, const float *W_router,
                             const float *bias, const uint16_t *W_gate, const uint16_t *W_up,

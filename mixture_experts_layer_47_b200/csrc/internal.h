@@ -72,7 +72,7 @@ RouterPlan router_plan(const Ctx& c, int T, int num_sms);
 // Workspace carve-up for T tokens (offsets from the 1024-aligned base).
 struct Layout {
   size_t status, part, wparts, topk_idx, topk_w, counts, offsets, perm, pos, blk_hist, sched,
-      x_perm, h_act, y_rows, x_stage, y_stage, down_part, grid_count, end;
+      x_perm, h_act, y_rows, x_stage, x_stage2, y_stage, down_part, grid_count, end;
   int nblk;           // dispatch blocks
   RouterPlan rplan;
 };

@@ -17,10 +17,23 @@
 #include "common.cuh"
 #include "internal.h"
 
+// The input copies of moe_forward_host / moe_forward_fp8_host run on a helper stream
+// (one per device, made at the context's first such call on it) into two staging slots
+// used in turn, so that a call's copy can start while the previous call's layer runs.
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t copy = nullptr;
+  cudaEvent_t copied[2] = {nullptr, nullptr};   // the slot's input copy has landed
+  cudaEvent_t freed[2] = {nullptr, nullptr};    // the layer that read the slot is done
+  unsigned next = 0;                            // slot of the next call
+};
+
 struct moe_ctx {
   moe::Ctx c;
   cudaEvent_t stage_events[MOE_STAGE_EVENTS];
   int n_stage_events;
+  HostPipe pipes[64];   // per device ordinal
+  std::mutex pipe_mu;
 };
 
 namespace moe {
@@ -90,6 +103,7 @@ Layout make_layout(const Ctx& c, int T, int num_sms) {
   L.h_act = take(rows * c.F * sizeof(uint16_t));
   L.y_rows = take(rows * c.d * sizeof(uint16_t));  // bf16 rows of moe_forward
   L.x_stage = take(size_t(T) * c.d * sizeof(uint16_t));
+  L.x_stage2 = take(size_t(T) * c.d * sizeof(uint16_t));
   L.y_stage = take(size_t(T) * c.d * sizeof(uint16_t));
   L.down_part = take(size_t(dense_down_ksplit(c, T) > 1 ? dense_down_ksplit(c, T) : 0) * T * c.d *
                      sizeof(float));
@@ -170,6 +184,20 @@ moe_status moe_create(int d_model, int n_experts, int top_k, int d_ff, int n_sha
 }
 
 moe_status moe_destroy(moe_handle h) {
+  if (!h) return MOE_OK;
+  int cur = -1;
+  const bool have_cur = cudaGetDevice(&cur) == cudaSuccess;
+  for (int d = 0; d < 64; ++d) {
+    HostPipe& hp = h->pipes[d];
+    if (!hp.ready || cudaSetDevice(d) != cudaSuccess) continue;
+    cudaStreamDestroy(hp.copy);
+    for (int i = 0; i < 2; ++i) {
+      cudaEventDestroy(hp.copied[i]);
+      cudaEventDestroy(hp.freed[i]);
+    }
+  }
+  if (have_cur) cudaSetDevice(cur);
+  cudaGetLastError();
   delete h;
   return MOE_OK;
 }
@@ -529,11 +557,33 @@ static moe_status forward_host_impl(moe_handle h, const uint16_t* x_host, const 
   const Layout L = make_layout(h->c, T, kPlanSms);
   uint8_t* ws = aligned_base(workspace);
   const size_t bytes = size_t(T) * h->c.d * sizeof(uint16_t);
-  uint16_t* x_dev = reinterpret_cast<uint16_t*>(ws + L.x_stage);
+  HostPipe& hp = h->pipes[dev->device];
+  unsigned slot;
+  {
+    std::lock_guard<std::mutex> lock(h->pipe_mu);
+    if (!hp.ready) {
+      bool ok = cudaStreamCreateWithFlags(&hp.copy, cudaStreamNonBlocking) == cudaSuccess;
+      for (int i = 0; i < 2 && ok; ++i)
+        ok = cudaEventCreateWithFlags(&hp.copied[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&hp.freed[i], cudaEventDisableTiming) == cudaSuccess;
+      if (!ok) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+      }
+      hp.ready = true;
+    }
+    slot = hp.next++ & 1u;
+  }
+  uint16_t* x_dev = reinterpret_cast<uint16_t*>(ws + (slot ? L.x_stage2 : L.x_stage));
   uint16_t* y_dev = reinterpret_cast<uint16_t*>(ws + L.y_stage);
-  if ((s = cuda_status(cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st))))
+  // input copy on the helper stream, once the layer that last read this slot is done
+  if ((s = cuda_status(cudaStreamWaitEvent(hp.copy, hp.freed[slot], 0)))) return s;
+  if ((s = cuda_status(cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, hp.copy))))
     return s;
+  if ((s = cuda_status(cudaEventRecord(hp.copied[slot], hp.copy)))) return s;
+  if ((s = cuda_status(cudaStreamWaitEvent(st, hp.copied[slot], 0)))) return s;
   if ((s = forward_device(h, x_dev, W_router, bias, w, T, y_dev, ws, L, dev, st))) return s;
+  if ((s = cuda_status(cudaEventRecord(hp.freed[slot], st)))) return s;
   return cuda_status(cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st));
 }
 
@@ -695,7 +745,9 @@ moe_status moe_forward_ihc(moe_handle h, const uint16_t* H, int n_streams, const
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const Layout L = make_layout(h->c, T, kPlanSms);
   uint8_t* ws = aligned_base(workspace);
-  uint16_t* x = reinterpret_cast<uint16_t*>(ws + L.x_stage);
+  // x goes to the y staging area: the host-activation calls' helper stream writes only
+  // the x staging slots, and everything on this stream is ordered
+  uint16_t* x = reinterpret_cast<uint16_t*>(ws + L.y_stage);
   if ((s = cuda_status(launch_ihc_mix(h->c, H, alpha, n_streams, T, x, st)))) return s;
   const IhcArgs ihc{H, B, gamma, n_streams, H_out};
   return forward_device(h, x, W_router, bias, w, T, nullptr, ws, L, dev, st, nullptr, &ihc);

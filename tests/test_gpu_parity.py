@@ -328,3 +328,31 @@ def test_zero_tokens_is_a_no_op():
     moe.moe_forward(h, x, dev.W_router, None, dev.W_gate, dev.W_up, dev.W_down, dev.Ws_gate,
                     dev.Ws_up, dev.Ws_down, y, ws)
     torch.cuda.synchronize()
+
+
+def test_back_to_back_host_calls_keep_each_input():
+    """moe_forward_host calls enqueued without synchronising, each on its own pinned input:
+    the input copies run ahead on the context's helper stream into two staging slots used in
+    turn, so a slot must not be overwritten before the layer that reads it is done.  A long
+    wait kernel on the stream first lets the copies run far ahead; every output must still
+    equal moe_forward's on its own input."""
+    wl_inp = make_small(96, 256, 16, 2, 128, 1, seed=61)
+    dev = to_device(wl_inp, "cuda")
+    wl = wl_inp.wl
+    h = moe.moe_create(wl.d, wl.E, wl.k, wl.F, wl.S)
+    ws = torch.empty(moe.moe_workspace_size(h, wl.T), dtype=torch.uint8, device="cuda")
+    W = (dev.W_gate, dev.W_up, dev.W_down, dev.Ws_gate, dev.Ws_up, dev.Ws_down)
+    g = torch.Generator().manual_seed(8)
+    xs = [torch.randn(wl.T, wl.d, generator=g).to(torch.bfloat16).pin_memory() for _ in range(5)]
+    ys = [torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory() for _ in range(5)]
+    torch.cuda.synchronize()
+    torch.cuda._sleep(50_000_000)                    # ~25 ms of spinning on the stream
+    for x, y in zip(xs, ys):
+        moe.moe_forward_host(h, x, dev.W_router, dev.bias, *W, y, ws)
+    torch.cuda.synchronize()
+    for x, y in zip(xs, ys):
+        ref = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda")
+        moe.moe_forward(h, x.cuda(), dev.W_router, dev.bias, *W, ref, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(ref.cpu().view(torch.int16), y.view(torch.int16))
+    assert moe.moe_device_status(h, wl.T, ws)[0] == moe.MOE_OK
