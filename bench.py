@@ -195,10 +195,12 @@ def algorithmic_work(wl: Workload, counts: np.ndarray) -> dict:
     }
 
 
-def measured_traffic(kernel: str, bound: str, units: int, weights: str = "bf16"):
+def measured_traffic(kernel: str, bound: str, units: int, weights: str = "bf16",
+                     d_model: int = 6144, d_ff: int = 2048):
     """DRAM bytes per launch of ``kernel`` scaled from the committed ncu capture
-    (profiles/traffic.json), or None when there is none or the kernel source has
-    changed since the counters were taken."""
+    (profiles/traffic.json) by the touched experts, or None when there is none, when the
+    experts' shape differs from the captured one (per-expert bytes do not carry over), or
+    when the kernel source has changed since the counters were taken."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
@@ -207,6 +209,8 @@ def measured_traffic(kernel: str, bound: str, units: int, weights: str = "bf16")
     with open(path) as f:
         entry = json.load(f).get(key)
     if not entry or entry.get("bound") != bound:
+        return None
+    if entry.get("d_model", d_model) != d_model or entry.get("d_ff", d_ff) != d_ff:
         return None
     src = os.path.join(ROOT, "mixture_experts_layer_47_b200", "csrc",
                        entry.get("kernel_source", "expert_gemm.cu"))
@@ -418,7 +422,7 @@ def roofline(wl: Workload, work: dict, stage_mean: dict, peaks: dict) -> dict:
                 "peak_sustained": peaks["bf16_tflops_sustained"],
                 "frac_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4)}
     traffic = measured_traffic(dominant, roof["bound"], work["touched_experts"] + wl.S,
-                               wl.weights)
+                               wl.weights, wl.d, wl.F)
     roof.update({"kernel": dominant, "traffic": traffic, "peak_source": peaks["source"],
                  "algorithmic_per_launch": work[key + ("_bytes" if roof["bound"] == "hbm"
                                                        else "_flops")],

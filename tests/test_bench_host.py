@@ -66,7 +66,8 @@ def test_measured_traffic_lookup_and_invalidation(tmp_path, monkeypatch):
     sha = hashlib.sha256(kernel.read_bytes()).hexdigest()
     table = {
         "gate_up_gemm/hbm": {"bound": "hbm", "bytes_per_touched_expert": 1000,
-                             "kernel_source": "k.cu", "kernel_source_sha256": sha},
+                             "kernel_source": "k.cu", "kernel_source_sha256": sha,
+                             "d_model": 6144, "d_ff": 2048},
         "gate_up_gemm/hbm/fp8": {"bound": "hbm", "bytes_per_touched_expert": 520,
                                  "kernel_source": "k.cu", "kernel_source_sha256": sha},
     }
@@ -76,6 +77,7 @@ def test_measured_traffic_lookup_and_invalidation(tmp_path, monkeypatch):
     assert bench.measured_traffic("gate_up_gemm", "hbm", 10, "fp8") == 5200
     assert bench.measured_traffic("gate_up_gemm", "tensor", 10) is None   # no entry
     assert bench.measured_traffic("down_gemm", "hbm", 10) is None
+    assert bench.measured_traffic("gate_up_gemm", "hbm", 1, "bf16", 6144, 18432) is None
     kernel.write_text("// kernel v2\n")                                     # source changed
     assert bench.measured_traffic("gate_up_gemm", "hbm", 10) is None
 
