@@ -195,8 +195,15 @@ def algorithmic_work(wl: Workload, counts: np.ndarray) -> dict:
     }
 
 
+def fp8_form(T: int) -> str:
+    """Which FP8 expert GEMM the library runs for a T-token batch: the warp-MMA form
+    (expert_gemv_fp8.cu) up to 16 tokens unless MOE_GEMM_TILES picks a tiling, else the
+    tcgen05 kernel (expert_gemm_fp8.cu)."""
+    return "fp8_mma" if T <= 16 and not os.environ.get("MOE_GEMM_TILES") else "fp8"
+
+
 def measured_traffic(kernel: str, bound: str, units: int, weights: str = "bf16",
-                     d_model: int = 6144, d_ff: int = 2048):
+                     d_model: int = 6144, d_ff: int = 2048, T: int = 16):
     """DRAM bytes per launch of ``kernel`` scaled from the committed ncu capture
     (profiles/traffic.json) by the touched experts, or None when there is none, when the
     experts' shape differs from the captured one (per-expert bytes do not carry over), or
@@ -205,7 +212,7 @@ def measured_traffic(kernel: str, bound: str, units: int, weights: str = "bf16",
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
-    key = f"{kernel}/{bound}" + ("/fp8" if weights == "fp8" else "")
+    key = f"{kernel}/{bound}" + ("/" + fp8_form(T) if weights == "fp8" else "")
     with open(path) as f:
         entry = json.load(f).get(key)
     if not entry or entry.get("bound") != bound:
@@ -422,7 +429,7 @@ def roofline(wl: Workload, work: dict, stage_mean: dict, peaks: dict) -> dict:
                 "peak_sustained": peaks["bf16_tflops_sustained"],
                 "frac_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4)}
     traffic = measured_traffic(dominant, roof["bound"], work["touched_experts"] + wl.S,
-                               wl.weights, wl.d, wl.F)
+                               wl.weights, wl.d, wl.F, wl.T)
     roof.update({"kernel": dominant, "traffic": traffic, "peak_source": peaks["source"],
                  "algorithmic_per_launch": work[key + ("_bytes" if roof["bound"] == "hbm"
                                                        else "_flops")],

@@ -70,11 +70,15 @@ typedef int moe_status;
  * made here; the device is checked (sm_100 required) at the first launch.
  * Three tuning overrides are read from the environment here, once, and fixed
  * for the context's lifetime: MOE_ROUTER=tc|ffma (router path),
- * MOE_GEMM_TILES=single|pair|swap|swap_pair (expert GEMM tiling) and
- * MOE_FUSED_COMBINE=1 (moe_forward merges the experts' rows into y inside the
- * down GEMM kernel, after a grid-wide barrier, instead of in a separate
- * kernel; weight-major tilings only, the same order of additions, so the
- * same bits).  All choices compute the same result.
+ * MOE_GEMM_TILES=single|pair|swap|swap_pair (expert GEMM tiling; with FP8
+ * weights any of them picks the tcgen05 kernel at every batch size --
+ * swap_pair its 2-SM form, the others its 1-SM form -- where the default
+ * takes the warp-MMA form up to 16 tokens) and MOE_FUSED_COMBINE=1
+ * (moe_forward merges the experts'
+ * rows into y inside the down GEMM kernel, after a grid-wide barrier,
+ * instead of in a separate kernel; weight-major tilings only, the same
+ * order of additions, so the same bits).  All choices compute the same
+ * result up to the order of fp32 additions.
  */
 moe_status moe_create(int d_model, int n_experts, int top_k, int d_ff, int n_shared,
                       moe_handle *out);
@@ -234,9 +238,13 @@ typedef struct moe_fp8_expert_weights {
 
 /*
  * moe_expert_ffn with FP8 expert weights.  The GEMMs decode codes and scales
- * to bf16 in shared memory and run the same bf16 tensor-core contractions
- * (fp32 accumulation, activation rounded to bf16, Y in fp32), so Y equals
- * moe_expert_ffn's Y given the decoded weights.  The decoding is exact for
+ * to bf16 and run the same bf16 tensor-core contractions (fp32 accumulation,
+ * activation rounded to bf16, Y in fp32), so Y equals moe_expert_ffn's Y
+ * given the decoded weights.  At up to 16 tokens (unless MOE_GEMM_TILES is
+ * set) the codes are decoded in registers and multiplied by warp-level
+ * m16n8k16 MMAs: the same exact bf16 x bf16 products, added in fp32 in
+ * another order, so there the activations and Y equal the tcgen05 path's up
+ * to that order.  The decoding is exact for
  * every finite code whose scaled value is zero or at least 2^-133 in
  * magnitude (bf16's smallest subnormal), which holds for scale bytes >= 7,
  * and for scale bytes up to 134 (scales up to 2^7, weights up to 57344 in

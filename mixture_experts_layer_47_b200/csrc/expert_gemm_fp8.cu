@@ -55,6 +55,7 @@
 #include <string.h>
 
 #include "common.cuh"
+#include "fp8_decode.cuh"
 #include "internal.h"
 #include "tensor_map.cuh"
 #include "weight_major.cuh"
@@ -126,44 +127,6 @@ constexpr size_t fp8_smem_bytes() {
   return 1024 + size_t(STAGES) * STAGE_BYTES + sizeof(SharedStorage);
 }
 static_assert(fp8_smem_bytes() <= 227 * 1024, "shared memory budget");
-
-// E4M3 -> bf16 without the conversion pipe.  Written into bits 4-10 of a bf16
-// (exponent field bits 7-10, mantissa bits 4-6) with its sign in bit 15, a code's
-// bits read as a bf16 equal to the code's value times 2^-120 -- for normal codes
-// (exponent e >= 1: 2^(e-127) (1 + m/8) against 2^(e-7) (1 + m/8)), for subnormal
-// ones (bf16 subnormal 2^-126 m/8 against 2^-6 m/8) and for zero.  One bf16
-// multiply by 2^(120 + s - 127) then gives code * 2^(s - 127) exactly (a product
-// with at most 4 significant bits) for scale bytes s <= 134, where that factor is
-// a finite bf16, and results at or above bf16's smallest subnormal.
-// PRMT selectors placing code bytes (0,1) or (2,3) of a word into bits 8-15 and
-// 24-31 of the result (the other bytes taken from the zero operand).
-constexpr uint32_t kSel01 = 0x1404u;
-constexpr uint32_t kSel23 = 0x3424u;
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(d) : "r"(a), "r"(sel));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-// Two codes (in bits 8-15 and 24-31 of x8) to a bf16 pair times mult2.
-__device__ __forceinline__ uint32_t decode_pair(uint32_t x8, uint32_t mult2) {
-  const uint32_t mag = (x8 >> 4) & 0x07F007F0u;       // magnitude bits -> bits 4-10, 20-26
-  const uint32_t v = mag | (x8 & 0x80008000u);        // sign bits stay at 15 and 31
-  return bf16x2_mul(v, mult2);
-}
-
-// bf16 pair (2^(s - 7), 2^(s - 7)) for scale byte s.
-__device__ __forceinline__ uint32_t scale_pair(uint32_t s) {
-  const uint32_t e = (s + 120u) << 7;
-  return e | (e << 16);
-}
 
 // Prefix sums of the 32-token tile counts per group (routed groups clamped to
 // [0, T] tokens, then S shared groups of T tokens), by one warp.
@@ -572,6 +535,9 @@ bool encode_set(CUtensorMap* codes, CUtensorMap* scales, const uint8_t* c, const
 
 moe_status launch_expert_ffn_fp8(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                                  cudaStream_t st) {
+  // Decode-size batches go to the CUDA-core form: a tensor-core MMA over 16 tokens costs
+  // about as much as the bf16 weights' HBM time, twice the FP8 codes'.
+  if (a.T <= kGemvMaxT && c.tiles == TilesMode::kAuto) return launch_expert_ffn_gemv_fp8(c, a, dev, st);
   if (!tensor_map_encoder()) return MOE_ERR_CUDA;
   const moe_fp8_expert_weights& R = *a.fp8_routed;
   const moe_fp8_expert_weights* Sh = a.fp8_shared;

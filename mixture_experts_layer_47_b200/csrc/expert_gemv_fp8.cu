@@ -1,0 +1,426 @@
+// expert_gemv_fp8.cu -- the FP8-weight expert FFNs at decode batch sizes (up to 16 tokens).
+//
+// The contractions of the layer's experts (m.xxqk.cn Hy4-preview MoE explainer, section
+// 2.1; ZAKER Hy4 Preview release news: 256 routed experts plus one shared expert):
+//   gate/up:  H_g = silu(X_g W_gate_g^T) * (X_g W_up_g^T)   -> bf16
+//   down:     Y_g = H_g W_down_g^T                           -> fp32 or bf16
+// with every weight an E4M3 code times a power-of-two scale per 32 K elements of its row
+// (scales K-block-major, [n][K/32][rows]).  At decode sizes a group holds a handful of
+// tokens.  The tensor-core FP8 kernel (codes decoded into tensor memory, tcgen05 MMAs of
+// M = 128, N = 16) is then bound by its MMA issue cost, not by the FP8 stream, and a
+// CUDA-core dot product spends about ten instructions per weight.  Here each weight costs
+// about two: the decoder's (per word of four codes, two byte planes, two PRMTs and two
+// bf16x2 multiplies), with the multiply-adds done by warp-level m16n8k16 bf16 MMAs on the
+// decoded registers.
+//
+// Work: a warp item is 16 feature rows of one group -- the gate and the up rows of 16
+// features, or 32 consecutive W_down rows as two 16-row tiles -- for all of the group's
+// tokens (one MMA column block of 8 tokens, two when the group has more than 8).  The
+// grid's warps take items round robin; an item walks K in blocks of 64.
+// Fragments: in an m16n8k16 MMA lane l = 4 g + t holds A rows g and g + 8 at k slots
+// {2t, 2t+1, 2t+8, 2t+9} and B (token g) at the same slots.  The sum over k does not care
+// which K position a slot stands for, so in K block kb, MMA s (0..3), the slots of lane t
+// stand for positions kb + 16 t + 4 s .. + 3: a lane's 16 consecutive codes per row (one
+// 16-byte load) and its 16 consecutive activations (32 bytes) feed all four MMAs of the
+// block, and each 32-wide scale block lies inside one lane's run.
+// Stream: each lane copies its rows' codes and its tokens' activations for a block with
+// cp.async into a per-warp 4-stage ring in shared memory, three blocks ahead of the block it
+// computes (the ring runs on across item boundaries; the lane keeps running source pointers),
+// so the loads in flight hold no registers; four lanes also copy the tiles' 16 scale bytes
+// per 32-wide K block, read by all lanes after the ring wait and a warp barrier.
+// Arithmetic: exact bf16 weights (the decoder of the tensor-core FP8 kernel) times bf16
+// activations into fp32 accumulators, as in the tensor-core path; only the order of the
+// fp32 additions differs.  The epilogue applies SwiGLU (gate/up) from registers: a lane's
+// gate and up accumulators hold the same (feature, token) pairs.
+#include "common.cuh"
+#include "fp8_decode.cuh"
+#include "internal.h"
+#include "weight_major.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int GV_WARPS = 12;
+constexpr int GV_THREADS = 32 * GV_WARPS;
+constexpr int GV_KB = 64;                        // K per block (4 MMAs)
+constexpr int GV_STAGES = 4;
+constexpr int GV_MAX_GROUPS = 1024 + 8;          // E + S upper bound
+constexpr int GV_MAX_TOK = 16;                   // tokens per group: two 8-token MMA columns
+// Per warp and stage: codes [tile 2][row half 2][lane 32][16 B], activations
+// [column block 2][lane 32][32 B], scales [tile 2][32-wide K block 2][16 B].
+constexpr int GV_CODE_OFF = 0;
+constexpr int GV_X_OFF = 2 * 2 * 32 * 16;
+constexpr int GV_SCALE_OFF = GV_X_OFF + 2 * 32 * 32;
+constexpr int GV_STAGE_BYTES = GV_SCALE_OFF + 2 * 2 * 16;
+constexpr size_t GV_SMEM = size_t(GV_WARPS) * GV_STAGES * GV_STAGE_BYTES;
+static_assert(GV_STAGE_BYTES % 16 == 0, "stages stay 16-byte aligned");
+
+struct GemvParams {
+  const uint8_t* w[2];         // routed codes: gate/up W_gate, W_up [E][F][d]; down W_down [E][d][F]
+  const uint8_t* s[2];         // their scales [E][K/32][rows]
+  const uint8_t* sw[2];        // shared-expert codes
+  const uint8_t* ss[2];        // shared-expert scales
+  const uint16_t* tok_routed;  // gate/up: X_perm [T*k][d]; down: H [T*k+S*T][F]
+  const uint16_t* tok_shared;  // gate/up: x [T][d];        down: H
+  const int32_t* offsets;      // [E+1]
+  void* out;                   // gate/up: H bf16 [T*k+S*T][F]; down: Y fp32 or bf16 [..][d]
+  int out_bf16;
+  int T, E, S, k;
+  int K;                       // reduction length (d or F), a multiple of 64
+  int n_out;                   // output features per group = weight rows per expert (F or d)
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// until at most GV_STAGES - 1 of this thread's copy groups are still in flight
+__device__ __forceinline__ void cp_async_wait_ring() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(GV_STAGES - 1) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// d += A (16 x 16 bf16, row-major fragments a) * B (16 x 8 bf16, column fragments b), fp32.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// One warp item: features f .. of group g (rows of tile m: gate/up -> matrix m rows f ..
+// f+15, down -> W_down rows f + 16 m .. f + 16 m + 15), its tokens and where its outputs go.
+struct Item {
+  size_t woff;           // codes of row f in its expert set
+  size_t soff;           // scale of row f, K block 0
+  const uint16_t* tok;   // first token's activation row
+  size_t out_row;        // first token's output row
+  int f;                 // first feature
+  int nt;                // tokens, 1..GV_MAX_TOK; 0 past the last item
+  bool shared;           // a shared expert's item
+};
+
+template <bool kGateUp>
+__device__ __forceinline__ Item describe(const GemvParams& p, const int16_t* units, int G,
+                                         int per_unit, int total, int item) {
+  constexpr int FEATS = kGateUp ? 16 : 32;
+  Item it;
+  it.nt = 0;
+  if (item >= total) return it;
+  const int u = item / per_unit;
+  it.f = (item - u * per_unit) * FEATS;
+  int lo = 0, hi = G;                                  // units[lo] <= u < units[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (units[mid] <= u) lo = mid; else hi = mid;
+  }
+  const int g = lo;
+  const bool shared = g >= p.E;
+  const int gl = shared ? g - p.E : g;
+  const int off = shared ? 0 : __ldg(p.offsets + g);
+  it.nt = shared ? p.T : min(p.T, __ldg(p.offsets + g + 1) - off);
+  const size_t row0 = shared ? size_t(p.T) * p.k + size_t(gl) * p.T : size_t(off);
+  const size_t tok_row = (shared && kGateUp) ? size_t(0) : row0;
+  it.tok = (shared && kGateUp ? p.tok_shared : p.tok_routed) + tok_row * size_t(p.K);
+  it.out_row = row0;
+  it.shared = shared;
+  it.woff = (size_t(gl) * p.n_out + it.f) * p.K;
+  it.soff = size_t(gl) * (p.K / 32) * p.n_out + it.f;
+  return it;
+}
+
+// What the loop over items needs besides the parameters.
+struct Walk {
+  const int16_t* units;
+  int G, per_unit, total, nblk, nwarps, lane;
+  uint8_t* ring;       // this warp's GV_STAGES stages
+  uint32_t ring_s;     // the same, as a shared-memory address
+};
+
+// The copies run GV_STAGES - 1 blocks ahead of the arithmetic, across item boundaries.  The
+// cursor keeps this lane's source pointers for its next block: codes of rows g and g + 8
+// of both tiles, the activations of tokens g and g + 8, and (lanes 0-3) a scale row.
+struct IssueCursor {
+  const uint8_t* code[4];   // [tile m * 2 + row half h]
+  const uint16_t* x[2];     // [column block n]
+  const uint8_t* scale;     // lane 2 m + b < 4: tile m's scales of 32-wide block 2 blk + b
+  int item, blk, nt;        // nt = 0 past the last item
+};
+
+template <bool kGateUp>
+__device__ __forceinline__ void cursor_at(const GemvParams& p, const Item& it, IssueCursor& ic,
+                                          int lane) {
+  ic.nt = it.nt;
+  ic.blk = 0;
+  if (it.nt == 0) return;
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const uint8_t* base = (it.shared ? p.sw[kGateUp ? m : 0] : p.w[kGateUp ? m : 0]) + it.woff +
+                          size_t(kGateUp ? 0 : 16 * m) * p.K + 16 * t;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) ic.code[m * 2 + h] = base + size_t(g + 8 * h) * p.K;
+  }
+#pragma unroll
+  for (int n = 0; n < 2; ++n) ic.x[n] = it.tok + size_t(g + 8 * n) * p.K + 16 * t;
+  const int m = (lane >> 1) & 1, b = lane & 1;
+  ic.scale = (it.shared ? p.ss[kGateUp ? m : 0] : p.s[kGateUp ? m : 0]) + it.soff +
+             (kGateUp ? 0 : 16 * m) + size_t(b) * p.n_out;
+}
+
+// Copies of the cursor's block into a stage, then the cursor moves one block on.
+template <bool kGateUp>
+__device__ __forceinline__ void issue_next(const GemvParams& p, const Walk& wk, IssueCursor& ic,
+                                           int slot) {
+  const uint32_t stage = wk.ring_s + uint32_t(slot * GV_STAGE_BYTES);
+  const int lane = wk.lane, g = lane >> 2;
+  if (ic.nt > 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      cp_async16(stage + uint32_t(GV_CODE_OFF + (i * 32 + lane) * 16), ic.code[i]);
+      ic.code[i] += GV_KB;
+    }
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+      if (g + 8 * n < ic.nt) {
+        const uint32_t dst = stage + uint32_t(GV_X_OFF + (n * 32 + lane) * 32);
+        cp_async16(dst, ic.x[n]);
+        cp_async16(dst + 16, ic.x[n] + 8);
+      }
+      ic.x[n] += GV_KB;
+    }
+    if (lane < 4) cp_async16(stage + uint32_t(GV_SCALE_OFF + lane * 16), ic.scale);
+    ic.scale += size_t(2) * p.n_out;
+  }
+  cp_async_commit();
+  if (++ic.blk == wk.nblk) {
+    ic.item += wk.nwarps;
+    cursor_at<kGateUp>(p, describe<kGateUp>(p, wk.units, wk.G, wk.per_unit, wk.total, ic.item),
+                       ic, lane);
+  }
+}
+
+// The four MMAs of one K block for NCOL 8-token column blocks.  The activation columns of
+// tokens past the group's end are never copied and hold stale values: an MMA's output
+// column depends on its own B column only, and those columns are not stored.
+template <int NCOL>
+__device__ __forceinline__ void compute_block(const uint8_t* stage, float (&acc)[2][2][4],
+                                              int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  uint4 code[2][2];
+  uint32_t mult[2][2];
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      code[m][h] = *reinterpret_cast<const uint4*>(stage + GV_CODE_OFF + ((m * 2 + h) * 32 + lane) * 16);
+      // this lane's 16 positions lie in 32-wide block t / 2 of the 64
+      mult[m][h] = scale_pair(stage[GV_SCALE_OFF + (m * 2 + (t >> 1)) * 16 + g + 8 * h]);
+    }
+  uint4 xv[NCOL][2];
+#pragma unroll
+  for (int n = 0; n < NCOL; ++n) {
+    const uint4* src = reinterpret_cast<const uint4*>(stage + GV_X_OFF + (n * 32 + lane) * 32);
+    xv[n][0] = src[0];
+    xv[n][1] = src[1];
+  }
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      // slots 2t, 2t+1 <- codes 4s, 4s+1 of the run; slots 2t+8, 2t+9 <- codes 4s+2, 4s+3
+      uint32_t a[4];
+      decode_word((&code[m][0].x)[s], mult[m][0], a[0], a[2]);
+      decode_word((&code[m][1].x)[s], mult[m][1], a[1], a[3]);
+#pragma unroll
+      for (int n = 0; n < NCOL; ++n) {
+        const uint4& xs = xv[n][s >> 1];
+        mma_bf16_16816(acc[m][n], a, (s & 1) ? xs.z : xs.x, (s & 1) ? xs.w : xs.y);
+      }
+    }
+  }
+}
+
+// After an item's last block: accumulator element i of column block n is
+// (row g + 8 (i / 2), token 8 n + 2 t + i % 2) of both tiles.
+template <bool kGateUp, int NCOL>
+__device__ __forceinline__ void finish_item(const GemvParams& p, const Item& it,
+                                            const float (&acc)[2][2][4], int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int n = 0; n < NCOL; ++n)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int tok = 8 * n + 2 * t + (i & 1);
+      if (tok >= it.nt) continue;
+      const int row = g + 8 * (i >> 1);
+      const size_t o = (it.out_row + tok) * size_t(p.n_out) + it.f + row;
+      if (kGateUp) {
+        reinterpret_cast<uint16_t*>(p.out)[o] =
+            uint16_t(pack_bf16x2(wm::swiglu(acc[0][n][i], acc[1][n][i]), 0.f) & 0xFFFFu);
+      } else {
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          if (p.out_bf16)
+            reinterpret_cast<uint16_t*>(p.out)[o + 16 * m] =
+                uint16_t(pack_bf16x2(acc[m][n][i], 0.f) & 0xFFFFu);
+          else
+            reinterpret_cast<float*>(p.out)[o + 16 * m] = acc[m][n][i];
+        }
+      }
+    }
+}
+
+
+// All K blocks of one item; slot is the stage its first block reads.
+template <bool kGateUp, int NCOL>
+__device__ __forceinline__ void run_item(const GemvParams& p, const Walk& wk, const Item& it,
+                                         IssueCursor& ic, int& slot) {
+  float acc[2][2][4];
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
+  for (int blk = 0; blk < wk.nblk; ++blk) {
+    // refill the stage computed last (its reads are done), GV_STAGES - 1 blocks ahead
+    issue_next<kGateUp>(p, wk, ic, slot == 0 ? GV_STAGES - 1 : slot - 1);
+    cp_async_wait_ring();
+    __syncwarp();   // the scale bytes were copied by lanes 0-3
+    compute_block<NCOL>(wk.ring + slot * GV_STAGE_BYTES, acc, wk.lane);
+    __syncwarp();   // every lane is done with the stage before lanes 0-3 refill it
+    slot = slot == GV_STAGES - 1 ? 0 : slot + 1;
+  }
+  finish_item<kGateUp, NCOL>(p, it, acc, wk.lane);
+}
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(GV_THREADS, 1)
+    expert_gemv_fp8_kernel(const __grid_constant__ GemvParams p) {
+  constexpr int FEATS = kGateUp ? 16 : 32;
+  __shared__ int16_t units[GV_MAX_GROUPS + 1];   // prefix sums of the non-empty groups
+  extern __shared__ __align__(16) uint8_t ring[];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.E + p.S;
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < G; base += 32) {
+      const int g = base + lane;
+      int n = 0;
+      if (g < p.E) n = min(p.T, max(0, p.offsets[g + 1] - p.offsets[g]));
+      else if (g < G) n = p.T;
+      int incl = n > 0 ? 1 : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (g < G) units[g + 1] = int16_t(carry + incl);
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) units[0] = 0;
+  }
+  __syncthreads();
+
+  Walk wk;
+  wk.units = units;
+  wk.G = G;
+  wk.per_unit = p.n_out / FEATS;
+  wk.total = int(units[G]) * wk.per_unit;
+  wk.nblk = p.K / GV_KB;
+  wk.nwarps = int(gridDim.x) * GV_WARPS;
+  wk.lane = lane;
+  wk.ring = ring + size_t(warp) * GV_STAGES * GV_STAGE_BYTES;
+  wk.ring_s = smem_u32(wk.ring);
+
+  const int first = int(blockIdx.x) * GV_WARPS + warp;
+  IssueCursor ic;
+  ic.item = first;
+  cursor_at<kGateUp>(p, describe<kGateUp>(p, units, G, wk.per_unit, wk.total, first), ic, lane);
+  for (int s = 0; s < GV_STAGES - 1; ++s) issue_next<kGateUp>(p, wk, ic, s);
+
+  int slot = 0;
+  for (int item = first; item < wk.total; item += wk.nwarps) {
+    const Item it = describe<kGateUp>(p, units, G, wk.per_unit, wk.total, item);
+    if (it.nt > 8) run_item<kGateUp, 2>(p, wk, it, ic, slot);
+    else run_item<kGateUp, 1>(p, wk, it, ic, slot);
+  }
+  cp_async_wait_all();
+}
+
+template <bool kGateUp>
+cudaError_t launch_gemv(const GemvParams& gp, int num_sms, cudaStream_t st) {
+  static thread_local int attrs_device = -1;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (attrs_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(expert_gemv_fp8_kernel<kGateUp>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(GV_SMEM));
+    if (e != cudaSuccess) return e;
+    attrs_device = dev;
+  }
+  return launch_pdl(expert_gemv_fp8_kernel<kGateUp>, dim3(unsigned(num_sms)), dim3(GV_THREADS),
+                    GV_SMEM, st, 1, gp);
+}
+
+}  // namespace
+
+moe_status launch_expert_ffn_gemv_fp8(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
+                                      cudaStream_t st) {
+  if (a.T > GV_MAX_TOK) return MOE_ERR_INVALID_ARG;
+  const moe_fp8_expert_weights& R = *a.fp8_routed;
+  const moe_fp8_expert_weights& Sh = c.S > 0 ? *a.fp8_shared : R;   // unused when S == 0
+  GemvParams gp = {};
+  gp.w[0] = R.gate;
+  gp.s[0] = R.gate_scale;
+  gp.w[1] = R.up;
+  gp.s[1] = R.up_scale;
+  gp.sw[0] = Sh.gate;
+  gp.ss[0] = Sh.gate_scale;
+  gp.sw[1] = Sh.up;
+  gp.ss[1] = Sh.up_scale;
+  gp.tok_routed = a.x_perm;
+  gp.tok_shared = a.x;
+  gp.offsets = a.offsets;
+  gp.out = a.h_act;
+  gp.out_bf16 = 1;
+  gp.T = a.T;
+  gp.E = c.E;
+  gp.S = c.S;
+  gp.k = c.k;
+  gp.K = c.d;
+  gp.n_out = c.F;
+  if (launch_gemv<true>(gp, dev.num_sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (a.after_gate_up && cudaEventRecord(a.after_gate_up, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  GemvParams dp = {};
+  dp.w[0] = dp.w[1] = R.down;
+  dp.s[0] = dp.s[1] = R.down_scale;
+  dp.sw[0] = dp.sw[1] = Sh.down;
+  dp.ss[0] = dp.ss[1] = Sh.down_scale;
+  dp.tok_routed = a.h_act;
+  dp.tok_shared = a.h_act;
+  dp.offsets = a.offsets;
+  dp.out = a.Y;
+  dp.out_bf16 = a.y_bf16 ? 1 : 0;
+  dp.T = a.T;
+  dp.E = c.E;
+  dp.S = c.S;
+  dp.k = c.k;
+  dp.K = c.F;
+  dp.n_out = c.d;
+  if (launch_gemv<false>(dp, dev.num_sms, st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace moe

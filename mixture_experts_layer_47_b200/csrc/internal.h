@@ -184,5 +184,10 @@ moe_status launch_expert_ffn_swap(const Ctx& c, const FfnArgs& a, const DeviceIn
                                   bool pair, cudaStream_t st);
 moe_status launch_expert_ffn_fp8(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                                  cudaStream_t st);
+// FP8 expert FFNs on the CUDA cores (expert_gemv_fp8.cu), taken by launch_expert_ffn_fp8
+// for batches of at most kGemvMaxT tokens unless a weight-major tiling is asked for.
+constexpr int kGemvMaxT = 16;
+moe_status launch_expert_ffn_gemv_fp8(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
+                                      cudaStream_t st);
 
 }  // namespace moe

@@ -70,11 +70,20 @@ def test_measured_traffic_lookup_and_invalidation(tmp_path, monkeypatch):
                              "d_model": 6144, "d_ff": 2048},
         "gate_up_gemm/hbm/fp8": {"bound": "hbm", "bytes_per_touched_expert": 520,
                                  "kernel_source": "k.cu", "kernel_source_sha256": sha},
+        "gate_up_gemm/hbm/fp8_mma": {"bound": "hbm", "bytes_per_touched_expert": 530,
+                                     "kernel_source": "k.cu", "kernel_source_sha256": sha},
     }
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(table))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.delenv("MOE_GEMM_TILES", raising=False)
     assert bench.measured_traffic("gate_up_gemm", "hbm", 10) == 10000
-    assert bench.measured_traffic("gate_up_gemm", "hbm", 10, "fp8") == 5200
+    # FP8: the warp-MMA form's capture up to 16 tokens, the tcgen05 kernel's above or when a
+    # tiling is picked
+    assert bench.measured_traffic("gate_up_gemm", "hbm", 10, "fp8", T=16) == 5300
+    assert bench.measured_traffic("gate_up_gemm", "hbm", 10, "fp8", T=256) == 5200
+    monkeypatch.setenv("MOE_GEMM_TILES", "swap")
+    assert bench.measured_traffic("gate_up_gemm", "hbm", 10, "fp8", T=16) == 5200
+    monkeypatch.delenv("MOE_GEMM_TILES")
     assert bench.measured_traffic("gate_up_gemm", "tensor", 10) is None   # no entry
     assert bench.measured_traffic("down_gemm", "hbm", 10) is None
     assert bench.measured_traffic("gate_up_gemm", "hbm", 1, "bf16", 6144, 18432) is None

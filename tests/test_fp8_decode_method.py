@@ -88,3 +88,52 @@ def test_the_workload_checkpoint_stays_inside_the_contract():
     for t in (routed.gate, routed.up, routed.down):
         c = t.numpy()
         assert not np.any((c & 0x7F) == 0x7F)    # no NaN codes
+
+
+def prmt(a: int, b: int, sel: int) -> int:
+    """PRMT in its default mode: result byte i is byte (nibble i of sel) & 7 of the eight
+    bytes b:a (a bytes 0-3, b bytes 4-7); bit 3 of the nibble replicates that byte's sign."""
+    src = (b << 32) | a
+    out = 0
+    for i in range(4):
+        nib = (sel >> (4 * i)) & 0xF
+        byte = (src >> (8 * (nib & 7))) & 0xFF
+        if nib & 8:
+            byte = 0xFF if byte & 0x80 else 0x00
+        out |= byte << (8 * i)
+    return out
+
+
+def word_planes(w: int):
+    """The word-level decoder's integer steps: byte planes of the low and high bf16 bytes,
+    interleaved into the pairs (code 0, code 1) and (code 2, code 3)."""
+    lo = (w << 4) & 0xF0F0F0F0
+    hi = ((w >> 4) & 0x07070707) | (w & 0x80808080)
+    return prmt(lo, hi, 0x5140), prmt(lo, hi, 0x7362)
+
+
+def pair_bits(w: int, sel: int) -> int:
+    """The pair decoder's integer steps: PRMT of two code bytes to bits 8-15 and 24-31 (zero
+    elsewhere), magnitude shifted down by 4, sign kept."""
+    x8 = prmt(w, 0, sel)
+    return ((x8 >> 4) & 0x07F007F0) | (x8 & 0x80008000)
+
+
+def test_word_decoder_places_every_code_like_the_pair_decoder():
+    """Both integer routes give, for every code in every byte position of a word, the bf16
+    half whose bits read as code * 2^-120 (the bit placement pinned above), so the one bf16
+    multiply that follows gives the same exact weights."""
+    rng = np.random.default_rng(11)
+    words = [int(c) * 0x01010101 for c in range(256)]
+    words += [int(v) for v in rng.integers(0, 2 ** 32, size=4096, dtype=np.uint64)]
+    for pos in range(4):                       # each code once in each byte, others random
+        for c in range(256):
+            words.append((int(rng.integers(0, 2 ** 32)) & ~(0xFF << (8 * pos)) | (c << (8 * pos)))
+                         & 0xFFFFFFFF)
+    for w in words:
+        p01, p23 = word_planes(w)
+        assert p01 == pair_bits(w, 0x1404) and p23 == pair_bits(w, 0x3424), hex(w)
+        codes = [(w >> (8 * i)) & 0xFF for i in range(4)]
+        halves = [p01 & 0xFFFF, p01 >> 16, p23 & 0xFFFF, p23 >> 16]
+        for c, h in zip(codes, halves):
+            assert h == ((c & 0x7F) << 4) | ((c & 0x80) << 8), (hex(w), hex(c), hex(h))

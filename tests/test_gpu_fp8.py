@@ -4,8 +4,11 @@ The reference is the fp64 oracle run on the decoded FP8 weights (oracle.fp8_inpu
 E4M3 codes decoded from the format definition, times the block scales).  Shapes span
 several tiles and ragged tails: d and d_ff that are not multiples of the 128- to
 512-feature weight tiles, groups that are not multiples of the 16-token N step, more
-than one token tile per group, two shared experts and none.  Both forms of the FP8
-kernel run: the 1-SM form (the default) and the 2-SM pair (MOE_GEMM_TILES=swap_pair).
+than one token tile per group, two shared experts and none.  Every form of the FP8 path
+runs: the tensor-core kernel's 1-SM form (MOE_GEMM_TILES=swap, and the default above 16
+tokens) and 2-SM pair (MOE_GEMM_TILES=swap_pair), and the CUDA-core form the default takes
+at up to 16 tokens, whose shapes add K lengths that leave part of the 512-wide K step
+empty and groups of 1 to 4 tokens plus groups that take several 4-token passes.
 """
 import numpy as np
 import pytest
@@ -25,7 +28,13 @@ FP8_SHAPES = [  # T, d, E, k, F, S, bias_scale
     (300, 192, 64, 8, 192, 1, 0.5),
     (600, 256, 4, 2, 128, 1, 0.0),     # ~300 rows per expert: three token tiles each
     (40, 256, 8, 8, 128, 0, 0.0),      # k == E, no shared expert
+    # up to 16 tokens: the default takes the CUDA-core form
+    (16, 320, 5, 3, 384, 2, 0.0),      # K = 320 and 384: part of the 512-wide K step empty
+    (1, 64, 1, 1, 64, 0, 0.0),         # one token, one expert, the smallest shape
+    (12, 192, 64, 8, 192, 1, 0.5),     # most groups empty or of one token
+    (13, 128, 2, 1, 128, 1, 0.0),      # groups of 4, 4, 4 and 1 (shared) tokens and ragged ones
 ]
+GEMV_SHAPES = [s for s in FP8_SHAPES if s[0] <= 16]
 
 
 def _ids(shapes):
@@ -54,12 +63,16 @@ def _forward_fp8(dev: Inputs, routed, shared):
     return y.cpu(), {k: v.cpu() for k, v in moe.workspace_views(h, wl.T, ws).items()}
 
 
-FORMS = ["pair", "swap"]
+FORMS = ["pair", "swap", "auto"]
 
 
 def _form(form, monkeypatch):
+    """pair: the tensor-core kernel's 2-SM form; swap: its 1-SM form; auto: the default
+    (the CUDA-core form at up to 16 tokens, else the 1-SM tensor-core form)."""
     if form == "pair":
         monkeypatch.setenv("MOE_GEMM_TILES", "swap_pair")
+    elif form == "swap":
+        monkeypatch.setenv("MOE_GEMM_TILES", "swap")
     else:
         monkeypatch.delenv("MOE_GEMM_TILES", raising=False)
 
@@ -113,7 +126,8 @@ def test_fp8_forward_matches_oracle(shape, form, monkeypatch):
     assert rel_err(y.float().numpy(), ref["y"]) < Y_REL_TOL
 
 
-@pytest.mark.parametrize("shape", FP8_SHAPES[1:5], ids=_ids(FP8_SHAPES[1:5]))
+@pytest.mark.parametrize("shape", FP8_SHAPES[1:5] + GEMV_SHAPES[:1],
+                         ids=_ids(FP8_SHAPES[1:5] + GEMV_SHAPES[:1]))
 def test_fp8_path_equals_bf16_path_on_decoded_weights(shape, monkeypatch):
     """The FP8 kernels decode each weight exactly and then run the MMAs of the 1-SM
     weight-major bf16 kernel in the same order, so on the decoded weights the two GPU
@@ -208,19 +222,86 @@ def test_fp8_special_codes_decode_exactly(monkeypatch):
 
 
 @pytest.mark.parametrize("name", ["decode_fp8"])
-def test_fp8_pair_and_single_forms_agree_at_full_size(name, monkeypatch):
-    """The 2-SM and 1-SM FP8 kernels on the Hy4 decode workload: the same routing and
-    outputs within the layer's tolerance of each other (the pair's M = 256 MMAs may order
-    the tensor core's partial sums differently from two M = 128 ones)."""
+def test_fp8_forms_agree_at_full_size(name, monkeypatch):
+    """The three FP8 forms on the Hy4 decode workload: the same routing, and the 2-SM
+    tensor-core kernel and the CUDA-core form (the default at 16 tokens) each within the
+    layer's tolerance of the 1-SM tensor-core kernel (the pair's M = 256 MMAs and the
+    CUDA cores' lane-by-lane sums may order the fp32 additions differently)."""
     wl = WORKLOADS[name]
     inp = make_inputs(wl, device="cuda")
     routed, shared = make_fp8(inp)
-    monkeypatch.setenv("MOE_GEMM_TILES", "swap_pair")
-    y_pair, v_pair = _forward_fp8(inp, routed, shared)
+    out = {}
+    for form in FORMS:
+        _form(form, monkeypatch)
+        out[form] = _forward_fp8(inp, routed, shared)
+    y_one, v_one = out["swap"]
+    for form in ("pair", "auto"):
+        y, v = out[form]
+        assert torch.equal(v["topk_idx"], v_one["topk_idx"])
+        err = rel_err(y.float().numpy(), y_one.float().numpy())
+        same = torch.equal(y.view(torch.int16), y_one.view(torch.int16))
+        print(f"{name}: {form} vs 1-SM FP8 rel diff {err:.3e}, bit-identical {same}")
+        assert err < Y_REL_TOL
+
+
+def _bf16_ulps(a: torch.Tensor, b: torch.Tensor) -> torch.Tensor:
+    """Distance in bf16 steps between two bf16 tensors of finite values (sign-magnitude
+    bit patterns mapped to a monotone integer line)."""
+    def line(t):
+        i = t.view(torch.int16).to(torch.int32)
+        return torch.where(i < 0, -(i & 0x7FFF), i)
+    return (line(a) - line(b)).abs()
+
+
+@pytest.mark.parametrize("shape", GEMV_SHAPES, ids=_ids(GEMV_SHAPES))
+def test_fp8_gemv_matches_tensor_core_form(shape, monkeypatch):
+    """The CUDA-core form forms the same exact bf16 x bf16 products as the tensor-core
+    kernel and adds them in fp32 in another order, so on the same dispatch its fp32 sums
+    differ from the tensor core's by a few fp32 rounding steps: every bf16 activation is the
+    tensor-core one or its neighbour, nearly all are equal, and the fp32 Y rows agree to far
+    within the layer's tolerance."""
+    T, d, E, k, F, S, bs = shape
+    inp = make_small(T, d, E, k, F, S, seed=1700 + T, bias_scale=bs)
+    routed, shared = make_fp8(inp)
+    logits = oracle.router_logits(inp.x, inp.W_router, inp.bias)
+    idx, _, _ = oracle.route(logits, k)
+    _, offsets, perm, _ = oracle.dispatch(idx, E)
+    rows = T * k + S * T
+    res = {}
+    for form in ("swap", "auto"):
+        _form(form, monkeypatch)
+        h = moe.moe_create(d, E, k, F, S)
+        ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
+        Y = torch.full((rows, d), float("nan"), dtype=torch.float32, device="cuda")
+        moe.moe_expert_ffn_fp8(h, inp.x.cuda(), torch.from_numpy(perm).cuda(),
+                               torch.from_numpy(offsets).cuda(), routed.to("cuda"),
+                               shared.to("cuda"), Y, ws)
+        assert moe.moe_device_status(h, T, ws)[0] == moe.MOE_OK
+        res[form] = (moe.workspace_views(h, T, ws)["h_act"][:rows].cpu(), Y.cpu())
+    (h_tc, y_tc), (h_cc, y_cc) = res["swap"], res["auto"]
+    ulps = _bf16_ulps(h_cc, h_tc)
+    assert int(ulps.max()) <= 1, int(ulps.max())
+    assert float((ulps > 0).float().mean()) < 0.02
+    assert torch.isfinite(y_cc).all()
+    assert rel_err(y_cc.numpy(), y_tc.numpy()) < 1e-3
+
+
+def test_fp8_gemv_special_codes(monkeypatch):
+    """The special codes and the largest scale byte of test_fp8_special_codes_decode_exactly
+    through the CUDA-core form (16 tokens): within the layer's tolerance of the oracle on
+    the decoded weights."""
+    T, d, E, k, F, S = 16, 256, 4, 2, 128, 1
+    inp = make_small(T, d, E, k, F, S, seed=37)
+    routed, shared = make_fp8(inp)
+    g = torch.Generator().manual_seed(6)
+    codes = torch.tensor(SPECIAL_CODES, dtype=torch.uint8)
+    for t in (routed.gate, routed.up, routed.down, shared.gate, shared.up, shared.down):
+        flat = t.view(-1)
+        where = torch.randint(0, flat.numel(), (4096,), generator=g)
+        flat[where] = codes[torch.randint(0, len(SPECIAL_CODES), (4096,), generator=g)]
+    routed.gate_scale[0, 0, :8] = 134
+    shared.down_scale[0, 0, :8] = 134
     monkeypatch.delenv("MOE_GEMM_TILES", raising=False)
-    y_one, v_one = _forward_fp8(inp, routed, shared)
-    assert torch.equal(v_pair["topk_idx"], v_one["topk_idx"])
-    err = rel_err(y_pair.float().numpy(), y_one.float().numpy())
-    same = torch.equal(y_pair.view(torch.int16), y_one.view(torch.int16))
-    print(f"{name}: pair vs 1-SM FP8 rel diff {err:.3e}, bit-identical {same}")
-    assert err < Y_REL_TOL
+    y8, v8 = _forward_fp8(to_device(inp, "cuda"), routed.to("cuda"), shared.to("cuda"))
+    ref = oracle.forward(decoded_inputs(inp, routed, shared), idx_override=v8["topk_idx"].numpy())
+    assert rel_err(y8.float().numpy(), ref["y"]) < Y_REL_TOL
