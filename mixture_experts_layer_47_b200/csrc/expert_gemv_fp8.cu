@@ -13,10 +13,15 @@
 // bf16x2 multiplies), with the multiply-adds done by warp-level m16n8k16 bf16 MMAs on the
 // decoded registers.
 //
-// Work: a warp item is 16 feature rows of one group -- the gate and the up rows of 16
-// features, or 32 consecutive W_down rows as two 16-row tiles -- for all of the group's
-// tokens (one MMA column block of 8 tokens, two when the group has more than 8).  The
-// grid's warps take items round robin; an item walks K in blocks of 64.
+// Work: an item is 16 feature rows of one group -- the gate and the up rows of 16 features,
+// or 32 consecutive W_down rows as two 16-row tiles -- for all of the group's tokens (one MMA
+// column block of 8 tokens, two when the group has more than 8), walked in K blocks of 64.
+// A CTA takes items round robin (about 90 per CTA at Hy4 decode); their K blocks are its
+// jobs, cut into equal runs for its 8 warps, so every warp has the same number of blocks
+// (taking whole items per warp left a tail of up to 9%).  A warp finishes an item it ran
+// whole from its registers; an item cut between warps leaves each warp's partial sums in
+// shared memory, and the last of its warps to arrive (a shared-memory counter, no waiting)
+// adds the parts in warp order and finishes it.
 // Fragments: in an m16n8k16 MMA lane l = 4 g + t holds A rows g and g + 8 at k slots
 // {2t, 2t+1, 2t+8, 2t+9} and B (token g) at the same slots.  The sum over k does not care
 // which K position a slot stands for, so in K block kb, MMA s (0..3), the slots of lane t
@@ -24,13 +29,12 @@
 // 16-byte load) and its 16 consecutive activations (32 bytes) feed all four MMAs of the
 // block, and each 32-wide scale block lies inside one lane's run.
 // Stream: each lane copies its rows' codes and its tokens' activations for a block with
-// cp.async into a per-warp 6-stage ring in shared memory, five blocks ahead of the block it
-// computes (the ring runs on across item boundaries; the lane keeps running source pointers),
-// so the loads in flight hold no registers; four lanes also copy the tiles' 16 scale bytes
-// per 32-wide K block, read by all lanes after the ring wait and a warp barrier.  One CTA of
-// 8 warps per SM: measured on B200 at Hy4 decode, 8 warps with 6 stages beat 10 x 4, 12 x 4
-// and 16 x 3 (gate/up 0.523 against 0.55-0.58 ms; the deeper ring keeps more of the HBM
-// stream in flight per warp).
+// cp.async into a per-warp 5-stage ring in shared memory, four blocks ahead of the block it
+// computes (the ring runs on across items; the lane keeps running source pointers), so the
+// loads in flight hold no registers; four lanes also copy the tiles' 16 scale bytes per
+// 32-wide K block, read by all lanes after the ring wait and a warp barrier.  Measured on
+// B200 at Hy4 decode: 8 warps with deep rings beat 10 x 4, 12 x 4 and 16 x 3 stages, and the
+// even cut of the jobs gained 7% on gate/up over whole items per warp.
 // Arithmetic: exact bf16 weights (the decoder of the tensor-core FP8 kernel) times bf16
 // activations into fp32 accumulators, as in the tensor-core path; only the order of the
 // fp32 additions differs.  The epilogue applies SwiGLU (gate/up) from registers: a lane's
@@ -46,7 +50,7 @@ namespace {
 constexpr int GV_WARPS = 8;
 constexpr int GV_THREADS = 32 * GV_WARPS;
 constexpr int GV_KB = 64;                        // K per block (4 MMAs)
-constexpr int GV_STAGES = 6;
+constexpr int GV_STAGES = 5;
 constexpr int GV_MAX_GROUPS = 1024 + 8;          // E + S upper bound
 constexpr int GV_MAX_TOK = 16;                   // tokens per group: two 8-token MMA columns
 // Per warp and stage: codes [tile 2][row half 2][lane 32][16 B], activations
@@ -55,7 +59,9 @@ constexpr int GV_CODE_OFF = 0;
 constexpr int GV_X_OFF = 2 * 2 * 32 * 16;
 constexpr int GV_SCALE_OFF = GV_X_OFF + 2 * 32 * 32;
 constexpr int GV_STAGE_BYTES = GV_SCALE_OFF + 2 * 2 * 16;
-constexpr size_t GV_SMEM = size_t(GV_WARPS) * GV_STAGES * GV_STAGE_BYTES;
+constexpr int GV_RING_BYTES = GV_WARPS * GV_STAGES * GV_STAGE_BYTES;
+// After the rings: the partial sums of cut items, [warp][slot 2][value 16][lane 32].
+constexpr size_t GV_SMEM = size_t(GV_RING_BYTES) + size_t(GV_WARPS) * 2 * 16 * 32 * sizeof(float);
 static_assert(GV_STAGE_BYTES % 16 == 0, "stages stay 16-byte aligned");
 
 struct GemvParams {
@@ -138,46 +144,68 @@ __device__ __forceinline__ Item describe(const GemvParams& p, const int16_t* uni
   return it;
 }
 
-// What the loop over items needs besides the parameters.
+// What the loop over items needs besides the parameters.  A CTA takes items blockIdx.x,
+// blockIdx.x + gridDim.x, ...; their K blocks, in order, are its jobs, and warp w takes the
+// jobs [jw, jw+1) with jw = w * jobs / GV_WARPS, so an item may be cut between warps.
 struct Walk {
   const int16_t* units;
-  int G, per_unit, total, nblk, nwarps, lane;
+  int G, per_unit, total, nblk, jobs, lane;
+  int j0, j1;          // this warp's jobs
   uint8_t* ring;       // this warp's GV_STAGES stages
   uint32_t ring_s;     // the same, as a shared-memory address
 };
 
-// The copies run GV_STAGES - 1 blocks ahead of the arithmetic, across item boundaries.  The
-// cursor keeps this lane's source pointers for its next block: codes of rows g and g + 8
-// of both tiles, the activations of tokens g and g + 8, and (lanes 0-3) a scale row.
+__device__ __forceinline__ int warp_first_job(int jobs, int w) { return w * jobs / GV_WARPS; }
+
+// The warp whose jobs hold job j.
+__device__ __forceinline__ int warp_of_job(int jobs, int j) {
+  int w = 0;
+#pragma unroll
+  for (int v = 1; v < GV_WARPS; ++v)
+    if (warp_first_job(jobs, v) <= j) w = v;
+  return w;
+}
+
+// The copies run GV_STAGES - 1 blocks ahead of the arithmetic, across items.  The cursor
+// keeps this lane's source pointers for its next job: codes of rows g and g + 8 of both
+// tiles, the activations of tokens g and g + 8, and (lanes 0-3) a scale row.
 struct IssueCursor {
   const uint8_t* code[4];   // [tile m * 2 + row half h]
   const uint16_t* x[2];     // [column block n]
   const uint8_t* scale;     // lane 2 m + b < 4: tile m's scales of 32-wide block 2 blk + b
-  int item, blk, nt;        // nt = 0 past the last item
+  int job, blk, nt;         // nt = 0 when this warp's jobs are all issued
 };
 
+// The cursor at block blk of an item.
 template <bool kGateUp>
-__device__ __forceinline__ void cursor_at(const GemvParams& p, const Item& it, IssueCursor& ic,
-                                          int lane) {
+__device__ __forceinline__ void cursor_at(const GemvParams& p, const Item& it, int blk,
+                                          IssueCursor& ic, int lane) {
   ic.nt = it.nt;
-  ic.blk = 0;
+  ic.blk = blk;
   if (it.nt == 0) return;
   const int g = lane >> 2, t = lane & 3;
+  const int k0 = blk * GV_KB + 16 * t;
 #pragma unroll
   for (int m = 0; m < 2; ++m) {
     const uint8_t* base = (it.shared ? p.sw[kGateUp ? m : 0] : p.w[kGateUp ? m : 0]) + it.woff +
-                          size_t(kGateUp ? 0 : 16 * m) * p.K + 16 * t;
+                          size_t(kGateUp ? 0 : 16 * m) * p.K + k0;
 #pragma unroll
     for (int h = 0; h < 2; ++h) ic.code[m * 2 + h] = base + size_t(g + 8 * h) * p.K;
   }
 #pragma unroll
-  for (int n = 0; n < 2; ++n) ic.x[n] = it.tok + size_t(g + 8 * n) * p.K + 16 * t;
+  for (int n = 0; n < 2; ++n) ic.x[n] = it.tok + size_t(g + 8 * n) * p.K + k0;
   const int m = (lane >> 1) & 1, b = lane & 1;
   ic.scale = (it.shared ? p.ss[kGateUp ? m : 0] : p.s[kGateUp ? m : 0]) + it.soff +
-             (kGateUp ? 0 : 16 * m) + size_t(b) * p.n_out;
+             (kGateUp ? 0 : 16 * m) + size_t(2 * blk + b) * p.n_out;
 }
 
-// Copies of the cursor's block into a stage, then the cursor moves one block on.
+template <bool kGateUp>
+__device__ __forceinline__ Item job_item(const GemvParams& p, const Walk& wk, int q) {
+  return describe<kGateUp>(p, wk.units, wk.G, wk.per_unit, wk.total,
+                           int(blockIdx.x) + q * int(gridDim.x));
+}
+
+// Copies of the cursor's job into a stage, then the cursor moves one job on.
 template <bool kGateUp>
 __device__ __forceinline__ void issue_next(const GemvParams& p, const Walk& wk, IssueCursor& ic,
                                            int slot) {
@@ -200,13 +228,13 @@ __device__ __forceinline__ void issue_next(const GemvParams& p, const Walk& wk, 
     }
     if (lane < 4) cp_async16(stage + uint32_t(GV_SCALE_OFF + lane * 16), ic.scale);
     ic.scale += size_t(2) * p.n_out;
+    if (++ic.job == wk.j1) {
+      ic.nt = 0;
+    } else if (++ic.blk == wk.nblk) {
+      cursor_at<kGateUp>(p, job_item<kGateUp>(p, wk, ic.job / wk.nblk), 0, ic, lane);
+    }
   }
   cp_async_commit();
-  if (++ic.blk == wk.nblk) {
-    ic.item += wk.nwarps;
-    cursor_at<kGateUp>(p, describe<kGateUp>(p, wk.units, wk.G, wk.per_unit, wk.total, ic.item),
-                       ic, lane);
-  }
 }
 
 // The four MMAs of one K block for NCOL 8-token column blocks.  The activation columns of
@@ -281,10 +309,17 @@ __device__ __forceinline__ void finish_item(const GemvParams& p, const Item& it,
 }
 
 
-// All K blocks of one item; slot is the stage its first block reads.
+// After an item's last block the lanes hold (or, for an item cut between warps, the summed
+// parts give) element i of column block n = (row g + 8 (i / 2), token 8 n + 2 t + i % 2)
+// of both tiles.
+// This warp's jobs of one item, blocks [blk0, blk0 + nb); slot is the stage the first one
+// reads.  A whole item is finished from the registers.  A part of a cut item goes to this
+// warp's partial slot (0: the item began before this warp's jobs, 1: it runs past them);
+// the last of the item's warps to arrive adds the parts in warp order and finishes it.
 template <bool kGateUp, int NCOL>
-__device__ __forceinline__ void run_item(const GemvParams& p, const Walk& wk, const Item& it,
-                                         IssueCursor& ic, int& slot) {
+__device__ __forceinline__ void run_segment(const GemvParams& p, const Walk& wk, const Item& it,
+                                            int q, int blk0, int nb, IssueCursor& ic, int& slot,
+                                            float* part, int* cut_count, int warp) {
   float acc[2][2][4];
 #pragma unroll
   for (int m = 0; m < 2; ++m)
@@ -292,8 +327,8 @@ __device__ __forceinline__ void run_item(const GemvParams& p, const Walk& wk, co
     for (int n = 0; n < 2; ++n)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
-  for (int blk = 0; blk < wk.nblk; ++blk) {
-    // refill the stage computed last (its reads are done), GV_STAGES - 1 blocks ahead
+  for (int b = 0; b < nb; ++b) {
+    // refill the stage computed last (its reads are done), GV_STAGES - 1 jobs ahead
     issue_next<kGateUp>(p, wk, ic, slot == 0 ? GV_STAGES - 1 : slot - 1);
     cp_async_wait_ring();
     __syncwarp();   // the scale bytes were copied by lanes 0-3
@@ -301,7 +336,51 @@ __device__ __forceinline__ void run_item(const GemvParams& p, const Walk& wk, co
     __syncwarp();   // every lane is done with the stage before lanes 0-3 refill it
     slot = slot == GV_STAGES - 1 ? 0 : slot + 1;
   }
-  finish_item<kGateUp, NCOL>(p, it, acc, wk.lane);
+  if (blk0 == 0 && nb == wk.nblk) {
+    finish_item<kGateUp, NCOL>(p, it, acc, wk.lane);
+    return;
+  }
+  const int lane = wk.lane;
+  const int first_job = q * wk.nblk;
+  float* mine = part + ((warp * 2 + (first_job < wk.j0 ? 0 : 1)) * 16) * 32;
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mine[(8 * m + 4 * n + i) * 32 + lane] = acc[m][n][i];
+  __threadfence_block();
+  __syncwarp();
+  // the item's parts: the warps from w_first to w_last that have jobs (with fewer jobs than
+  // warps, some warps have none)
+  const int w_first = warp_of_job(wk.jobs, first_job);
+  const int w_last = warp_of_job(wk.jobs, first_job + wk.nblk - 1);
+  int parts = 0;
+  for (int w = w_first; w <= w_last; ++w)
+    parts += warp_first_job(wk.jobs, w + 1) > warp_first_job(wk.jobs, w) ? 1 : 0;
+  int arrived = 0;
+  if (lane == 0) arrived = atomicAdd(cut_count + w_first, 1);
+  arrived = __shfl_sync(0xffffffffu, arrived, 0);
+  if (arrived != parts - 1) return;   // another part is still running
+  __threadfence_block();
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
+  for (int w = w_first; w <= w_last; ++w) {
+    const int jw = warp_first_job(wk.jobs, w);
+    if (warp_first_job(wk.jobs, w + 1) == jw) continue;   // no jobs, no part
+    const float* src = part + ((w * 2 + (first_job < jw ? 0 : 1)) * 16) * 32;
+#pragma unroll
+    for (int m = 0; m < 2; ++m)
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[m][n][i] += src[(8 * m + 4 * n + i) * 32 + lane];
+  }
+  finish_item<kGateUp, NCOL>(p, it, acc, lane);
 }
 
 template <bool kGateUp>
@@ -309,7 +388,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     expert_gemv_fp8_kernel(const __grid_constant__ GemvParams p) {
   constexpr int FEATS = kGateUp ? 16 : 32;
   __shared__ int16_t units[GV_MAX_GROUPS + 1];   // prefix sums of the non-empty groups
-  extern __shared__ __align__(16) uint8_t ring[];
+  __shared__ int cut_count[GV_WARPS];            // arrivals at each cut item, by its first warp
+  extern __shared__ __align__(16) uint8_t smem[];
   pdl_wait();
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -331,6 +411,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) units[0] = 0;
+    if (lane < GV_WARPS) cut_count[lane] = 0;
   }
   __syncthreads();
 
@@ -340,22 +421,31 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
   wk.per_unit = p.n_out / FEATS;
   wk.total = int(units[G]) * wk.per_unit;
   wk.nblk = p.K / GV_KB;
-  wk.nwarps = int(gridDim.x) * GV_WARPS;
+  const int n_items = int(blockIdx.x) < wk.total
+                          ? (wk.total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
+  wk.jobs = n_items * wk.nblk;
+  wk.j0 = warp_first_job(wk.jobs, warp);
+  wk.j1 = warp_first_job(wk.jobs, warp + 1);
   wk.lane = lane;
-  wk.ring = ring + size_t(warp) * GV_STAGES * GV_STAGE_BYTES;
+  wk.ring = smem + size_t(warp) * GV_STAGES * GV_STAGE_BYTES;
   wk.ring_s = smem_u32(wk.ring);
+  float* part = reinterpret_cast<float*>(smem + GV_RING_BYTES);
 
-  const int first = int(blockIdx.x) * GV_WARPS + warp;
   IssueCursor ic;
-  ic.item = first;
-  cursor_at<kGateUp>(p, describe<kGateUp>(p, units, G, wk.per_unit, wk.total, first), ic, lane);
+  ic.job = wk.j0;
+  ic.nt = 0;
+  if (wk.j0 < wk.j1)
+    cursor_at<kGateUp>(p, job_item<kGateUp>(p, wk, wk.j0 / wk.nblk), wk.j0 % wk.nblk, ic, lane);
   for (int s = 0; s < GV_STAGES - 1; ++s) issue_next<kGateUp>(p, wk, ic, s);
 
   int slot = 0;
-  for (int item = first; item < wk.total; item += wk.nwarps) {
-    const Item it = describe<kGateUp>(p, units, G, wk.per_unit, wk.total, item);
-    if (it.nt > 8) run_item<kGateUp, 2>(p, wk, it, ic, slot);
-    else run_item<kGateUp, 1>(p, wk, it, ic, slot);
+  for (int j = wk.j0; j < wk.j1;) {
+    const int q = j / wk.nblk, blk0 = j - q * wk.nblk;
+    const int nb = min(wk.j1, (q + 1) * wk.nblk) - j;
+    const Item it = job_item<kGateUp>(p, wk, q);
+    if (it.nt > 8) run_segment<kGateUp, 2>(p, wk, it, q, blk0, nb, ic, slot, part, cut_count, warp);
+    else run_segment<kGateUp, 1>(p, wk, it, q, blk0, nb, ic, slot, part, cut_count, warp);
+    j += nb;
   }
   cp_async_wait_all();
 }
