@@ -535,8 +535,8 @@ bool encode_set(CUtensorMap* codes, CUtensorMap* scales, const uint8_t* c, const
 
 moe_status launch_expert_ffn_fp8(const Ctx& c, const FfnArgs& a, const DeviceInfo& dev,
                                  cudaStream_t st) {
-  // Decode-size batches go to the CUDA-core form: a tensor-core MMA over 16 tokens costs
-  // about as much as the bf16 weights' HBM time, twice the FP8 codes'.
+  // Decode-size batches go to the warp-MMA form (expert_gemv_fp8.cu): this kernel's MMAs over
+  // 16-32 token tiles cost about as much as the bf16 weights' HBM time, twice the FP8 codes'.
   if (a.T <= kGemvMaxT && c.tiles == TilesMode::kAuto) return launch_expert_ffn_gemv_fp8(c, a, dev, st);
   if (!tensor_map_encoder()) return MOE_ERR_CUDA;
   const moe_fp8_expert_weights& R = *a.fp8_routed;

@@ -5,10 +5,10 @@ E4M3 codes decoded from the format definition, times the block scales).  Shapes 
 several tiles and ragged tails: d and d_ff that are not multiples of the 128- to
 512-feature weight tiles, groups that are not multiples of the 16-token N step, more
 than one token tile per group, two shared experts and none.  Every form of the FP8 path
-runs: the tensor-core kernel's 1-SM form (MOE_GEMM_TILES=swap, and the default above 16
-tokens) and 2-SM pair (MOE_GEMM_TILES=swap_pair), and the CUDA-core form the default takes
-at up to 16 tokens, whose shapes add K lengths that leave part of the 512-wide K step
-empty and groups of 1 to 4 tokens plus groups that take several 4-token passes.
+runs: the tcgen05 kernel's 1-SM form (MOE_GEMM_TILES=swap, and the default above 16
+tokens) and 2-SM pair (MOE_GEMM_TILES=swap_pair), and the warp-MMA form the default takes
+at up to 16 tokens, whose shapes add K lengths of fewer 64-wide blocks than a CTA has warps,
+groups of 1 to 8 tokens (one MMA column block) and of 9 to 16 (two).
 """
 import numpy as np
 import pytest
@@ -28,11 +28,11 @@ FP8_SHAPES = [  # T, d, E, k, F, S, bias_scale
     (300, 192, 64, 8, 192, 1, 0.5),
     (600, 256, 4, 2, 128, 1, 0.0),     # ~300 rows per expert: three token tiles each
     (40, 256, 8, 8, 128, 0, 0.0),      # k == E, no shared expert
-    # up to 16 tokens: the default takes the CUDA-core form
-    (16, 320, 5, 3, 384, 2, 0.0),      # K = 320 and 384: part of the 512-wide K step empty
-    (1, 64, 1, 1, 64, 0, 0.0),         # one token, one expert, the smallest shape
+    # up to 16 tokens: the default takes the warp-MMA form
+    (16, 320, 5, 3, 384, 2, 0.0),      # K = 320 and 384: 5 and 6 blocks of 64 for 8 warps
+    (1, 64, 1, 1, 64, 0, 0.0),         # one token, one expert, one K block: the smallest shape
     (12, 192, 64, 8, 192, 1, 0.5),     # most groups empty or of one token
-    (13, 128, 2, 1, 128, 1, 0.0),      # groups of 4, 4, 4 and 1 (shared) tokens and ragged ones
+    (13, 128, 2, 1, 128, 1, 0.0),      # routed groups of 6-7 tokens, the shared one of 13 (two column blocks)
 ]
 GEMV_SHAPES = [s for s in FP8_SHAPES if s[0] <= 16]
 
@@ -68,7 +68,7 @@ FORMS = ["pair", "swap", "auto"]
 
 def _form(form, monkeypatch):
     """pair: the tensor-core kernel's 2-SM form; swap: its 1-SM form; auto: the default
-    (the CUDA-core form at up to 16 tokens, else the 1-SM tensor-core form)."""
+    (the warp-MMA form at up to 16 tokens, else the tcgen05 kernel's 1-SM form)."""
     if form == "pair":
         monkeypatch.setenv("MOE_GEMM_TILES", "swap_pair")
     elif form == "swap":
@@ -224,7 +224,7 @@ def test_fp8_special_codes_decode_exactly(monkeypatch):
 @pytest.mark.parametrize("name", ["decode_fp8"])
 def test_fp8_forms_agree_at_full_size(name, monkeypatch):
     """The three FP8 forms on the Hy4 decode workload: the same routing, and the 2-SM
-    tensor-core kernel and the CUDA-core form (the default at 16 tokens) each within the
+    tcgen05 kernel and the warp-MMA form (the default at 16 tokens) each within the
     layer's tolerance of the 1-SM tensor-core kernel (the pair's M = 256 MMAs and the
     CUDA cores' lane-by-lane sums may order the fp32 additions differently)."""
     wl = WORKLOADS[name]
@@ -255,7 +255,7 @@ def _bf16_ulps(a: torch.Tensor, b: torch.Tensor) -> torch.Tensor:
 
 @pytest.mark.parametrize("shape", GEMV_SHAPES, ids=_ids(GEMV_SHAPES))
 def test_fp8_gemv_matches_tensor_core_form(shape, monkeypatch):
-    """The CUDA-core form forms the same exact bf16 x bf16 products as the tensor-core
+    """The warp-MMA form forms the same exact bf16 x bf16 products as the tcgen05
     kernel and adds them in fp32 in another order, so on the same dispatch its fp32 sums
     differ from the tensor core's by a few fp32 rounding steps: every bf16 activation is the
     tensor-core one or its neighbour, nearly all are equal, and the fp32 Y rows agree to far
@@ -288,7 +288,7 @@ def test_fp8_gemv_matches_tensor_core_form(shape, monkeypatch):
 
 def test_fp8_gemv_special_codes(monkeypatch):
     """The special codes and the largest scale byte of test_fp8_special_codes_decode_exactly
-    through the CUDA-core form (16 tokens): within the layer's tolerance of the oracle on
+    through the warp-MMA form (16 tokens): within the layer's tolerance of the oracle on
     the decoded weights."""
     T, d, E, k, F, S = 16, 256, 4, 2, 128, 1
     inp = make_small(T, d, E, k, F, S, seed=37)
