@@ -25,9 +25,11 @@
 //   2-SM (kPair = true): a CTA pair runs tcgen05.mma.cta_group::2 with M = 256
 //     weight rows (128 per CTA) and a token tile of N <= 256 whose rows are
 //     split between the two CTAs' shared memory --
-//       gate/up  a gate MMA and an up MMA per K step, accumulators at TMEM
-//                columns [0, N) and [256, 256+N) (one 512-column buffer);
-//       down     one MMA per K step, two 256-column accumulators.
+//       gate/up  a gate MMA and an up MMA per K step,
+//       down     two MMAs per K step on 512 consecutive W_down rows,
+//     accumulators at TMEM columns [0, N) and [256, 256+N) (one 512-column
+//     buffer: the epilogue reads the tile into registers, rounded to bf16, and
+//     hands TMEM back before it stores).
 //     Each CTA stages its 128 weight rows and half the tokens, so a CTA moves
 //     about half the shared-memory bytes per MMA cycle of the 1-SM tiling --
 //     on sm_100a the TMA writes and the tensor core's operand reads share the
@@ -63,16 +65,23 @@ constexpr int TMEM_COLS = 512;
 constexpr int MAX_GROUPS = 1024 + 8;
 constexpr int MAX_STAGES = 6;
 
+// Every tiling issues two MMAs per K step that share the token tile (their A operands are
+// the gate and up rows, or two consecutive blocks of W_down rows).  Measured on B200 at Hy4
+// prefill (T = 8192, two alternating repetitions): 2-SM down tiles of 512 W_down rows (two
+// 256-row MMAs per K step) take 2.01-2.04 ms against 2.29-2.30 for 256-row tiles with one
+// MMA per K step; the gate/up tiles already issue two MMAs per step and reach about 103
+// cycles per MMA where the single-MMA down tiles took 163.
 template <bool kGateUp, bool kPair>
 struct SwapCfg {
   static constexpr int TN = kPair ? 256 : 128;               // largest token tile (MMA N)
-  static constexpr int NUM_A = (kPair && !kGateUp) ? 1 : 2;  // A boxes per stage
+  static constexpr int NUM_A = 2;                            // A boxes per stage
   static constexpr int STAGE_BYTES = NUM_A * W_BYTES + B_BYTES;
-  static constexpr int STAGES = (kPair && !kGateUp) ? 6 : 4;
-  static constexpr int NUM_ACC = (kPair && kGateUp) ? 1 : 2;
+  static constexpr int STAGES = 4;
+  static constexpr int NUM_ACC = kPair ? 1 : 2;
   static constexpr int ACC_STRIDE = TMEM_COLS / NUM_ACC;
   static constexpr int SECOND = kPair ? 256 : 128;           // TMEM column of the 2nd MMA's D
-  static constexpr int FEAT = (kGateUp && !kPair) ? 128 : 256;  // output features per tile
+  static constexpr int A_ROWS = kPair ? 2 * WM : WM;         // weight rows of one MMA's A
+  static constexpr int FEAT = kGateUp ? A_ROWS : 2 * A_ROWS; // output features per tile
   static constexpr int MMA_M = kPair ? 256 : 128;
   static constexpr int EPI_THREADS = (kPair ? 2 : 1) * 32 * EPI_WARPS;  // arrivals freeing an acc
 };
@@ -338,7 +347,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const CUtensorMap* mW1 = kGateUp ? (tl.shared ? &p.s1 : &p.w1) : mW0;
         // this CTA's weight rows and token rows
         const int w0_row = tl.w_row + (kPair ? int(rank) * WM : 0);
-        const int w1_row = kGateUp ? w0_row : w0_row + WM;   // 1-SM down: second 128 rows
+        const int w1_row = kGateUp ? w0_row : w0_row + C::A_ROWS;   // down: the next row block
         const int t_row = tl.tok_row + (kPair ? int(rank) * (tl.n >> 1) : 0);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&ss.empty[stage], phase ^ 1)) {
@@ -534,11 +543,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             wm::store_block_transposed<true>(stg, h, lane, p.out, p.n_out, tl.out_row + c,
                                          tl.cnt - c, col0, p.out_rows);
         }
+      } else if (kPair && ksplit == 1 && p.out_bf16) {
+        // The pair's down accumulator fills all 512 columns as well: read both row blocks
+        // into registers (rounded to bf16, as they are stored), hand TMEM back, then store.
+        uint32_t yp[2][4][16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = 32 * (2 * j + sub);
+          if (c < tl.n) {
+            uint32_t r0[32], r1[32];
+            tmem_ld_32cols(tbase + uint32_t(c), r0);
+            tmem_ld_32cols(tbase + uint32_t(C::SECOND + c), r1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              yp[0][j][i] = pack_bf16x2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
+              yp[1][j][i] = pack_bf16x2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive_cluster(mapa_shared(smem_u32(&ss.tmem_empty[acc]), 0));
+        released = true;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int col0 = tl.f0 + feat_cta + half * C::A_ROWS + quarter * 32;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = 32 * (2 * j + sub);
+            if (c < tl.n && col0 < p.n_out) {
+              float v[32];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                v[2 * i] = bf16_bits_to_float(yp[half][j][i] & 0xFFFFu);
+                v[2 * i + 1] = bf16_bits_to_float(yp[half][j][i] >> 16);
+              }
+              wm::store_block_transposed<true>(stg, v, lane, p.out, p.n_out, tl.out_row + c,
+                                           tl.cnt - c, col0, p.out_rows);
+            }
+          }
+        }
       } else {
-        constexpr int kHalves = kPair ? 1 : 2;
 #pragma unroll 1
-        for (int half = 0; half < kHalves; ++half) {
-          const int col0 = tl.f0 + feat_cta + half * WM + quarter * 32;
+        for (int half = 0; half < 2; ++half) {
+          const int col0 = tl.f0 + feat_cta + half * C::A_ROWS + quarter * 32;
           const bool cols_ok = col0 < p.n_out;
           const uint32_t hbase = tbase + uint32_t(half * C::SECOND);
           int c = 32 * sub;
