@@ -274,8 +274,7 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
     weights = (inp.W_gate, inp.W_up, inp.W_down, inp.Ws_gate, inp.Ws_up, inp.Ws_down)
     dense = wl.layer == "dense"
     ihc = make_ihc(wl, device) if wl.layer == "ihc" else None
-    x_stage = torch.empty_like(inp.x) if dense else None
-    y_stage = torch.empty_like(y) if dense else None
+    x_stage = y_stage = None
     if ihc is not None:   # the activations are the residual streams H [T, n, d]
         inp.x = ihc[0]
         y = torch.empty_like(ihc[0])
@@ -290,14 +289,9 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
                                 *weights, H_out, ws, stream)
             if host:
                 y_arg.copy_(y_stage, non_blocking=True)
-        elif dense:   # the dense FFN layer; host activations go through two copies around it
-            if host:
-                x_stage.copy_(x_arg, non_blocking=True)
-                moe.moe_dense_ffn(h, x_stage, inp.W_gate, inp.W_up, inp.W_down, y_stage, ws,
-                                  stream)
-                y_arg.copy_(y_stage, non_blocking=True)
-            else:
-                moe.moe_dense_ffn(h, x_arg, inp.W_gate, inp.W_up, inp.W_down, y_arg, ws, stream)
+        elif dense:   # the dense FFN layer
+            f = moe.moe_dense_ffn_host if host else moe.moe_dense_ffn
+            f(h, x_arg, inp.W_gate, inp.W_up, inp.W_down, y_arg, ws, stream)
         elif fp8 is not None:
             f = moe.moe_forward_fp8_host if host else moe.moe_forward_fp8
             f(h, x_arg, inp.W_router, inp.bias, fp8[0], fp8[1], y_arg, ws, stream)
@@ -449,7 +443,7 @@ def workload_config(wl: Workload, world: int) -> dict:
 def e2e_api(wl: Workload, fp8: bool) -> str:
     """The call the end-to-end number goes through."""
     if wl.layer == "dense":
-        api = "moe_dense_ffn between pinned host copies"
+        api = "moe_dense_ffn_host (pinned host x in, host y out)"
     elif wl.layer == "ihc":
         api = "moe_forward_ihc between pinned host copies of the streams"
     else:

@@ -389,6 +389,19 @@ moe_status moe_dense_ffn(moe_handle h, const uint16_t *x, const uint16_t *W_gate
                          void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * moe_dense_ffn with the activations in host memory, as moe_forward_host:
+ * x_host [T][d] and y_host [T][d] bf16 in host memory (pinned for the copies
+ * to be asynchronous).  The input copy runs on the same per-device helper
+ * stream and the same two workspace staging slots as moe_forward_host, so a
+ * call's copy overlaps the previous call's layer; the output copy runs on
+ * `stream` after the layer.  y_host is complete when `stream` reaches the end
+ * of the call.  Checks and errors as in moe_dense_ffn.
+ */
+moe_status moe_dense_ffn_host(moe_handle h, const uint16_t *x_host, const uint16_t *W_gate,
+                              const uint16_t *W_up, const uint16_t *W_down, int T,
+                              uint16_t *y_host, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Synchronise the stream and read the workspace's device status word, which
  * the last call on this workspace wrote: MOE_OK, MOE_ERR_TIMEOUT or
  * MOE_ERR_BAD_INDEX.  *device_detail receives the raw word (0 if none).
@@ -398,7 +411,7 @@ moe_status moe_device_status(moe_handle h, int T, const void *workspace, void *s
 
 /*
  * Profiling hook.  With n_events == MOE_STAGE_EVENTS and events non-NULL,
- * every later moe_forward / moe_forward_host / moe_dense_ffn call on this
+ * every later moe_forward / moe_forward_host / moe_dense_ffn(_host) call on this
  * context records events[0..6] (cudaEvent_t handles the caller created) on
  * its stream at the stage boundaries: before the router, after the router,
  * after dispatch, after the gather, after the gate/up GEMM, after the down

@@ -38,7 +38,7 @@ EXPORTS = ("moe_create", "moe_destroy", "moe_workspace_size", "moe_get_workspace
            "moe_forward_host", "moe_device_status", "moe_set_stage_events",
            "moe_dispatch_noalloc", "moe_selftest_wait_timeout", "moe_forward_kernel_count",
            "moe_status_string", "moe_expert_ffn_fp8", "moe_forward_fp8", "moe_forward_fp8_host",
-           "moe_forward_partial", "moe_reduce_partials", "moe_dense_ffn",
+           "moe_forward_partial", "moe_reduce_partials", "moe_dense_ffn", "moe_dense_ffn_host",
            "moe_dense_ffn_kernel_count", "moe_ihc_mix", "moe_forward_ihc")
 MOE_STAGE_EVENTS = 7
 STAGE_NAMES = ("router", "dispatch", "gather", "gate_up_gemm", "down_gemm", "combine")
@@ -102,6 +102,7 @@ def load_library() -> ctypes.CDLL:
         "moe_forward_partial": ([P, P, P, P, I, I, P, P, P, P, P, P, I, P, P, Z, P], I),
         "moe_reduce_partials": ([P, ctypes.POINTER(P), I, I, P, P], I),
         "moe_dense_ffn": ([P, P, P, P, P, I, P, P, Z, P], I),
+        "moe_dense_ffn_host": ([P, P, P, P, P, I, P, P, Z, P], I),
         "moe_dense_ffn_kernel_count": ([P, I], I),
         "moe_ihc_mix": ([P, P, I, P, I, P, P], I),
         "moe_forward_ihc": ([P, P, I, P, P, P, P, P, P, P, P, P, P, P, I, P, P, Z, P], I),
@@ -389,6 +390,22 @@ def moe_dense_ffn(h: Handle, x, W_gate, W_up, W_down, y, workspace, stream=None)
         _ptr(Wu, torch.bfloat16, "W_up", (h.F, h.d)),
         _ptr(Wd, torch.bfloat16, "W_down", (h.d, h.F)), T,
         _ptr(y, torch.bfloat16, "y", (T, h.d)), wp, wn, _stream(stream)), "moe_dense_ffn")
+
+
+def moe_dense_ffn_host(h: Handle, x_host, W_gate, W_up, W_down, y_host, workspace,
+                       stream=None) -> None:
+    """moe_dense_ffn with x_host / y_host CPU bf16 tensors (pinned for asynchronous copies)."""
+    T = x_host.shape[0]
+    wp, wn = _ws(workspace)
+    Wg, Wu, Wd = (W.reshape(W.shape[-2:]) if W.dim() == 3 else W
+                  for W in (W_gate, W_up, W_down))
+    _check(load_library().moe_dense_ffn_host(
+        h.value, _ptr(x_host, torch.bfloat16, "x_host", (T, h.d), "cpu"),
+        _ptr(Wg, torch.bfloat16, "W_gate", (h.F, h.d)),
+        _ptr(Wu, torch.bfloat16, "W_up", (h.F, h.d)),
+        _ptr(Wd, torch.bfloat16, "W_down", (h.d, h.F)), T,
+        _ptr(y_host, torch.bfloat16, "y_host", (T, h.d), "cpu"), wp, wn, _stream(stream)),
+        "moe_dense_ffn_host")
 
 
 def moe_reduce_partials(h: Handle, partials, y, stream=None) -> None:

@@ -542,6 +542,48 @@ static moe_status forward_impl(moe_handle h, const uint16_t* x, const float* W_r
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
+// The input copy of a host-activation call: on the device's helper stream, into the next of
+// the two staging slots once the layer that last read that slot is done; the caller's stream
+// then waits for it.  *slot receives the slot, *x_dev its device address.
+static moe_status stage_host_input(moe_handle h, const DeviceInfo* dev, const Layout& L,
+                                   uint8_t* ws, const uint16_t* x_host, size_t bytes,
+                                   cudaStream_t st, unsigned* slot, uint16_t** x_dev) {
+  HostPipe& hp = h->pipes[dev->device];
+  {
+    std::lock_guard<std::mutex> lock(h->pipe_mu);
+    if (!hp.ready) {
+      bool ok = cudaStreamCreateWithFlags(&hp.copy, cudaStreamNonBlocking) == cudaSuccess;
+      for (int i = 0; i < 2 && ok; ++i)
+        ok = cudaEventCreateWithFlags(&hp.copied[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&hp.freed[i], cudaEventDisableTiming) == cudaSuccess;
+      if (!ok) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+      }
+      hp.ready = true;
+    }
+    *slot = hp.next++ & 1u;
+  }
+  *x_dev = reinterpret_cast<uint16_t*>(ws + (*slot ? L.x_stage2 : L.x_stage));
+  moe_status s;
+  if ((s = cuda_status(cudaStreamWaitEvent(hp.copy, hp.freed[*slot], 0)))) return s;
+  if ((s = cuda_status(
+           cudaMemcpyAsync(*x_dev, x_host, bytes, cudaMemcpyHostToDevice, hp.copy))))
+    return s;
+  if ((s = cuda_status(cudaEventRecord(hp.copied[*slot], hp.copy)))) return s;
+  return cuda_status(cudaStreamWaitEvent(st, hp.copied[*slot], 0));
+}
+
+// After the layer that read a staging slot: the slot is free again once the stream gets
+// here, and the output goes back to the host on the caller's stream.
+static moe_status finish_host_output(moe_handle h, const DeviceInfo* dev, unsigned slot,
+                                     uint16_t* y_host, const uint16_t* y_dev, size_t bytes,
+                                     cudaStream_t st) {
+  moe_status s;
+  if ((s = cuda_status(cudaEventRecord(h->pipes[dev->device].freed[slot], st)))) return s;
+  return cuda_status(cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st));
+}
+
 static moe_status forward_host_impl(moe_handle h, const uint16_t* x_host, const float* W_router,
                                     const float* bias, const Weights& w, int T, uint16_t* y_host,
                                     void* workspace, size_t ws_bytes, void* stream) {
@@ -557,34 +599,12 @@ static moe_status forward_host_impl(moe_handle h, const uint16_t* x_host, const 
   const Layout L = make_layout(h->c, T, kPlanSms);
   uint8_t* ws = aligned_base(workspace);
   const size_t bytes = size_t(T) * h->c.d * sizeof(uint16_t);
-  HostPipe& hp = h->pipes[dev->device];
   unsigned slot;
-  {
-    std::lock_guard<std::mutex> lock(h->pipe_mu);
-    if (!hp.ready) {
-      bool ok = cudaStreamCreateWithFlags(&hp.copy, cudaStreamNonBlocking) == cudaSuccess;
-      for (int i = 0; i < 2 && ok; ++i)
-        ok = cudaEventCreateWithFlags(&hp.copied[i], cudaEventDisableTiming) == cudaSuccess &&
-             cudaEventCreateWithFlags(&hp.freed[i], cudaEventDisableTiming) == cudaSuccess;
-      if (!ok) {
-        cudaGetLastError();
-        return MOE_ERR_CUDA;
-      }
-      hp.ready = true;
-    }
-    slot = hp.next++ & 1u;
-  }
-  uint16_t* x_dev = reinterpret_cast<uint16_t*>(ws + (slot ? L.x_stage2 : L.x_stage));
+  uint16_t* x_dev;
+  if ((s = stage_host_input(h, dev, L, ws, x_host, bytes, st, &slot, &x_dev))) return s;
   uint16_t* y_dev = reinterpret_cast<uint16_t*>(ws + L.y_stage);
-  // input copy on the helper stream, once the layer that last read this slot is done
-  if ((s = cuda_status(cudaStreamWaitEvent(hp.copy, hp.freed[slot], 0)))) return s;
-  if ((s = cuda_status(cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, hp.copy))))
-    return s;
-  if ((s = cuda_status(cudaEventRecord(hp.copied[slot], hp.copy)))) return s;
-  if ((s = cuda_status(cudaStreamWaitEvent(st, hp.copied[slot], 0)))) return s;
   if ((s = forward_device(h, x_dev, W_router, bias, w, T, y_dev, ws, L, dev, st))) return s;
-  if ((s = cuda_status(cudaEventRecord(hp.freed[slot], st)))) return s;
-  return cuda_status(cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st));
+  return finish_host_output(h, dev, slot, y_host, y_dev, bytes, st);
 }
 
 moe_status moe_forward(moe_handle h, const uint16_t* x, const float* W_router, const float* bias,
@@ -654,9 +674,10 @@ moe_status moe_forward_partial(moe_handle h, const uint16_t* x, const float* W_r
                         reinterpret_cast<cudaStream_t>(stream), &shard);
 }
 
-moe_status moe_dense_ffn(moe_handle h, const uint16_t* x, const uint16_t* W_gate,
-                         const uint16_t* W_up, const uint16_t* W_down, int T, uint16_t* y,
-                         void* workspace, size_t ws_bytes, void* stream) {
+// The checks of moe_dense_ffn and moe_dense_ffn_host (x and y device or host pointers).
+static moe_status check_dense_args(moe_handle h, const uint16_t* x, const uint16_t* W_gate,
+                                   const uint16_t* W_up, const uint16_t* W_down, int T,
+                                   const uint16_t* y, void* workspace, size_t ws_bytes) {
   if (!h) return MOE_ERR_INVALID_ARG;
   const Ctx& c = h->c;
   if (c.E != 1 || c.k != 1 || c.S != 0) return MOE_ERR_INVALID_ARG;
@@ -667,12 +688,16 @@ moe_status moe_dense_ffn(moe_handle h, const uint16_t* x, const uint16_t* W_gate
   if (!aligned16(x) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down) ||
       !aligned16(y))
     return MOE_ERR_ALIGNMENT;
-  if ((s = check_ws(h, T, workspace, ws_bytes))) return s;
-  DeviceInfo* dev;
-  if ((s = ensure_device(&dev))) return s;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const Layout L = make_layout(c, T, kPlanSms);
-  uint8_t* ws = aligned_base(workspace);
+  return check_ws(h, T, workspace, ws_bytes);
+}
+
+// The dense layer on device activations: the checks are done.
+static moe_status dense_device(moe_handle h, const uint16_t* x, const uint16_t* W_gate,
+                               const uint16_t* W_up, const uint16_t* W_down, int T, uint16_t* y,
+                               uint8_t* ws, const Layout& L, const DeviceInfo* dev,
+                               cudaStream_t st) {
+  const Ctx& c = h->c;
+  moe_status s;
   int* status = reinterpret_cast<int*>(ws + L.status);
   int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
   int32_t* sched = reinterpret_cast<int32_t*>(ws + L.sched);
@@ -705,6 +730,38 @@ moe_status moe_dense_ffn(moe_handle h, const uint16_t* x, const uint16_t* W_gate
   if ((s = launch_expert_ffn(c, a, *dev, st))) return s;
   if ((s = mark(5))) return s;
   return mark(6);   // no combine
+}
+
+moe_status moe_dense_ffn(moe_handle h, const uint16_t* x, const uint16_t* W_gate,
+                         const uint16_t* W_up, const uint16_t* W_down, int T, uint16_t* y,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  moe_status s = check_dense_args(h, x, W_gate, W_up, W_down, T, y, workspace, ws_bytes);
+  if (s || T == 0) return s;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  const Layout L = make_layout(h->c, T, kPlanSms);
+  return dense_device(h, x, W_gate, W_up, W_down, T, y, aligned_base(workspace), L, dev,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_dense_ffn_host(moe_handle h, const uint16_t* x_host, const uint16_t* W_gate,
+                              const uint16_t* W_up, const uint16_t* W_down, int T,
+                              uint16_t* y_host, void* workspace, size_t ws_bytes, void* stream) {
+  moe_status s = check_dense_args(h, x_host, W_gate, W_up, W_down, T, y_host, workspace,
+                                  ws_bytes);
+  if (s || T == 0) return s;
+  DeviceInfo* dev;
+  if ((s = ensure_device(&dev))) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Layout L = make_layout(h->c, T, kPlanSms);
+  uint8_t* ws = aligned_base(workspace);
+  const size_t bytes = size_t(T) * h->c.d * sizeof(uint16_t);
+  unsigned slot;
+  uint16_t* x_dev;
+  if ((s = stage_host_input(h, dev, L, ws, x_host, bytes, st, &slot, &x_dev))) return s;
+  uint16_t* y_dev = reinterpret_cast<uint16_t*>(ws + L.y_stage);
+  if ((s = dense_device(h, x_dev, W_gate, W_up, W_down, T, y_dev, ws, L, dev, st))) return s;
+  return finish_host_output(h, dev, slot, y_host, y_dev, bytes, st);
 }
 
 moe_status moe_ihc_mix(moe_handle h, const uint16_t* H, int n_streams, const float* alpha, int T,

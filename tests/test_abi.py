@@ -270,6 +270,16 @@ def test_shard_and_dense_entry_points_validate_on_the_host(lib):
     assert L.moe_dense_ffn(hd.value, A, A, A + 2, A, T, A, A, wsd, None) == moe.MOE_ERR_ALIGNMENT
     assert L.moe_dense_ffn(hd.value, A, A, A, A, T, A, A, wsd - 1, None) == moe.MOE_ERR_WORKSPACE
     assert L.moe_dense_ffn(hd.value, None, None, None, None, 0, None, None, 0, None) == moe.MOE_OK
+    # the host-activation form takes the same checks
+    assert L.moe_dense_ffn_host(hv, A, A, A, A, T, A, A, ws, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_dense_ffn_host(hd.value, A, A, A + 2, A, T, A, A, wsd, None) == \
+        moe.MOE_ERR_ALIGNMENT
+    assert L.moe_dense_ffn_host(hd.value, A, A, A, A, T, A, A, wsd - 1, None) == \
+        moe.MOE_ERR_WORKSPACE
+    assert L.moe_dense_ffn_host(hd.value, A, A, A, A, T, None, A, wsd, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert L.moe_dense_ffn_host(hd.value, None, None, None, None, 0, None, None, 0, None) == \
+        moe.MOE_OK
     # up to 128 tokens the down projection is split over K (one launch more)
     assert L.moe_dense_ffn_kernel_count(hd.value, 16) == 4
     assert L.moe_dense_ffn_kernel_count(hd.value, 4096) == 3

@@ -84,3 +84,31 @@ def test_dense_first_layer_full_size(name):
     err = rel_err(y.float().cpu().numpy()[tokens], ref)
     print(f"{name}: {len(tokens)} tokens, rel err {err:.3e}")
     assert err < Y_REL_TOL, err
+
+
+@pytest.mark.parametrize("shape", [(64, 256, 640), (517, 256, 2304)],
+                         ids=lambda s: "T{}_d{}_F{}".format(*s))
+def test_dense_ffn_host_matches_the_device_call(shape):
+    """moe_dense_ffn_host on pinned host activations gives moe_dense_ffn's bits.  Calls are
+    enqueued back to back without synchronising, each on its own input, so the staging slots
+    alternate while earlier layers still run; every output is its own input's."""
+    T, d, F = shape
+    inputs = [make_small(T, d, 1, 1, F, 0, seed=1200 + T + i) for i in range(3)]
+    dev = to_device(inputs[0], "cuda")
+    h = moe.moe_create(d, 1, 1, F, 0)
+    ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
+    want = []
+    for inp in inputs:
+        y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+        moe.moe_dense_ffn(h, inp.x.cuda(), dev.W_gate, dev.W_up, dev.W_down, y, ws)
+        want.append(y.cpu())
+    xs = [inp.x.pin_memory() for inp in inputs]
+    ys = [torch.full((T, d), float("nan"), dtype=torch.bfloat16).pin_memory() for _ in inputs]
+    for _ in range(2):
+        for x, y in zip(xs, ys):
+            moe.moe_dense_ffn_host(h, x, dev.W_gate, dev.W_up, dev.W_down, y, ws)
+    torch.cuda.synchronize()
+    st, detail = moe.moe_device_status(h, T, ws)
+    assert st == moe.MOE_OK, hex(detail)
+    for y, w in zip(ys, want):
+        assert torch.equal(y.view(torch.int16), w.view(torch.int16))
