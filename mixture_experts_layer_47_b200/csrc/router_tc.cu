@@ -14,12 +14,15 @@
 //    parts) go into a fresh TMEM accumulator, and the epilogue warps add the
 //    chunk results in fp32 on the CUDA cores, in chunk order (deterministic).
 // Layout: a persistent kernel, one CTA per SM, 192 threads.  Warp 0 issues TMA
-// loads (128 x 64 x-tile, three 64 x 64 W-part tiles, 128-byte swizzle, 4
-// stages); warp 1 owns 512 TMEM columns = a ring of 8 accumulators of 128 x 64
-// fp32 and issues tcgen05.mma (M=128, N=64); warps 2-5 drain the ring, one
-// token row per thread.  A tile is (128 tokens, 64 experts, one K range); K is
+// loads (128 x 64 x-tile, three 128 x 64 W-part tiles, 128-byte swizzle, 3
+// stages); warp 1 owns 512 TMEM columns = a ring of 4 accumulators of 128 x 128
+// fp32 and issues tcgen05.mma (M=128, N=128); warps 2-5 drain the ring, one
+// token row per thread.  A tile is (128 tokens, 128 experts, one K range); K is
 // split across CTAs when there are too few tiles to fill the GPU, and the
-// partial logits are added in split order by the top-k kernel.
+// partial logits are added in split order by the top-k kernel.  Measured on B200
+// at T = 8192, E = 256 (moe_route: the weight split, this kernel and the top-k):
+// 0.109 ms with 128-expert tiles (one wave of 128 tiles) against 0.167 ms with
+// 64-expert tiles (256 tiles in 1.7 waves, each x tile staged twice as often).
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -31,13 +34,13 @@ namespace moe {
 namespace {
 
 constexpr int RT_BM = 128;
-constexpr int RT_BN = 64;
+constexpr int RT_BN = 128;
 constexpr int RT_BK = 64;
-constexpr int RT_STAGES = 4;
+constexpr int RT_STAGES = 3;
 constexpr int RT_A_BYTES = RT_BM * RT_BK * 2;
 constexpr int RT_B_BYTES = RT_BN * RT_BK * 2;
 constexpr int RT_STAGE_BYTES = RT_A_BYTES + 3 * RT_B_BYTES;
-constexpr int RT_RING = 8;          // accumulators of RT_BN columns
+constexpr int RT_RING = 4;          // accumulators of RT_BN columns
 constexpr int RT_CHUNK_KB = 2;      // 64-wide K blocks accumulated per chunk (K = 128)
 constexpr int RT_THREADS = 192;
 constexpr uint32_t RT_IDESC = umma_idesc_bf16_f32(RT_BM, RT_BN);
@@ -228,14 +231,17 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t taddr = tmem_base + lane_addr + slot * RT_BN;
-        uint32_t v0[32], v1[32];   // both halves in flight, one wait
-        tmem_ld_32cols(taddr, v0);
-        tmem_ld_32cols(taddr + 32u, v1);
-        tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          sum[j] += __uint_as_float(v0[j]);
-          sum[32 + j] += __uint_as_float(v1[j]);
+        for (int half = 0; half < RT_BN / 64; ++half) {
+          uint32_t v0[32], v1[32];   // 64 columns in flight, one wait
+          tmem_ld_32cols(taddr + uint32_t(64 * half), v0);
+          tmem_ld_32cols(taddr + uint32_t(64 * half + 32), v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            sum[64 * half + j] += __uint_as_float(v0[j]);
+            sum[64 * half + 32 + j] += __uint_as_float(v1[j]);
+          }
         }
         tc_fence_before();
         mbar_arrive(&ss.chunk_free[slot]);
