@@ -308,10 +308,6 @@ __device__ __forceinline__ void finish_item(const GemvParams& p, const Item& it,
     }
 }
 
-
-// After an item's last block the lanes hold (or, for an item cut between warps, the summed
-// parts give) element i of column block n = (row g + 8 (i / 2), token 8 n + 2 t + i % 2)
-// of both tiles.
 // This warp's jobs of one item, blocks [blk0, blk0 + nb); slot is the stage the first one
 // reads.  A whole item is finished from the registers.  A part of a cut item goes to this
 // warp's partial slot (0: the item began before this warp's jobs, 1: it runs past them);
