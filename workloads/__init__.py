@@ -124,6 +124,11 @@ PROFILE_WORKLOADS = {
         "profile_prefill_e32", T=1024, d=6144, E=32, k=8, F=2048, S=1, router="uniform", seed=0,
         description="prefill-shaped profiling case: T=1024 (256 rows per expert), d=6144, "
                     "32 experts top-8 + 1 shared"),
+    "profile_router_prefill": Workload(
+        "profile_router_prefill", T=8192, d=6144, E=256, k=8, F=64, S=1, router="uniform",
+        seed=0,
+        description="the prefill router at full size (T=8192, d=6144, 256 experts top-8) with "
+                    "64-wide experts, so the case holds about 1 GB on the device"),
     "profile_decode_fp8_e32": Workload(
         "profile_decode_fp8_e32", T=16, d=6144, E=32, k=8, F=2048, S=1, router="normal", seed=0,
         weights="fp8",
