@@ -14,8 +14,9 @@
 // decoded registers.
 //
 // Work: an item is 16 feature rows of one group -- the gate and the up rows of 16 features,
-// or 32 consecutive W_down rows as two 16-row tiles -- for all of the group's tokens (one MMA
-// column block of 8 tokens, two when the group has more than 8), walked in K blocks of 64.
+// or 32 consecutive W_down rows as two 16-row tiles -- for one unit of up to 8 of the group's
+// tokens (one MMA column block; a group of n tokens is ceil(n/8) units, and a second unit
+// decodes the rows again, its codes then coming from L2), walked in K blocks of 64.
 // A CTA takes items round robin (about 90 per CTA at Hy4 decode); their K blocks are its
 // jobs, cut into equal runs for its 8 warps, so every warp has the same number of blocks
 // (taking whole items per warp left a tail of up to 9%).  A warp finishes an item it ran
@@ -29,12 +30,14 @@
 // 16-byte load) and its 16 consecutive activations (32 bytes) feed all four MMAs of the
 // block, and each 32-wide scale block lies inside one lane's run.
 // Stream: each lane copies its rows' codes and its tokens' activations for a block with
-// cp.async into a per-warp 5-stage ring in shared memory, four blocks ahead of the block it
+// cp.async into a per-warp 8-stage ring in shared memory, seven blocks ahead of the block it
 // computes (the ring runs on across items; the lane keeps running source pointers), so the
 // loads in flight hold no registers; four lanes also copy the tiles' 16 scale bytes per
 // 32-wide K block, read by all lanes after the ring wait and a warp barrier.  Measured on
-// B200 at Hy4 decode: 8 warps with deep rings beat 10 x 4, 12 x 4 and 16 x 3 stages, and the
-// even cut of the jobs gained 7% on gate/up over whole items per warp.
+// B200 at Hy4 decode: 8 warps with deep rings beat 10 x 4, 12 x 4 and 16 x 3 stages, the even
+// cut of the jobs gained 7% on gate/up over whole items per warp, and units of 8 tokens (one
+// column block: 3 KB stages, 8-value partial slots, so 8 stages fit beside them) took the
+// layer from 0.761 to 0.749 ms against 16-token units with 5 stages.
 // Arithmetic: exact bf16 weights (the decoder of the tensor-core FP8 kernel) times bf16
 // activations into fp32 accumulators, as in the tensor-core path; only the order of the
 // fp32 additions differs.  The epilogue applies SwiGLU (gate/up) from registers: a lane's
@@ -50,18 +53,19 @@ namespace {
 constexpr int GV_WARPS = 8;
 constexpr int GV_THREADS = 32 * GV_WARPS;
 constexpr int GV_KB = 64;                        // K per block (4 MMAs)
-constexpr int GV_STAGES = 5;
+constexpr int GV_STAGES = 8;
 constexpr int GV_MAX_GROUPS = 1024 + 8;          // E + S upper bound
-constexpr int GV_MAX_TOK = 16;                   // tokens per group: two 8-token MMA columns
-// Per warp and stage: codes [tile 2][row half 2][lane 32][16 B], activations
-// [column block 2][lane 32][32 B], scales [tile 2][32-wide K block 2][16 B].
+constexpr int GV_MAX_TOK = 16;                   // tokens per group
+constexpr int GV_UNIT_TOK = 8;                   // tokens per unit: one 8-token MMA column block
+// Per warp and stage: codes [tile 2][row half 2][lane 32][16 B], activations [lane 32][32 B],
+// scales [tile 2][32-wide K block 2][16 B].
 constexpr int GV_CODE_OFF = 0;
 constexpr int GV_X_OFF = 2 * 2 * 32 * 16;
-constexpr int GV_SCALE_OFF = GV_X_OFF + 2 * 32 * 32;
+constexpr int GV_SCALE_OFF = GV_X_OFF + 32 * 32;
 constexpr int GV_STAGE_BYTES = GV_SCALE_OFF + 2 * 2 * 16;
 constexpr int GV_RING_BYTES = GV_WARPS * GV_STAGES * GV_STAGE_BYTES;
-// After the rings: the partial sums of cut items, [warp][slot 2][value 16][lane 32].
-constexpr size_t GV_SMEM = size_t(GV_RING_BYTES) + size_t(GV_WARPS) * 2 * 16 * 32 * sizeof(float);
+// After the rings: the partial sums of cut items, [warp][slot 2][value 8][lane 32].
+constexpr size_t GV_SMEM = size_t(GV_RING_BYTES) + size_t(GV_WARPS) * 2 * 8 * 32 * sizeof(float);
 static_assert(GV_STAGE_BYTES % 16 == 0, "stages stay 16-byte aligned");
 
 struct GemvParams {
@@ -111,7 +115,7 @@ struct Item {
   const uint16_t* tok;   // first token's activation row
   size_t out_row;        // first token's output row
   int f;                 // first feature
-  int nt;                // tokens, 1..GV_MAX_TOK; 0 past the last item
+  int nt;                // tokens of this unit, 1..GV_UNIT_TOK; 0 past the last item
   bool shared;           // a shared expert's item
 };
 
@@ -133,9 +137,11 @@ __device__ __forceinline__ Item describe(const GemvParams& p, const int16_t* uni
   const bool shared = g >= p.E;
   const int gl = shared ? g - p.E : g;
   const int off = shared ? 0 : __ldg(p.offsets + g);
-  it.nt = shared ? p.T : min(p.T, __ldg(p.offsets + g + 1) - off);
-  const size_t row0 = shared ? size_t(p.T) * p.k + size_t(gl) * p.T : size_t(off);
-  const size_t tok_row = (shared && kGateUp) ? size_t(0) : row0;
+  const int n = shared ? p.T : min(p.T, __ldg(p.offsets + g + 1) - off);
+  const int t0 = (u - units[g]) * GV_UNIT_TOK;           // this unit's first token of the group
+  it.nt = min(GV_UNIT_TOK, n - t0);
+  const size_t row0 = (shared ? size_t(p.T) * p.k + size_t(gl) * p.T : size_t(off)) + t0;
+  const size_t tok_row = (shared && kGateUp) ? size_t(t0) : row0;
   it.tok = (shared && kGateUp ? p.tok_shared : p.tok_routed) + tok_row * size_t(p.K);
   it.out_row = row0;
   it.shared = shared;
@@ -168,10 +174,10 @@ __device__ __forceinline__ int warp_of_job(int jobs, int j) {
 
 // The copies run GV_STAGES - 1 blocks ahead of the arithmetic, across items.  The cursor
 // keeps this lane's source pointers for its next job: codes of rows g and g + 8 of both
-// tiles, the activations of tokens g and g + 8, and (lanes 0-3) a scale row.
+// tiles, the activations of token g, and (lanes 0-3) a scale row.
 struct IssueCursor {
   const uint8_t* code[4];   // [tile m * 2 + row half h]
-  const uint16_t* x[2];     // [column block n]
+  const uint16_t* x;        // token g
   const uint8_t* scale;     // lane 2 m + b < 4: tile m's scales of 32-wide block 2 blk + b
   int job, blk, nt;         // nt = 0 when this warp's jobs are all issued
 };
@@ -192,8 +198,7 @@ __device__ __forceinline__ void cursor_at(const GemvParams& p, const Item& it, i
 #pragma unroll
     for (int h = 0; h < 2; ++h) ic.code[m * 2 + h] = base + size_t(g + 8 * h) * p.K;
   }
-#pragma unroll
-  for (int n = 0; n < 2; ++n) ic.x[n] = it.tok + size_t(g + 8 * n) * p.K + k0;
+  ic.x = it.tok + size_t(g) * p.K + k0;
   const int m = (lane >> 1) & 1, b = lane & 1;
   ic.scale = (it.shared ? p.ss[kGateUp ? m : 0] : p.s[kGateUp ? m : 0]) + it.soff +
              (kGateUp ? 0 : 16 * m) + size_t(2 * blk + b) * p.n_out;
@@ -217,15 +222,12 @@ __device__ __forceinline__ void issue_next(const GemvParams& p, const Walk& wk, 
       cp_async16(stage + uint32_t(GV_CODE_OFF + (i * 32 + lane) * 16), ic.code[i]);
       ic.code[i] += GV_KB;
     }
-#pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      if (g + 8 * n < ic.nt) {
-        const uint32_t dst = stage + uint32_t(GV_X_OFF + (n * 32 + lane) * 32);
-        cp_async16(dst, ic.x[n]);
-        cp_async16(dst + 16, ic.x[n] + 8);
-      }
-      ic.x[n] += GV_KB;
+    if (g < ic.nt) {
+      const uint32_t dst = stage + uint32_t(GV_X_OFF + lane * 32);
+      cp_async16(dst, ic.x);
+      cp_async16(dst + 16, ic.x + 8);
     }
+    ic.x += GV_KB;
     if (lane < 4) cp_async16(stage + uint32_t(GV_SCALE_OFF + lane * 16), ic.scale);
     ic.scale += size_t(2) * p.n_out;
     if (++ic.job == wk.j1) {
@@ -237,11 +239,10 @@ __device__ __forceinline__ void issue_next(const GemvParams& p, const Walk& wk, 
   cp_async_commit();
 }
 
-// The four MMAs of one K block for NCOL 8-token column blocks.  The activation columns of
-// tokens past the group's end are never copied and hold stale values: an MMA's output
-// column depends on its own B column only, and those columns are not stored.
-template <int NCOL>
-__device__ __forceinline__ void compute_block(const uint8_t* stage, float (&acc)[2][2][4],
+// The four MMAs of one K block.  The activation columns of tokens past the unit's end are
+// never copied and hold stale values: an MMA's output column depends on its own B column only,
+// and those columns are not stored.
+__device__ __forceinline__ void compute_block(const uint8_t* stage, float (&acc)[2][4],
                                               int lane) {
   const int g = lane >> 2, t = lane & 3;
   uint4 code[2][2];
@@ -254,13 +255,8 @@ __device__ __forceinline__ void compute_block(const uint8_t* stage, float (&acc)
       // this lane's 16 positions lie in 32-wide block t / 2 of the 64
       mult[m][h] = scale_pair(stage[GV_SCALE_OFF + (m * 2 + (t >> 1)) * 16 + g + 8 * h]);
     }
-  uint4 xv[NCOL][2];
-#pragma unroll
-  for (int n = 0; n < NCOL; ++n) {
-    const uint4* src = reinterpret_cast<const uint4*>(stage + GV_X_OFF + (n * 32 + lane) * 32);
-    xv[n][0] = src[0];
-    xv[n][1] = src[1];
-  }
+  const uint4* xsrc = reinterpret_cast<const uint4*>(stage + GV_X_OFF + lane * 32);
+  const uint4 xv[2] = {xsrc[0], xsrc[1]};
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
 #pragma unroll
@@ -269,82 +265,73 @@ __device__ __forceinline__ void compute_block(const uint8_t* stage, float (&acc)
       uint32_t a[4];
       decode_word((&code[m][0].x)[s], mult[m][0], a[0], a[2]);
       decode_word((&code[m][1].x)[s], mult[m][1], a[1], a[3]);
-#pragma unroll
-      for (int n = 0; n < NCOL; ++n) {
-        const uint4& xs = xv[n][s >> 1];
-        mma_bf16_16816(acc[m][n], a, (s & 1) ? xs.z : xs.x, (s & 1) ? xs.w : xs.y);
-      }
+      const uint4& xs = xv[s >> 1];
+      mma_bf16_16816(acc[m], a, (s & 1) ? xs.z : xs.x, (s & 1) ? xs.w : xs.y);
     }
   }
 }
 
-// After an item's last block: accumulator element i of column block n is
-// (row g + 8 (i / 2), token 8 n + 2 t + i % 2) of both tiles.
-template <bool kGateUp, int NCOL>
+// After an item's last block: accumulator element i of tile m is (row g + 8 (i / 2), token
+// 2 t + i % 2 of the unit).
+template <bool kGateUp>
 __device__ __forceinline__ void finish_item(const GemvParams& p, const Item& it,
-                                            const float (&acc)[2][2][4], int lane) {
+                                            const float (&acc)[2][4], int lane) {
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int n = 0; n < NCOL; ++n)
+  for (int i = 0; i < 4; ++i) {
+    const int tok = 2 * t + (i & 1);
+    if (tok >= it.nt) continue;
+    const int row = g + 8 * (i >> 1);
+    const size_t o = (it.out_row + tok) * size_t(p.n_out) + it.f + row;
+    if (kGateUp) {
+      reinterpret_cast<uint16_t*>(p.out)[o] =
+          uint16_t(pack_bf16x2(wm::swiglu(acc[0][i], acc[1][i]), 0.f) & 0xFFFFu);
+    } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int tok = 8 * n + 2 * t + (i & 1);
-      if (tok >= it.nt) continue;
-      const int row = g + 8 * (i >> 1);
-      const size_t o = (it.out_row + tok) * size_t(p.n_out) + it.f + row;
-      if (kGateUp) {
-        reinterpret_cast<uint16_t*>(p.out)[o] =
-            uint16_t(pack_bf16x2(wm::swiglu(acc[0][n][i], acc[1][n][i]), 0.f) & 0xFFFFu);
-      } else {
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          if (p.out_bf16)
-            reinterpret_cast<uint16_t*>(p.out)[o + 16 * m] =
-                uint16_t(pack_bf16x2(acc[m][n][i], 0.f) & 0xFFFFu);
-          else
-            reinterpret_cast<float*>(p.out)[o + 16 * m] = acc[m][n][i];
-        }
+      for (int m = 0; m < 2; ++m) {
+        if (p.out_bf16)
+          reinterpret_cast<uint16_t*>(p.out)[o + 16 * m] =
+              uint16_t(pack_bf16x2(acc[m][i], 0.f) & 0xFFFFu);
+        else
+          reinterpret_cast<float*>(p.out)[o + 16 * m] = acc[m][i];
       }
     }
+  }
 }
 
 // This warp's jobs of one item, blocks [blk0, blk0 + nb); slot is the stage the first one
 // reads.  A whole item is finished from the registers.  A part of a cut item goes to this
 // warp's partial slot (0: the item began before this warp's jobs, 1: it runs past them);
 // the last of the item's warps to arrive adds the parts in warp order and finishes it.
-template <bool kGateUp, int NCOL>
+template <bool kGateUp>
 __device__ __forceinline__ void run_segment(const GemvParams& p, const Walk& wk, const Item& it,
                                             int q, int blk0, int nb, IssueCursor& ic, int& slot,
                                             float* part, int* cut_count, int warp) {
-  float acc[2][2][4];
+  float acc[2][4];
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
-    for (int n = 0; n < 2; ++n)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
+    for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
   for (int b = 0; b < nb; ++b) {
     // refill the stage computed last (its reads are done), GV_STAGES - 1 jobs ahead
     issue_next<kGateUp>(p, wk, ic, slot == 0 ? GV_STAGES - 1 : slot - 1);
     cp_async_wait_ring();
     __syncwarp();   // the scale bytes were copied by lanes 0-3
-    compute_block<NCOL>(wk.ring + slot * GV_STAGE_BYTES, acc, wk.lane);
+    compute_block(wk.ring + slot * GV_STAGE_BYTES, acc, wk.lane);
     __syncwarp();   // every lane is done with the stage before lanes 0-3 refill it
     slot = slot == GV_STAGES - 1 ? 0 : slot + 1;
   }
   if (blk0 == 0 && nb == wk.nblk) {
-    finish_item<kGateUp, NCOL>(p, it, acc, wk.lane);
+    finish_item<kGateUp>(p, it, acc, wk.lane);
     return;
   }
   const int lane = wk.lane;
   const int first_job = q * wk.nblk;
-  float* mine = part + ((warp * 2 + (first_job < wk.j0 ? 0 : 1)) * 16) * 32;
+  float* mine = part + ((warp * 2 + (first_job < wk.j0 ? 0 : 1)) * 8) * 32;
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
-    for (int n = 0; n < 2; ++n)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) mine[(8 * m + 4 * n + i) * 32 + lane] = acc[m][n][i];
+    for (int i = 0; i < 4; ++i) mine[(4 * m + i) * 32 + lane] = acc[m][i];
   __threadfence_block();
   __syncwarp();
   // the item's parts: the warps from w_first to w_last that have jobs (with fewer jobs than
@@ -362,21 +349,17 @@ __device__ __forceinline__ void run_segment(const GemvParams& p, const Walk& wk,
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
-    for (int n = 0; n < 2; ++n)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
+    for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
   for (int w = w_first; w <= w_last; ++w) {
     const int jw = warp_first_job(wk.jobs, w);
     if (warp_first_job(wk.jobs, w + 1) == jw) continue;   // no jobs, no part
-    const float* src = part + ((w * 2 + (first_job < jw ? 0 : 1)) * 16) * 32;
+    const float* src = part + ((w * 2 + (first_job < jw ? 0 : 1)) * 8) * 32;
 #pragma unroll
     for (int m = 0; m < 2; ++m)
 #pragma unroll
-      for (int n = 0; n < 2; ++n)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[m][n][i] += src[(8 * m + 4 * n + i) * 32 + lane];
+      for (int i = 0; i < 4; ++i) acc[m][i] += src[(4 * m + i) * 32 + lane];
   }
-  finish_item<kGateUp, NCOL>(p, it, acc, lane);
+  finish_item<kGateUp>(p, it, acc, lane);
 }
 
 template <bool kGateUp>
@@ -397,7 +380,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
       int n = 0;
       if (g < p.E) n = min(p.T, max(0, p.offsets[g + 1] - p.offsets[g]));
       else if (g < G) n = p.T;
-      int incl = n > 0 ? 1 : 0;
+      int incl = (n + GV_UNIT_TOK - 1) / GV_UNIT_TOK;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -439,8 +422,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     const int q = j / wk.nblk, blk0 = j - q * wk.nblk;
     const int nb = min(wk.j1, (q + 1) * wk.nblk) - j;
     const Item it = job_item<kGateUp>(p, wk, q);
-    if (it.nt > 8) run_segment<kGateUp, 2>(p, wk, it, q, blk0, nb, ic, slot, part, cut_count, warp);
-    else run_segment<kGateUp, 1>(p, wk, it, q, blk0, nb, ic, slot, part, cut_count, warp);
+    run_segment<kGateUp>(p, wk, it, q, blk0, nb, ic, slot, part, cut_count, warp);
     j += nb;
   }
   cp_async_wait_all();

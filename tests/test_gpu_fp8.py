@@ -8,7 +8,7 @@ than one token tile per group, two shared experts and none.  Every form of the F
 runs: the tcgen05 kernel's 1-SM form (MOE_GEMM_TILES=swap, and the default above 16
 tokens) and 2-SM pair (MOE_GEMM_TILES=swap_pair), and the warp-MMA form the default takes
 at up to 16 tokens, whose shapes add K lengths of fewer 64-wide blocks than a CTA has warps,
-groups of 1 to 8 tokens (one MMA column block) and of 9 to 16 (two).
+groups of 1 to 8 tokens (one 8-token unit) and of 9 to 16 (two units).
 """
 import numpy as np
 import pytest
@@ -32,7 +32,7 @@ FP8_SHAPES = [  # T, d, E, k, F, S, bias_scale
     (16, 320, 5, 3, 384, 2, 0.0),      # K = 320 and 384: 5 and 6 blocks of 64 for 8 warps
     (1, 64, 1, 1, 64, 0, 0.0),         # one token, one expert, one K block: the smallest shape
     (12, 192, 64, 8, 192, 1, 0.5),     # most groups empty or of one token
-    (13, 128, 2, 1, 128, 1, 0.0),      # routed groups of 6-7 tokens, the shared one of 13 (two column blocks)
+    (13, 128, 2, 1, 128, 1, 0.0),      # routed groups of 6-7 tokens, the shared one of 13 (two units)
 ]
 GEMV_SHAPES = [s for s in FP8_SHAPES if s[0] <= 16]
 
