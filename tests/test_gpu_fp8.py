@@ -305,3 +305,33 @@ def test_fp8_gemv_special_codes(monkeypatch):
     y8, v8 = _forward_fp8(to_device(inp, "cuda"), routed.to("cuda"), shared.to("cuda"))
     ref = oracle.forward(decoded_inputs(inp, routed, shared), idx_override=v8["topk_idx"].numpy())
     assert rel_err(y8.float().numpy(), ref["y"]) < Y_REL_TOL
+
+
+@pytest.mark.parametrize("shape", [FP8_SHAPES[1], GEMV_SHAPES[0]], ids=_ids([FP8_SHAPES[1], GEMV_SHAPES[0]]))
+def test_fp8_host_activations_match_the_device_call(shape):
+    """moe_forward_fp8_host (pinned host x in, host y out) gives moe_forward_fp8's bits, for the
+    tcgen05 form (64 tokens) and the warp-MMA form (7 tokens).  Calls are enqueued back to back
+    without synchronising, each on its own input, so the staging slots alternate while earlier
+    layers still run; every output is its own input's."""
+    T, d, E, k, F, S, bs = shape
+    inputs = [make_small(T, d, E, k, F, S, seed=1900 + T + i, bias_scale=bs) for i in range(3)]
+    routed, shared = make_fp8(inputs[0])
+    routed, shared = routed.to("cuda"), shared.to("cuda")
+    dev = to_device(inputs[0], "cuda")
+    h = moe.moe_create(d, E, k, F, S)
+    ws = torch.empty(moe.moe_workspace_size(h, T), dtype=torch.uint8, device="cuda")
+    want = []
+    for inp in inputs:
+        y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+        moe.moe_forward_fp8(h, inp.x.cuda(), dev.W_router, dev.bias, routed, shared, y, ws)
+        want.append(y.cpu())
+    xs = [inp.x.pin_memory() for inp in inputs]
+    ys = [torch.full((T, d), float("nan"), dtype=torch.bfloat16).pin_memory() for _ in inputs]
+    for _ in range(2):
+        for x, y in zip(xs, ys):
+            moe.moe_forward_fp8_host(h, x, dev.W_router, dev.bias, routed, shared, y, ws)
+    torch.cuda.synchronize()
+    st, detail = moe.moe_device_status(h, T, ws)
+    assert st == moe.MOE_OK, hex(detail)
+    for y, w in zip(ys, want):
+        assert torch.equal(y.view(torch.int16), w.view(torch.int16))
