@@ -33,6 +33,8 @@ FP8_SHAPES = [  # T, d, E, k, F, S, bias_scale
     (1, 64, 1, 1, 64, 0, 0.0),         # one token, one expert, one K block: the smallest shape
     (12, 192, 64, 8, 192, 1, 0.5),     # most groups empty or of one token
     (13, 128, 2, 1, 128, 1, 0.0),      # routed groups of 6-7 tokens, the shared one of 13 (two units)
+    (16, 64, 1024, 8, 64, 1, 0.0),     # 1024 experts: ~120 non-empty groups, the unit table's limit
+    (16, 128, 8, 8, 64, 0, 0.0),       # k == E, no shared expert: every group two 8-token units
 ]
 GEMV_SHAPES = [s for s in FP8_SHAPES if s[0] <= 16]
 
