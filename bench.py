@@ -203,7 +203,7 @@ def fp8_form(T: int) -> str:
 
 
 def measured_traffic(kernel: str, bound: str, units: int, weights: str = "bf16",
-                     d_model: int = 6144, d_ff: int = 2048, T: int = 16):
+                     d_model: int = 6144, d_ff: int = 2048, T: int = 16, layer: str = "moe"):
     """DRAM bytes per launch of ``kernel`` scaled from the committed ncu capture
     (profiles/traffic.json) by the touched experts, or None when there is none, when the
     experts' shape differs from the captured one (per-expert bytes do not carry over), or
@@ -212,7 +212,8 @@ def measured_traffic(kernel: str, bound: str, units: int, weights: str = "bf16",
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
-    key = f"{kernel}/{bound}" + ("/" + fp8_form(T) if weights == "fp8" else "")
+    key = f"{kernel}/{bound}" + ("/" + fp8_form(T) if weights == "fp8" else "") + \
+        ("/dense" if layer == "dense" else "")
     with open(path) as f:
         entry = json.load(f).get(key)
     if not entry or entry.get("bound") != bound:
@@ -423,7 +424,7 @@ def roofline(wl: Workload, work: dict, stage_mean: dict, peaks: dict) -> dict:
                 "peak_sustained": peaks["bf16_tflops_sustained"],
                 "frac_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4)}
     traffic = measured_traffic(dominant, roof["bound"], work["touched_experts"] + wl.S,
-                               wl.weights, wl.d, wl.F, wl.T)
+                               wl.weights, wl.d, wl.F, wl.T, wl.layer)
     roof.update({"kernel": dominant, "traffic": traffic, "peak_source": peaks["source"],
                  "algorithmic_per_launch": work[key + ("_bytes" if roof["bound"] == "hbm"
                                                        else "_flops")],

@@ -84,6 +84,9 @@ def test_measured_traffic_lookup_and_invalidation(tmp_path, monkeypatch):
     monkeypatch.setenv("MOE_GEMM_TILES", "swap")
     assert bench.measured_traffic("gate_up_gemm", "hbm", 10, "fp8", T=16) == 5200
     monkeypatch.delenv("MOE_GEMM_TILES")
+    # the dense layer has entries of its own (one expert of its width per launch)
+    assert bench.measured_traffic("gate_up_gemm", "hbm", 1, "bf16", 6144, 2048,
+                                  layer="dense") is None
     assert bench.measured_traffic("gate_up_gemm", "tensor", 10) is None   # no entry
     assert bench.measured_traffic("down_gemm", "hbm", 10) is None
     assert bench.measured_traffic("gate_up_gemm", "hbm", 1, "bf16", 6144, 18432) is None
