@@ -281,24 +281,27 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
         y = torch.empty_like(ihc[0])
         x_stage, y_stage = torch.empty_like(ihc[0]), torch.empty_like(ihc[0])
 
-    def forward(x_arg, y_arg, host=False):
+    def forward(x_arg, y_arg, host=False, lane=None):
+        # lane: (stream, workspace, iHC staging buffers) of an end-to-end step
+        st, w_s, stage = lane if lane is not None else (stream, ws, (x_stage, y_stage))
         if ihc is not None:   # the layer inside iHC streams; host streams copied around it
-            H_in, H_out = (x_stage, y_stage) if host else (x_arg, y_arg)
-            if host:
-                x_stage.copy_(x_arg, non_blocking=True)
-            moe.moe_forward_ihc(h, H_in, ihc[1], ihc[2], ihc[3], inp.W_router, inp.bias,
-                                *weights, H_out, ws, stream)
-            if host:
-                y_arg.copy_(y_stage, non_blocking=True)
+            H_in, H_out = stage if host else (x_arg, y_arg)
+            with torch.cuda.stream(st):
+                if host:
+                    H_in.copy_(x_arg, non_blocking=True)
+                moe.moe_forward_ihc(h, H_in, ihc[1], ihc[2], ihc[3], inp.W_router, inp.bias,
+                                    *weights, H_out, w_s, st)
+                if host:
+                    y_arg.copy_(H_out, non_blocking=True)
         elif dense:   # the dense FFN layer
             f = moe.moe_dense_ffn_host if host else moe.moe_dense_ffn
-            f(h, x_arg, inp.W_gate, inp.W_up, inp.W_down, y_arg, ws, stream)
+            f(h, x_arg, inp.W_gate, inp.W_up, inp.W_down, y_arg, w_s, st)
         elif fp8 is not None:
             f = moe.moe_forward_fp8_host if host else moe.moe_forward_fp8
-            f(h, x_arg, inp.W_router, inp.bias, fp8[0], fp8[1], y_arg, ws, stream)
+            f(h, x_arg, inp.W_router, inp.bias, fp8[0], fp8[1], y_arg, w_s, st)
         else:
             f = moe.moe_forward_host if host else moe.moe_forward
-            f(h, x_arg, inp.W_router, inp.bias, *weights, y_arg, ws, stream)
+            f(h, x_arg, inp.W_router, inp.bias, *weights, y_arg, w_s, st)
 
     def step():
         forward(inp.x, y)
@@ -349,21 +352,28 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
 
     # ---- end to end: every step copies its x in from pinned host memory and its y back
     # out, through the host-activation call.  The steps are enqueued back to back, as a
-    # serving loop issues them (a step's input copy may overlap the previous step's layer),
-    # and the whole run is timed on the host clock, synchronised on both sides.  Every step
-    # streams GBs of weights, far more than L2, so no flush separates them. ----
+    # serving loop issues them, on two streams in turn, each with its own workspace and
+    # host output buffer, so a step's output copy (on its own stream, after its layer)
+    # overlaps the next step's layer, and its input copy the previous step's.  The whole
+    # run is timed on the host clock, synchronised on both sides.  Every step streams GBs
+    # of weights, far more than L2, so no flush separates them. ----
     x_host = inp.x.cpu().pin_memory()
-    y_host = torch.empty(y.shape, dtype=torch.bfloat16).pin_memory()
-    for _ in range(max(1, args.warmup)):
-        forward(x_host, y_host, host=True)
+    lanes = [(stream, ws, (x_stage, y_stage)),
+             (torch.cuda.Stream(device), torch.empty_like(ws),
+              (torch.empty_like(x_stage), torch.empty_like(y_stage)) if ihc is not None
+              else (None, None))]
+    y_hosts = [torch.empty(y.shape, dtype=torch.bfloat16).pin_memory() for _ in lanes]
+    for i in range(max(2, args.warmup + (args.warmup & 1))):   # even: each lane keeps a slot
+        forward(x_host, y_hosts[i & 1], host=True, lane=lanes[i & 1])
     torch.cuda.synchronize(device)
     barrier(world)
     t0 = time.perf_counter()
     for i in range(args.steps):
-        forward(x_host, y_host, host=True)
+        forward(x_host, y_hosts[i & 1], host=True, lane=lanes[i & 1])
     torch.cuda.synchronize(device)
     e2e_ms = [(time.perf_counter() - t0) * 1e3 / args.steps] * args.steps
     barrier(world)
+    del lanes
 
     raw = {"step_ms": step_ms, "stage_ms": stage_ms.mean(0).tolist(), "e2e_ms": e2e_ms,
            "counts": counts, "clocks": clocks.summary(),
@@ -371,12 +381,13 @@ def time_workload(wl: Workload, args, rank: int, world: int, device, cpu_seconds
                                 else moe.moe_forward_kernel_count(h, wl.T)
                                 + (1 if ihc is not None else 0)),   # + the iHC mix
            "h2d_bytes": int(x_host.numel() * x_host.element_size()),
-           "d2h_bytes": int(y_host.numel() * y_host.element_size()), "fp8": fp8 is not None}
+           "d2h_bytes": int(y_hosts[0].numel() * y_hosts[0].element_size()),
+           "fp8": fp8 is not None}
     if rank == 0 and world == 1 and cpu_seconds > 0 and ihc is None:
         raw["cpu_baseline"] = cpu_baseline(inp, cpu_seconds, fp8, cpu_tokens)
     if hbm_bound(wl, algorithmic_work(wl, counts), load_peaks()):
         raw["read_only_gbs"] = read_only_peak(device)
-    del inp, fp8, weights, ws, y, flush, x_host, y_host, x_stage, y_stage, ihc
+    del inp, fp8, weights, ws, y, flush, x_host, y_hosts, x_stage, y_stage, ihc
     moe.moe_destroy(h)
     torch.cuda.synchronize(device)
     torch.cuda.empty_cache()
@@ -450,7 +461,8 @@ def e2e_api(wl: Workload, fp8: bool) -> str:
     else:
         api = ("moe_forward_fp8_host" if fp8 else "moe_forward_host") + \
             " (pinned host x in, host y out)"
-    return api + "; steps enqueued back to back"
+    return api + ("; steps enqueued back to back on two streams in turn, each with its own "
+                  "workspace (a step's output copy overlaps the next step's layer)")
 
 
 def report_workload(wl: Workload, raw: dict, args, world: int, device, stage_names) -> dict:

@@ -207,7 +207,9 @@ moe_status moe_forward(moe_handle h, const uint16_t *x, const float *W_router, c
  * x_host must therefore stay unchanged from the call until the stream has
  * passed it.  Host buffers should be page-locked for the copies to be
  * asynchronous.  Weights and the workspace are device memory as in
- * moe_forward.
+ * moe_forward.  Calls may run on several streams at once when each stream has
+ * its own workspace and output buffer: a serving loop that alternates two
+ * streams lets one call's output copy overlap the next call's layer.
  */
 moe_status moe_forward_host(moe_handle h, const uint16_t *x_host, const float *W_router,
                             const float *bias, const uint16_t *W_gate, const uint16_t *W_up,
