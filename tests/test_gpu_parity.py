@@ -356,3 +356,36 @@ def test_back_to_back_host_calls_keep_each_input():
         torch.cuda.synchronize()
         assert torch.equal(ref.cpu().view(torch.int16), y.view(torch.int16))
     assert moe.moe_device_status(h, wl.T, ws)[0] == moe.MOE_OK
+
+
+def test_host_calls_on_two_streams_each_with_its_own_workspace():
+    """moe_forward_host calls alternating two streams, each with its own workspace and output
+    buffer, enqueued without synchronising (as a serving loop that overlaps one call's output
+    copy with the next call's layer): the calls may run at once, and every output must still
+    equal moe_forward's on its own input."""
+    wl_inp = make_small(160, 256, 16, 2, 128, 1, seed=67)
+    dev = to_device(wl_inp, "cuda")
+    wl = wl_inp.wl
+    h = moe.moe_create(wl.d, wl.E, wl.k, wl.F, wl.S)
+    size = moe.moe_workspace_size(h, wl.T)
+    lanes = [(torch.cuda.current_stream(), torch.empty(size, dtype=torch.uint8, device="cuda")),
+             (torch.cuda.Stream(), torch.empty(size, dtype=torch.uint8, device="cuda"))]
+    W = (dev.W_gate, dev.W_up, dev.W_down, dev.Ws_gate, dev.Ws_up, dev.Ws_down)
+    g = torch.Generator().manual_seed(9)
+    xs = [torch.randn(wl.T, wl.d, generator=g).to(torch.bfloat16).pin_memory() for _ in range(7)]
+    ys = [torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory() for _ in range(7)]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(lanes[0][0]):
+        torch.cuda._sleep(20_000_000)                # the first stream starts late
+    for i, (x, y) in enumerate(zip(xs, ys)):
+        st, ws = lanes[i & 1]
+        moe.moe_forward_host(h, x, dev.W_router, dev.bias, *W, y, ws, st)
+    torch.cuda.synchronize()
+    ws = lanes[0][1]
+    for x, y in zip(xs, ys):
+        ref = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda")
+        moe.moe_forward(h, x.cuda(), dev.W_router, dev.bias, *W, ref, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(ref.cpu().view(torch.int16), y.view(torch.int16))
+    for _, ws in lanes:
+        assert moe.moe_device_status(h, wl.T, ws)[0] == moe.MOE_OK
