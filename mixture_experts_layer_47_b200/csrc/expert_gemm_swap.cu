@@ -105,6 +105,9 @@ struct __align__(64) SwapParams {
   int out_rows;            // rows of the output buffer (T*k + S*T)
   int ksplit;              // down, 1-SM only: K ranges per output tile (1 = no split)
   float* part;             // with ksplit > 1: fp32 parts [ksplit][out_rows][n_out]
+  unsigned int* split_count;  // with ksplit > 1: zeroed counters, one per output tile and
+                              // epilogue warp, or null (a separate kernel adds the parts)
+  int dense_T;             // > 0: one group of dense_T rows (E = 1, S = 0), schedule built here
   // Fused combine (down, bf16 Y rows): after all tiles and a grid-wide barrier,
   //   y[t] = sum_s Y[T*k + s*T + t] + sum_i topk_w[t][i] * Y[pos[t*k + i]]
   int fuse_combine;
@@ -259,6 +262,51 @@ __device__ __forceinline__ void fused_combine(const SwapParams& p, int& all_done
   }
 }
 
+// The down projection split over K (1-SM tiling).  Epilogue warp w of every K range's CTA
+// stores the same share of the output tile's fp32 part (its 32-token chunks of its TMEM lane
+// quarter's features in both 128-row halves) and then arrives on that share's counter; the
+// warp that arrives last (the ksplit-th) adds the ranges' parts of the share in range order
+// and rounds once to bf16 -- the sum a separate kernel would form, in its order.  No barrier
+// is involved, so a warp that gives up on a fault leaves its share unsummed and nothing
+// waiting.  The parts of other CTAs are read through L2 (__ldcg).
+__device__ __forceinline__ void split_sum(const SwapParams& p, const wm::Tile& tl, int ot,
+                                          int ksplit, int quarter, int sub, int lane) {
+  __threadfence();   // this lane's part stores, before the warp's arrival
+  __syncwarp();
+  unsigned last = 0;
+  if (lane == 0)
+    last = atomicAdd(p.split_count + size_t(ot) * EPI_WARPS + (sub * 4 + quarter), 1u) ==
+                   unsigned(ksplit - 1)
+               ? 1u
+               : 0u;
+  if (!__shfl_sync(0xffffffffu, last, 0)) return;
+  __threadfence();
+  const size_t plane = size_t(p.out_rows) * p.n_out;
+  // items: (row of a chunk, half, 8 features); 32 rows x 2 halves x 4 pieces per chunk
+  for (int c = 32 * sub; c < tl.cnt; c += 64) {
+    const int rows = min(32, tl.cnt - c);
+    for (int i = lane; i < rows * 8; i += 32) {
+      const int row = tl.out_row + c + (i >> 3);
+      const int col = tl.f0 + ((i >> 2) & 1) * 128 + quarter * 32 + (i & 3) * 8;
+      if (col >= p.n_out || row >= p.out_rows) continue;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const float* src = p.part + size_t(row) * p.n_out + col;
+      for (int r = 0; r < ksplit; ++r) {
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(src + r * plane));
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(src + r * plane + 4));
+        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+      }
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + size_t(row) * p.n_out + col) = o;
+    }
+  }
+}
+
 template <bool kGateUp, bool kPair>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_swap_kernel(const __grid_constant__ SwapParams p) {
@@ -313,8 +361,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // With the fused combine every CTA waits for all the others, so the next kernel may not
   // take an SM before all of them are resident: its launch is released after the barrier.
   if (kGateUp || !p.fuse_combine) pdl_launch_dependents();
-  for (int i = threadIdx.x; i <= G; i += NUM_THREADS) ss.sched[i] = p.sched[i];
-  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) ss.offsets[i] = p.offsets[i];
+  if (p.dense_T > 0) {   // one group of dense_T rows in token tiles of at most TN
+    if (threadIdx.x == 0) {
+      ss.sched[0] = 0;
+      ss.sched[1] = (p.dense_T + C::TN - 1) / C::TN;
+      ss.offsets[0] = 0;
+      ss.offsets[1] = p.dense_T;
+    }
+  } else {
+    for (int i = threadIdx.x; i <= G; i += NUM_THREADS) ss.sched[i] = p.sched[i];
+    for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) ss.offsets[i] = p.offsets[i];
+  }
   tc_fence_before();
   if (kPair) cluster_sync_all(); else __syncthreads();   // barriers of both CTAs initialised
   tc_fence_after();
@@ -621,6 +678,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         else
           mbar_arrive(&ss.tmem_empty[acc]);
       }
+      if (!kPair && ksplit > 1 && p.split_count)
+        split_sum(p, tl, t / ksplit, ksplit, quarter, sub, lane);
       if (++acc == C::NUM_ACC) {
         acc = 0;
         acc_phase ^= 1;
@@ -742,6 +801,7 @@ moe_status launch_expert_ffn_swap(const Ctx& c, const FfnArgs& a, const DeviceIn
   if (!ok) return MOE_ERR_CUDA;
   gp.offsets = a.offsets;
   gp.sched = sched;
+  gp.dense_T = a.dense_T;
   gp.out = a.h_act;
   gp.status = a.status;
   gp.T = T;
@@ -772,6 +832,7 @@ moe_status launch_expert_ffn_swap(const Ctx& c, const FfnArgs& a, const DeviceIn
   dp.s1 = dp.s0;
   dp.offsets = a.offsets;
   dp.sched = sched;
+  dp.dense_T = a.dense_T;
   dp.out = a.Y;
   dp.out_bf16 = a.y_bf16 ? 1 : 0;
   dp.status = a.status;
@@ -786,6 +847,7 @@ moe_status launch_expert_ffn_swap(const Ctx& c, const FfnArgs& a, const DeviceIn
   const bool split = !pair && a.down_ksplit > 1 && a.down_part && a.y_bf16;
   dp.ksplit = split ? a.down_ksplit : 1;
   dp.part = split ? a.down_part : nullptr;
+  dp.split_count = split ? a.split_count : nullptr;
   if (a.fuse_combine && a.y_bf16 && !split) {   // grid_count was zeroed with the status word
     dp.fuse_combine = 1;
     dp.topk_w = a.topk_w;
@@ -796,7 +858,7 @@ moe_status launch_expert_ffn_swap(const Ctx& c, const FfnArgs& a, const DeviceIn
   err = pair ? launch_swap<false, true>(dp, dev.num_sms, st)
              : launch_swap<false, false>(dp, dev.num_sms, st);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
-  if (split) {   // y = bf16(sum of the K ranges' parts, in range order)
+  if (split && !a.split_count) {   // y = bf16(sum of the K ranges' parts, in range order)
     PartialPtrs parts = {};
     for (int j = 0; j < dp.ksplit; ++j) parts.p[j] = a.down_part + size_t(j) * rows * c.d;
     if (launch_reduce_partials(parts, dp.ksplit, size_t(rows) * c.d,

@@ -169,6 +169,12 @@ struct FfnArgs {
   // [down_ksplit][rows][d] in the workspace, added in order into Y.
   int down_ksplit = 1;
   float* down_part = nullptr;
+  // With split_count (zeroed, one counter per output tile) the down GEMM adds the parts
+  // itself: the last K range to finish an output tile sums them, in range order.
+  unsigned int* split_count = nullptr;
+  // The dense layer: one group of dense_T rows and no shared group; the weight-major GEMMs
+  // build that schedule themselves (offsets and sched are then not read).
+  int dense_T = 0;
   // The combine fused into the down GEMM (weight-major tilings, bf16 Y rows): the down
   // kernel writes y itself after a grid-wide barrier on grid_count (workspace).
   bool fuse_combine = false;

@@ -88,7 +88,7 @@ Layout make_layout(const Ctx& c, int T, int num_sms) {
     off = align_up(off + std::max<size_t>(bytes, 16), kWsAlign);
     return o;
   };
-  L.status = take(256);
+  L.status = take(2048);   // status word, grid counter, and the dense K split's counters
   L.part = take(size_t(L.rplan.ksplit) * T * c.E * sizeof(float));
   L.wparts = take(L.rplan.tc ? 3 * size_t(c.E) * c.d * sizeof(uint16_t) : 0);
   L.topk_idx = take(nslots * sizeof(int32_t));
@@ -692,6 +692,20 @@ static moe_status check_dense_args(moe_handle h, const uint16_t* x, const uint16
 }
 
 // The dense layer on device activations: the checks are done.
+// The dense layer on the weight-major tilings: the GEMMs build the one-group schedule
+// themselves, and the down GEMM's K ranges add their parts in the kernel when the counters
+// (one per output tile and epilogue warp) fit the status block's last kilobyte.
+static bool dense_weight_major(const Ctx& c, int T) {
+  const GemmTiling t = gemm_tiling(c, T);
+  return t == GemmTiling::kSwap || t == GemmTiling::kSwapPair;
+}
+constexpr size_t kSplitCountOffset = 1024;   // inside the 2 KB status block
+constexpr int kMaxSplitCounters = 256;
+static bool dense_split_summed_in_gemm(const Ctx& c, int T) {
+  return dense_down_ksplit(c, T) > 1 &&
+         ((T + 127) / 128) * ((c.d + 255) / 256) * 8 <= kMaxSplitCounters;
+}
+
 static moe_status dense_device(moe_handle h, const uint16_t* x, const uint16_t* W_gate,
                                const uint16_t* W_up, const uint16_t* W_down, int T, uint16_t* y,
                                uint8_t* ws, const Layout& L, const DeviceInfo* dev,
@@ -705,10 +719,13 @@ static moe_status dense_device(moe_handle h, const uint16_t* x, const uint16_t* 
   auto mark = [&](int i) -> moe_status {
     return prof ? cuda_status(cudaEventRecord(h->stage_events[i], st)) : MOE_OK;
   };
-  if ((s = cuda_status(cudaMemsetAsync(status, 0, sizeof(int), st)))) return s;
+  const bool wm = dense_weight_major(c, T);
+  const bool split_in_gemm = wm && dense_split_summed_in_gemm(c, T);
+  // the status word and the down GEMM's K-split counters (same 2 KB block)
+  if ((s = cuda_status(cudaMemsetAsync(status, 0, 2048, st)))) return s;
   if ((s = mark(0))) return s;
   if ((s = mark(1))) return s;   // no router
-  if ((s = cuda_status(launch_dense_schedule(T, offsets, sched, st)))) return s;
+  if (!wm && (s = cuda_status(launch_dense_schedule(T, offsets, sched, st)))) return s;
   if ((s = mark(2))) return s;   // the one-group schedule in place of dispatch
   if ((s = mark(3))) return s;   // no gather
   // One group holding every token in order: the GEMMs read x itself as the group's rows and
@@ -727,6 +744,9 @@ static moe_status dense_device(moe_handle h, const uint16_t* x, const uint16_t* 
   a.after_gate_up = prof ? h->stage_events[4] : nullptr;
   a.down_ksplit = dense_down_ksplit(c, T);
   a.down_part = reinterpret_cast<float*>(ws + L.down_part);
+  a.dense_T = wm ? T : 0;
+  a.split_count =
+      split_in_gemm ? reinterpret_cast<unsigned int*>(ws + L.status + kSplitCountOffset) : nullptr;
   if ((s = launch_expert_ffn(c, a, *dev, st))) return s;
   if ((s = mark(5))) return s;
   return mark(6);   // no combine
@@ -867,7 +887,9 @@ int moe_dense_ffn_kernel_count(moe_handle h, int T) {
   const Ctx& c = h->c;
   if (c.E != 1 || c.k != 1 || c.S != 0) return -1;
   if (T == 0) return 0;
-  return 3 + (dense_down_ksplit(c, T) > 1 ? 1 : 0);   // schedule, GEMMs [, K-range sum]
+  if (!dense_weight_major(c, T)) return 3;   // schedule, GEMMs
+  // the GEMMs [, the K ranges' sum when the kernel cannot add them itself]
+  return 2 + (dense_down_ksplit(c, T) > 1 && !dense_split_summed_in_gemm(c, T) ? 1 : 0);
 }
 
 moe_status moe_set_stage_events(moe_handle h, void* const* events, int n_events) {

@@ -280,9 +280,14 @@ def test_shard_and_dense_entry_points_validate_on_the_host(lib):
         moe.MOE_ERR_INVALID_ARG
     assert L.moe_dense_ffn_host(hd.value, None, None, None, None, 0, None, None, 0, None) == \
         moe.MOE_OK
-    # up to 128 tokens the down projection is split over K (one launch more)
-    assert L.moe_dense_ffn_kernel_count(hd.value, 16) == 4
-    assert L.moe_dense_ffn_kernel_count(hd.value, 4096) == 3
+    # the weight-major GEMMs build the one-group schedule, and the K ranges of the split down
+    # projection (up to 128 tokens) add their parts in the kernel while the output tiles'
+    # counters fit (32): two launches; wider layers take the separate sum (three)
+    assert L.moe_dense_ffn_kernel_count(hd.value, 16) == 2
+    assert L.moe_dense_ffn_kernel_count(hd.value, 4096) == 2
+    hw = moe.moe_create(8448, 1, 1, 640, 0)
+    assert L.moe_dense_ffn_kernel_count(hw.value, 16) == 3
+    assert L.moe_dense_ffn_kernel_count(hw.value, 4096) == 2
 
 
 def test_fused_combine_option_is_fixed_at_create(lib, monkeypatch):
