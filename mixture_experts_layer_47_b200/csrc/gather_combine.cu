@@ -104,23 +104,35 @@ __global__ void __launch_bounds__(kGatherThreads)
   }
 }
 
+// Eight consecutive values of a row: loaded raw (Raw), then widened to fp32.
 struct RowF32 {
-  __device__ static void load8(const float* __restrict__ row, float (&v)[8]) {
-    const float4 a = *reinterpret_cast<const float4*>(row);
-    const float4 b = *reinterpret_cast<const float4*>(row + 4);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  struct Raw {
+    float4 a, b;
+  };
+  __device__ static Raw load(const float* __restrict__ row) {
+    return {*reinterpret_cast<const float4*>(row), *reinterpret_cast<const float4*>(row + 4)};
   }
+  __device__ static void widen(const Raw& r, float (&v)[8]) {
+    v[0] = r.a.x; v[1] = r.a.y; v[2] = r.a.z; v[3] = r.a.w;
+    v[4] = r.b.x; v[5] = r.b.y; v[6] = r.b.z; v[7] = r.b.w;
+  }
+  __device__ static void load8(const float* __restrict__ row, float (&v)[8]) { widen(load(row), v); }
 };
 struct RowBF16 {
-  __device__ static void load8(const uint16_t* __restrict__ row, float (&v)[8]) {
-    const uint4 a = *reinterpret_cast<const uint4*>(row);
+  using Raw = uint4;
+  __device__ static Raw load(const uint16_t* __restrict__ row) {
+    return *reinterpret_cast<const uint4*>(row);
+  }
+  __device__ static void widen(const Raw& a, float (&v)[8]) {
     const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       v[2 * q] = bf16_bits_to_float(w[q] & 0xFFFFu);
       v[2 * q + 1] = bf16_bits_to_float(w[q] >> 16);
     }
+  }
+  __device__ static void load8(const uint16_t* __restrict__ row, float (&v)[8]) {
+    widen(load(row), v);
   }
 };
 
@@ -154,13 +166,28 @@ __device__ __forceinline__ void combine_sum8(const TY* __restrict__ Y,
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] += v[j];
   }
-  for (int i = 0; i < k; ++i) {
-    const int p = pos[size_t(t) * k + i];
-    if (p < 0 || size_t(p) >= nslots) continue;
-    const float w = topk_w[size_t(t) * k + i];
-    Row::load8(Y + size_t(p) * d + c, v);
+  // The routed rows kChunk at a time: every load of a chunk is issued before its rows are
+  // added (in slot order), so a thread keeps several rows in flight.
+  constexpr int kChunk = 4;
+  for (int i0 = 0; i0 < k; i0 += kChunk) {
+    typename Row::Raw r[kChunk];
+    float w[kChunk];
+    bool live[kChunk];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = fmaf(w, v[j], acc[j]);
+    for (int j = 0; j < kChunk; ++j) {
+      const int i = i0 + j;
+      const int p = i < k ? pos[size_t(t) * k + i] : -1;
+      live[j] = p >= 0 && size_t(p) < nslots;
+      w[j] = live[j] ? topk_w[size_t(t) * k + i] : 0.f;
+      if (live[j]) r[j] = Row::load(Y + size_t(p) * d + c);
+    }
+#pragma unroll
+    for (int j = 0; j < kChunk; ++j) {
+      if (!live[j]) continue;
+      Row::widen(r[j], v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(w[j], v[e], acc[e]);
+    }
   }
 }
 
