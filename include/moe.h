@@ -384,7 +384,9 @@ moe_status moe_forward_ihc(moe_handle h, const uint16_t *H, int n_streams, const
  * output rows once from the fp32 accumulator.  At up to 128 tokens the down
  * projection's K is split into ranges whose fp32 parts are added in range
  * order (deterministic) before that rounding, so that enough SMs stream the
- * weights.
+ * weights; the down GEMM adds them itself (d up to 8192), or a separate kernel
+ * does.  The workspace's status block (its first 2 KB) holds the counters of
+ * that sum and is cleared by every call.
  */
 moe_status moe_dense_ffn(moe_handle h, const uint16_t *x, const uint16_t *W_gate,
                          const uint16_t *W_up, const uint16_t *W_down, int T, uint16_t *y,
@@ -418,8 +420,9 @@ moe_status moe_device_status(moe_handle h, int T, const void *workspace, void *s
  * its stream at the stage boundaries: before the router, after the router,
  * after dispatch, after the gather, after the gate/up GEMM, after the down
  * GEMM, after the combine.  The elapsed time between consecutive events is
- * then the device time of one stage (moe_dense_ffn: its one-group schedule
- * counts as dispatch; router, gather and combine are empty).  events == NULL
+ * then the device time of one stage (moe_dense_ffn: its one-group schedule,
+ * where a kernel builds it, counts as dispatch; router, gather and combine
+ * are empty).  events == NULL
  * (n_events == 0) switches it off.  The
  * context keeps the handles only; the caller keeps the events alive.
  */
